@@ -1,0 +1,168 @@
+"""FP8 (E4M3) quantisation and the FP8 MoE forward -- TEST INFRASTRUCTURE ONLY.
+
+Follows [MegaMoE] ("MegaMoE math model -> DeepGEMM source walk-through",
+2kiu.com news 6052262) §2.3 and §5.1: E4M3 for the forward pass, one scale
+per token per 128-element group of activations (1x128) and one per 128x128
+block of weights, fp32 accumulation, and the scaled product
+C ~ (A_q / scale_A)(B_q / scale_B) scale_C.
+
+Readings (the pages leave these open):
+  * a scale s is stored as the DEQUANTISING multiplier (a ~ q * s), i.e. the
+    page's scale_A is 1/s and scale_C = 1;
+  * s = fp32(amax / 448) with IEEE float32 division (s = 1 when amax = 0),
+    q = E4M3(fp32(a / s)) with IEEE float32 division, E4M3 rounding to
+    nearest even with saturation to +-448 (OCP 8-bit floating point:
+    bias 7, no infinities, code 0x7F/0xFF = NaN, subnormals down to 2^-9);
+  * the scales vary along K, so the product is promoted per 128-wide K
+    block: C = sum_kb (sum_{k in kb} qa qb) * sa[m, kb] * sb[n/128, kb];
+  * the intermediate h = silu(gate) * up is rounded to fp32 and quantised per
+    row per 128 columns before the down projection;
+  * the router stays in bf16; the shared expert runs in FP8 like the others.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+from .moe_oracle import as_f64, bf16_round, route
+
+__all__ = [
+    "E4M3_MAX", "e4m3_magnitudes", "e4m3_decode", "e4m3_encode", "quantize_1x128",
+    "quantize_128x128", "dequantize_1x128", "dequantize_128x128", "fp8_gemm",
+    "swiglu_ffn_fp8", "moe_forward_fp8",
+]
+
+E4M3_MAX = 448.0
+
+
+def e4m3_magnitudes() -> np.ndarray:
+    """Values of the non-negative finite codes 0x00..0x7E, ascending with the code."""
+    vals = np.empty(127, dtype=np.float64)
+    for code in range(127):
+        e, m = code >> 3, code & 7
+        vals[code] = (m / 8.0) * 2.0 ** -6 if e == 0 else (1.0 + m / 8.0) * 2.0 ** (e - 7)
+    return vals
+
+
+_MAGS = e4m3_magnitudes()
+
+
+def e4m3_decode(codes) -> np.ndarray:
+    """uint8 E4M3 codes -> float64 (0x7F / 0xFF decode to NaN)."""
+    c = np.asarray(codes, dtype=np.uint8)
+    mag = c & 0x7F
+    v = np.where(mag == 0x7F, np.nan, _MAGS[np.minimum(mag, 126)])
+    return np.where(c & 0x80, -v, v)
+
+
+def e4m3_encode(v) -> np.ndarray:
+    """float32 values -> E4M3 codes, round to nearest (ties to even code), saturating.
+
+    The sign bit is kept, so a negative value that rounds to zero gives 0x80.
+    Inputs must be finite.
+    """
+    v = np.asarray(v, dtype=np.float32)
+    a = np.abs(v).astype(np.float64)
+    hi = np.clip(np.searchsorted(_MAGS, a, side="left"), 1, 126)
+    lo = hi - 1
+    dlo = a - _MAGS[lo]
+    dhi = _MAGS[hi] - a
+    code = np.where(dlo < dhi, lo, np.where(dhi < dlo, hi, np.where(lo % 2 == 0, lo, hi)))
+    code = np.where(a >= E4M3_MAX, 126, code).astype(np.uint8)
+    return np.where(np.signbit(v), code | 0x80, code).astype(np.uint8)
+
+
+def _scale_of(amax32: np.ndarray) -> np.ndarray:
+    s = (amax32.astype(np.float32) / np.float32(E4M3_MAX)).astype(np.float32)
+    return np.where(amax32 == 0, np.float32(1.0), s).astype(np.float32)
+
+
+def quantize_1x128(a) -> tuple[np.ndarray, np.ndarray]:
+    """Per row, per 128-column group: (codes [M, K], scales [M, K/128] fp32)."""
+    a = np.asarray(a, dtype=np.float32)
+    M, K = a.shape
+    if K % 128:
+        raise ValueError("K must be a multiple of 128")
+    g = a.reshape(M, K // 128, 128)
+    s = _scale_of(np.abs(g).max(axis=2))
+    q = e4m3_encode((g / s[:, :, None]).astype(np.float32))
+    return q.reshape(M, K), s
+
+
+def quantize_128x128(W) -> tuple[np.ndarray, np.ndarray]:
+    """Per 128x128 block: (codes [N, K], scales [N/128, K/128] fp32)."""
+    W = np.asarray(W, dtype=np.float32)
+    N, K = W.shape
+    if N % 128 or K % 128:
+        raise ValueError("N and K must be multiples of 128")
+    b = W.reshape(N // 128, 128, K // 128, 128)
+    s = _scale_of(np.abs(b).max(axis=(1, 3)))
+    q = e4m3_encode((b / s[:, None, :, None]).astype(np.float32))
+    return q.reshape(N, K), s
+
+
+def dequantize_1x128(q, s) -> np.ndarray:
+    M, K = q.shape
+    return (e4m3_decode(q).reshape(M, K // 128, 128) * as_f64(s)[:, :, None]).reshape(M, K)
+
+
+def dequantize_128x128(q, s) -> np.ndarray:
+    N, K = q.shape
+    d = e4m3_decode(q).reshape(N // 128, 128, K // 128, 128) * as_f64(s)[:, None, :, None]
+    return d.reshape(N, K)
+
+
+def fp8_gemm(qa, sa, qb, sb) -> np.ndarray:
+    """C[m, n] = sum_kb (sum_{k in kb} qa[m,k] qb[n,k]) * sa[m,kb] * sb[n//128, kb] (fp64)."""
+    A = e4m3_decode(qa)
+    B = e4m3_decode(qb)
+    sa = as_f64(sa)
+    sb = as_f64(sb)
+    M, K = A.shape
+    N = B.shape[0]
+    C = np.zeros((M, N), dtype=np.float64)
+    for kb in range(K // 128):
+        ks = slice(128 * kb, 128 * kb + 128)
+        partial = A[:, ks] @ B[:, ks].T
+        C += partial * sa[:, kb][:, None] * np.repeat(sb[:, kb], 128)[None, :]
+    return C
+
+
+def swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2) -> dict:
+    """SiLU-gated FFN on quantised operands; h is re-quantised 1x128."""
+    I = W1q.shape[0] // 2
+    gu = fp8_gemm(xq, sx, W1q, s1)
+    g, u = gu[:, :I], gu[:, I:]
+    h = g / (1.0 + np.exp(-g)) * u
+    hq, sh = quantize_1x128(h.astype(np.float32))
+    return dict(h=h, hq=hq, sh=sh, y=fp8_gemm(hq, sh, W2q, s2))
+
+
+def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
+                    renormalize: bool = False, tokens=None, idx=None, w=None) -> dict:
+    """FP8 variant of oracle.moe_forward: same routing, quantised expert GEMMs.
+
+    Each expert's W1[e] / W2[e] (bf16 values) is quantised per 128x128 block;
+    x (as bf16) per token per 128 columns.
+    """
+    xs = x if tokens is None else x[tokens]
+    r = route(xs, W_r, bias, k, renormalize)
+    if idx is not None:
+        from .moe_oracle import gate_weights
+        r["idx"] = np.asarray(idx)
+        r["w"] = as_f64(w) if w is not None else gate_weights(r["p"], r["idx"], renormalize)
+    sel, wts = r["idx"], r["w"]
+    xe = bf16_round(as_f64(xs)).astype(np.float32)
+    xq, sx = quantize_1x128(xe)
+    out = np.zeros(xe.shape, dtype=np.float64)
+    if W1s is not None:
+        W1q, s1 = quantize_128x128(as_f64(W1s))
+        W2q, s2 = quantize_128x128(as_f64(W2s))
+        out += swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)["y"]
+    for e in np.unique(sel):
+        t_rows, slots = np.nonzero(sel == e)
+        W1q, s1 = quantize_128x128(as_f64(W1[int(e)]))
+        W2q, s2 = quantize_128x128(as_f64(W2[int(e)]))
+        y = swiglu_ffn_fp8(xq[t_rows], sx[t_rows], W1q, s1, W2q, s2)["y"]
+        out[t_rows] += wts[t_rows, slots][:, None] * y
+    r.update(out=out, xq=xq, sx=sx)
+    return r

@@ -1,0 +1,150 @@
+"""Pins of the oracle's E4M3 quantisation and blockwise-scaled GEMM.
+
+  * every finite E4M3 code decodes and re-encodes to itself, both signs;
+  * the encoder agrees with torch's float8_e4m3fn conversion (a library
+    routine) on random in-range values, subnormals and exact midpoints;
+  * midpoints round to the even code; values beyond 448 saturate to 448;
+  * the largest element of each group quantises to +-448 * s exactly;
+  * with every group's amax equal to 448 and values on the E4M3 grid the
+    scales are 1 and the FP8 GEMM equals the exact matmul;
+  * the blockwise-promoted GEMM equals a matmul of the dequantised operands
+    (a different association of the same sum), which catches a wrong scale
+    index or a transposed block;
+  * the FP8 forward with identical experts follows the same closed form as
+    the bf16 one within quantisation error.
+(MegaMoE walk-through §2.3 and §5.1: per-token / per-block scales, E4M3 forward.)
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import fp8
+
+
+def test_codes_round_trip():
+    codes = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)
+    vals = fp8.e4m3_decode(codes)
+    assert np.array_equal(fp8.e4m3_encode(vals.astype(np.float32)), codes)
+    assert fp8.e4m3_decode(np.array([0x7E]))[0] == 448.0
+    assert fp8.e4m3_decode(np.array([0x01]))[0] == 2.0 ** -9
+    assert fp8.e4m3_decode(np.array([0x38]))[0] == 1.0
+    assert np.isnan(fp8.e4m3_decode(np.array([0x7F, 0xFF]))).all()
+
+
+def _torch_codes(v):
+    return torch.from_numpy(np.asarray(v, dtype=np.float32)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def test_encoder_matches_torch_in_range():
+    rng = np.random.default_rng(0)
+    v = np.concatenate([
+        rng.normal(size=20000) * 40,
+        rng.uniform(-2 ** -6, 2 ** -6, size=5000),            # subnormal range
+        rng.uniform(-448, 448, size=5000),
+    ]).astype(np.float32)
+    mags = fp8.e4m3_magnitudes()
+    mids = ((mags[:-1] + mags[1:]) / 2).astype(np.float32)   # exact midpoints
+    v = np.concatenate([v, mids, -mids, np.float32([0.0, -0.0, 448.0, -448.0])])
+    v = v[np.abs(v) <= 448]
+    assert np.array_equal(fp8.e4m3_encode(v), _torch_codes(v))
+
+
+def test_midpoints_go_to_even_code_and_saturation():
+    mags = fp8.e4m3_magnitudes()
+    for c in range(126):
+        mid = np.float32((mags[c] + mags[c + 1]) / 2)
+        if float(mid) != (mags[c] + mags[c + 1]) / 2:
+            continue
+        code = int(fp8.e4m3_encode(mid))
+        assert code % 2 == 0 and code in (c, c + 1)
+    big = np.float32([449.0, 463.9, 464.0, 1e6, -500.0, -3.0e38])
+    assert fp8.e4m3_encode(big).tolist() == [0x7E] * 4 + [0xFE] * 2
+    assert int(fp8.e4m3_encode(np.float32(-1e-9))) == 0x80   # signed zero
+
+
+def test_group_max_maps_to_448():
+    rng = np.random.default_rng(1)
+    a = (rng.normal(size=(8, 512)) * rng.uniform(1e-3, 1e3, size=(8, 1))).astype(np.float32)
+    q, s = fp8.quantize_1x128(a)
+    assert s.shape == (8, 4) and s.dtype == np.float32
+    deq = fp8.e4m3_decode(q)
+    for m in range(8):
+        for g in range(4):
+            blk = a[m, 128 * g:128 * g + 128]
+            j = int(np.argmax(np.abs(blk)))
+            assert abs(deq[m, 128 * g + j]) == 448.0
+            assert s[m, g] == np.float32(np.abs(blk).max()) / np.float32(448.0)
+    z, sz = fp8.quantize_1x128(np.zeros((2, 128), np.float32))
+    assert np.all(z == 0) and np.all(sz == 1.0)
+
+
+def test_dequantised_error_within_half_ulp():
+    rng = np.random.default_rng(2)
+    a = rng.normal(size=(16, 256)).astype(np.float32)
+    q, s = fp8.quantize_1x128(a)
+    d = fp8.dequantize_1x128(q, s)
+    # relative spacing of E4M3 normals is 2^-3; half of it bounds the error, plus the subnormal floor
+    bound = np.maximum(np.abs(a) * 2.0 ** -4, np.repeat(s, 128, axis=1) * 2.0 ** -10) * (1 + 1e-6)
+    assert np.all(np.abs(d - a) <= bound)
+
+
+def _grid_operand(rng, rows, K):
+    codes = rng.integers(0, 126, size=(rows, K)).astype(np.uint8) | (rng.integers(0, 2, size=(rows, K)) * 0x80).astype(np.uint8)
+    v = fp8.e4m3_decode(codes)
+    return v
+
+
+def test_unit_scales_give_exact_matmul():
+    rng = np.random.default_rng(3)
+    A = _grid_operand(rng, 8, 256)
+    B = _grid_operand(rng, 128, 256)
+    for g in range(2):   # force every 1x128 group and 128x128 block amax to 448
+        A[:, 128 * g] = 448.0
+        B[0, 128 * g:128 * g + 128] = 448.0
+    qa, sa = fp8.quantize_1x128(A.astype(np.float32))
+    qb, sb = fp8.quantize_128x128(B.astype(np.float32))
+    assert np.all(sa == 1.0) and np.all(sb == 1.0)
+    assert np.array_equal(fp8.e4m3_decode(qa), A)
+    assert np.array_equal(fp8.fp8_gemm(qa, sa, qb, sb), A @ B.T)
+
+
+def test_blockwise_promotion_equals_dequantised_matmul():
+    rng = np.random.default_rng(4)
+    A = (rng.normal(size=(24, 384)) * rng.uniform(0.1, 10, size=(24, 1))).astype(np.float32)
+    B = (rng.normal(size=(256, 384)) * 0.02).astype(np.float32)
+    B[128:] *= 50.0   # second row-block has a very different scale
+    qa, sa = fp8.quantize_1x128(A)
+    qb, sb = fp8.quantize_128x128(B)
+    C = fp8.fp8_gemm(qa, sa, qb, sb)
+    ref = fp8.dequantize_1x128(qa, sa) @ fp8.dequantize_128x128(qb, sb).T
+    assert np.allclose(C, ref, rtol=1e-12, atol=1e-12 * np.abs(ref).max())
+    # and it approximates the unquantised product to FP8 accuracy: each operand carries a
+    # relative rounding error of at most 2^-4 (RMS ~2.5%), so the product lands within ~5%
+    exact = A.astype(np.float64) @ B.astype(np.float64).T
+    assert np.linalg.norm(C - exact) / np.linalg.norm(exact) < 6e-2
+
+
+def test_fp8_forward_identical_experts_closed_form():
+    rng = np.random.default_rng(5)
+    T, d, E, I = 16, 256, 4, 128
+    x = oracle.bf16_round(rng.normal(size=(T, d)))
+    Wr = rng.normal(size=(E, d)) * 0.05
+    W1 = np.repeat(rng.normal(size=(1, 2 * I, d)) * 0.05, E, axis=0)
+    W2 = np.repeat(rng.normal(size=(1, d, I)) * 0.05, E, axis=0)
+    r = fp8.moe_forward_fp8(x, Wr, None, W1, W2, k=2)
+    psum = np.take_along_axis(r["p"], r["idx"], axis=1).sum(axis=1)
+    xq, sx = fp8.quantize_1x128(x.astype(np.float32))
+    W1q, s1 = fp8.quantize_128x128(W1[0])
+    W2q, s2 = fp8.quantize_128x128(W2[0])
+    dense = fp8.swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)["y"]
+    assert np.allclose(r["out"], psum[:, None] * dense, rtol=1e-12, atol=1e-12)
+    # and the FP8 forward stays at quantisation-noise distance from the bf16 oracle
+    ref = oracle.moe_forward(x, Wr, None, W1, W2, k=2)["out"]
+    assert np.linalg.norm(r["out"] - ref) / np.linalg.norm(ref) < 1e-1
+
+
+@pytest.mark.parametrize("shape", [(128, 127), (100, 128)])
+def test_quantiser_rejects_ragged_blocks(shape):
+    with pytest.raises(ValueError):
+        fp8.quantize_128x128(np.zeros(shape, np.float32))
