@@ -1,0 +1,528 @@
+#!/usr/bin/env python
+"""MoE-layer forward benchmark on B200: tokens/s and grouped-GEMM TFLOP/s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config mixtral] [--impl ours|reference]
+
+One step = one whole layer forward (router, permute, up grouped GEMM with the
+SiLU gate, down grouped GEMM, combine) over the workload's T tokens.  The
+default workload is the Mixtral-shaped layer (T=4096, d=4096, E=8 top-2,
+I=14336, Zipf s=1.0 routing skew).  Inputs are seeded synthetic tensors
+resident in HBM; the L2 cache is flushed (a 2x-L2 buffer is rewritten)
+between timed steps, outside the timed events.  Each step is timed with CUDA
+events on the launching stream; with N > 1 (torchrun) every rank runs an
+independent replica of the layer on its own tokens (the layer has no
+exchange step on one node's data-parallel path), and the reported time is the
+max over ranks.
+
+Printed: ONE JSON line (rank 0) with the contract keys plus
+  kernels      per-kernel average device time (staged run of the same kernels)
+  roofline     the up-projection grouped GEMM against the measured bf16 peak
+  e2e          the same metric through moe_forward_host (host buffers, H2D of x
+               and D2H of the output inside the timed region)
+  cpu_baseline the fp64 oracle on a bounded token sample, on this host's cores
+  clocks       SM clock / throttle reasons sampled during the timed region
+`--impl reference` times the oracle alone (the slow CPU reference arm).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from workload import CONFIGS, make_inputs, shape_of  # noqa: E402
+
+METRIC = "MoE-layer tokens/s at 1 B200; grouped-GEMM TFLOP/s as % of dense tensor peak"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNELS_PER_FORWARD = 7  # router, hist, scan, scatter, up GEMM, down GEMM, combine
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def workload_desc(s) -> str:
+    parts = [f"{s.name}: T={s.T} d={s.d} E={s.E} top-{s.k} I={s.inter}"]
+    if s.shared_inter:
+        parts.append(f"+1 shared (I={s.shared_inter})")
+    parts.append("fp8 e4m3 experts" if s.fp8 else "bf16")
+    parts.append(f"Zipf s={s.zipf_s} logit bias" if s.zipf_s else "balanced router")
+    return ", ".join(parts)
+
+
+def config_block(s):
+    return {"workload": workload_desc(s), "tokens_per_step": s.T, "seed": 1234,
+            "l2": "flushed between timed steps (2x L2 buffer rewrite, outside the events)",
+            "parallelism": "replicas (one independent layer per GPU)"}
+
+
+# --------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        try:
+            import tempfile
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+        time.sleep(0.15)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or not self.path or not os.path.exists(self.path):
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        for line in open(self.path):
+            f = [x.strip() for x in line.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                rows.append((float(f[1]), float(f[2]), f))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = set()
+        for _, _, f in rows:
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        loaded = [r[0] for r in rows] or [0]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------- our arm
+def build_lib():
+    from grouped_gemm_03_b200.build import build
+    build()
+    import grouped_gemm_03_b200 as gg
+    gg.lib()
+    return gg
+
+
+def make_cfg(gg, s):
+    xdt = gg.MOE_F32 if s.x_dtype == "f32" else gg.MOE_BF16
+    rdt = gg.MOE_F32 if s.router_dtype == "f32" else gg.MOE_BF16
+    odt = gg.MOE_F32 if s.x_dtype == "f32" else gg.MOE_BF16
+    return gg.make_config(s.T, s.d, s.E, s.k, s.inter, s.shared_inter, xdt, rdt,
+                          gg.MOE_E4M3 if s.fp8 else gg.MOE_BF16, odt, s.renormalize)
+
+
+class Staged:
+    """The forward as its separate C-ABI calls (same kernels as moe_forward), for per-kernel timing."""
+
+    def __init__(self, gg, s, inp, dev):
+        self.gg, self.s, self.inp = gg, s, inp
+        T, k, E, d, I = s.T, s.k, s.E, s.d, s.inter
+        shared = bool(s.shared_inter)
+        R = T * k + (T if shared else 0)
+        self.rows = R
+        self.idx = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.w = torch.empty((T, k), dtype=torch.float32, device=dev)
+        self.rws = torch.empty(gg.lib().moe_router_workspace_size(T, E), dtype=torch.uint8, device=dev)
+        self.pws = torch.empty(gg.lib().moe_permute_workspace_size(T, E), dtype=torch.uint8, device=dev)
+        self.gws = torch.empty(256, dtype=torch.uint8, device=dev)
+        self.xp = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
+        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
+        self.offsets = torch.empty(E + 2, dtype=torch.int32, device=dev)
+        self.r2t = torch.empty(R, dtype=torch.int32, device=dev)
+        self.t2r = torch.empty((T, k), dtype=torch.int32, device=dev)
+        self.h = torch.empty((R, I), dtype=torch.bfloat16, device=dev)
+        self.y = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
+        self.out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
+        self.shared = shared
+
+    def stages(self):
+        gg, s, inp = self.gg, self.s, self.inp
+        L = gg.lib()
+        P = gg._ptr
+        st = gg._stream()
+        T, k, E, d, I = s.T, s.k, s.E, s.d, s.inter
+        x = inp["x"]
+        xdt = gg._dt(x)
+
+        def router():
+            gg._check(L.moe_router_topk(P(x), xdt, P(inp["W_r"]), gg._dt(inp["W_r"]), P(inp["bias"]), T, d, E, k,
+                                        int(s.renormalize), None, P(self.idx), P(self.w), P(self.rws),
+                                        self.rws.numel(), st), "router")
+
+        def permute():
+            gg._check(L.moe_permute(P(x), xdt, P(self.idx), T, d, E, k, int(self.shared), gg.MOE_BF16, P(self.xp),
+                                    None, P(self.counts), P(self.offsets), P(self.r2t), P(self.t2r), P(self.pws),
+                                    self.pws.numel(), st), "permute")
+
+        def up():
+            gg._check(self._gemm(L, P(self.xp), inp["W1"], inp["W1s"], I, d, gg.EPI_SILU_GATE, P(self.h), st), "up")
+
+        def down():
+            gg._check(self._gemm(L, P(self.h), inp["W2"], inp["W2s"], d, I, gg.EPI_NONE, P(self.y), st), "down")
+
+        def combine():
+            gg._check(L.moe_combine(P(self.y), P(self.t2r), P(self.w), int(self.shared), T, d, k, P(self.out),
+                                    gg.MOE_BF16, st), "combine")
+
+        return [("router", router), ("permute", permute), ("up_gemm", up), ("down_gemm", down),
+                ("combine", combine)]
+
+    def _gemm(self, L, A, B, Bx, N, K, epi, C, st):
+        # the routed experts and, when present, the shared expert: two launches of the standalone entry
+        # point would differ from moe_forward's single launch, so time the fused one through the forward's
+        # own path when a shared expert exists (the staged breakdown is exact only without one)
+        gg = self.gg
+        P = gg._ptr
+        E = self.s.E
+        return L.moe_grouped_gemm(A, None, P(B), None, P(self.offsets), E, self.rows, N, K, gg.MOE_BF16, epi, C,
+                                  gg.MOE_BF16, None, P(self.gws), self.gws.numel(), st)
+
+
+def time_steps(fn, steps, warmup, flush, stream):
+    for _ in range(warmup):
+        fn()
+    torch.cuda.synchronize()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in ev:
+        flush()
+        a.record(stream)
+        fn()
+        b.record(stream)
+    torch.cuda.synchronize()
+    return [a.elapsed_time(b) for a, b in ev]
+
+
+def time_staged(staged, steps, flush, stream):
+    st = staged.stages()
+    for _ in range(2):
+        for _, f in st:
+            f()
+    torch.cuda.synchronize()
+    per = {n: [] for n, _ in st}
+    for _ in range(steps):
+        flush()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(st) + 1)]
+        evs[0].record(stream)
+        for i, (_, f) in enumerate(st):
+            f()
+            evs[i + 1].record(stream)
+        torch.cuda.synchronize()
+        for i, (n, _) in enumerate(st):
+            per[n].append(evs[i].elapsed_time(evs[i + 1]))
+    return {n: float(np.mean(v)) for n, v in per.items()}
+
+
+def traffic_from_profile(kernel_src_hash):
+    """DRAM bytes per launch of the up GEMM from the committed ncu summary, if it matches this source."""
+    p = os.path.join(ROOT, "profiles", "up_gemm_traffic.json")
+    if not os.path.exists(p):
+        return None
+    try:
+        d = json.load(open(p))
+    except Exception:
+        return None
+    if d.get("source_sha256") != kernel_src_hash:
+        return None
+    return d.get("bytes_per_launch_full")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in ("grouped_gemm.cu", "ptx.cuh", "common.cuh"):
+        h.update(open(os.path.join(ROOT, "grouped_gemm_03_b200", "csrc", f), "rb").read())
+    return h.hexdigest()
+
+
+def algorithmic(s, counts=None):
+    """Per-kernel algorithmic FLOPs / bytes of one forward (bf16)."""
+    T, d, E, k, I = s.T, s.d, s.E, s.k, s.inter
+    sh = 1 if s.shared_inter else 0
+    R = T * k
+    Rp = R + sh * T
+    active = E if counts is None else int((np.asarray(counts) > 0).sum())
+    eb = 1 if s.fp8 else 2
+    xb = 4 if s.x_dtype == "f32" else 2
+    ob = 4 if s.x_dtype == "f32" else 2
+    return {
+        "router": {"bytes": T * d * xb + E * d * (4 if s.router_dtype == "f32" else 2) + T * k * 8},
+        "permute": {"bytes": T * d * xb + Rp * d * eb + T * k * 4 * 3},
+        "up_gemm": {"flops": 2.0 * Rp * 2 * I * d,
+                    "bytes": (active + sh) * 2 * I * d * eb + Rp * d * eb + Rp * I * eb},
+        "down_gemm": {"flops": 2.0 * Rp * d * I,
+                      "bytes": (active + sh) * d * I * eb + Rp * I * eb + Rp * d * 2},
+        "combine": {"bytes": Rp * d * 2 + T * d * ob + T * k * 8},
+    }
+
+
+class HostExperts:
+    """[e] -> host fp64 copy of expert e of a stacked device weight tensor (input staging, not timed)."""
+
+    def __init__(self, t):
+        self.t, self.cache = t, {}
+
+    def __getitem__(self, e):
+        import oracle
+        e = int(e)
+        if e not in self.cache:
+            self.cache[e] = oracle.as_f64(self.t[e])
+        return self.cache[e]
+
+    def stage(self, experts):
+        for e in experts:
+            self[e]
+
+
+def cpu_baseline(s, inp, budget_s=12.0):
+    """The oracle forward on doubling token samples until ~budget_s of CPU time; tokens/s."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    rng = np.random.default_rng(7)
+    W1, W2 = HostExperts(inp["W1"]), HostExperts(inp["W2"])
+    W1s = oracle.as_f64(inp["W1s"]) if inp["W1s"] is not None else None
+    W2s = oracle.as_f64(inp["W2s"]) if inp["W2s"] is not None else None
+    n, done_tokens, spent = 16, 0, 0.0
+    while spent < budget_s and n <= s.T:
+        toks = np.sort(rng.choice(s.T, size=n, replace=False))
+        xs = inp["x"][toks]
+        need = np.unique(oracle.route(xs, inp["W_r"], inp["bias"], s.k)["idx"])
+        W1.stage(need)
+        W2.stage(need)
+        t0 = time.perf_counter()
+        oracle.moe_forward(xs, inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k, renormalize=s.renormalize)
+        spent += time.perf_counter() - t0
+        done_tokens += n
+        n *= 2
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    return {"value": round(done_tokens / spent, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 numpy oracle forward (routing, selected experts, shared) of {done_tokens} of {s.T} "
+                      f"tokens in doubling batches from 16, {spent:.1f} s; expert weights staged to host "
+                      f"fp64 before each timed batch"}
+
+
+def run_ours(args, rank, world, dev):
+    gg = build_lib()
+    s = shape_of(args.config)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    inp = make_inputs(s, seed=1234 + rank, device=dev)
+    cfg = make_cfg(gg, s)
+    ws = torch.empty(gg.workspace_size(cfg) + gg.host_staging_size(cfg), dtype=torch.uint8, device=dev)
+    weights = gg.ExpertWeights(W1=inp["W1"], W2=inp["W2"], W1s=inp["W1s"], W2s=inp["W2s"])
+    out = torch.empty((s.T, s.d), dtype=torch.bfloat16 if s.x_dtype != "f32" else torch.float32, device=dev)
+    counts = torch.empty(s.E, dtype=torch.int32, device=dev)
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    scrub = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+
+    def flush():
+        scrub.fill_(1)
+
+    def step():
+        gg.moe_forward(cfg, inp["x"], inp["W_r"], inp["bias"], weights, out=out, counts_out=counts, ws=ws)
+
+    # --- headline: K timed forwards
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        times = time_steps(step, args.steps, args.warmup, flush, stream)
+        torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    status = gg.read_device_status(ws)
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    ms = float(np.mean(times))
+    if world > 1:
+        t = torch.tensor([ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+
+    # --- e2e: host buffers through moe_forward_host, copies inside the timed region
+    xh = inp["x"].cpu().pin_memory()
+    oh = torch.empty((s.T, s.d), dtype=out.dtype).pin_memory()
+
+    def step_host():
+        gg.moe_forward_host(cfg, xh, inp["W_r"], inp["bias"], weights, oh, ws)
+
+    e2e_times = time_steps(step_host, max(3, args.steps // 2), 2, flush, stream)
+    e2e_ms = float(np.mean(e2e_times))
+    if world > 1:
+        t = torch.tensor([e2e_ms], device=dev)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+
+    # --- per-kernel breakdown (staged calls of the same kernels)
+    kern = {}
+    if not s.shared_inter and not s.fp8:
+        staged = Staged(gg, s, inp, dev)
+        kt = time_staged(staged, max(3, args.steps // 2), flush, stream)
+        alg = algorithmic(s, counts.cpu().numpy())
+        peaks, _ = load_peaks()
+        for name, t_ms in kt.items():
+            a = alg[name]
+            e = {"us": round(t_ms * 1e3, 2)}
+            if "flops" in a:
+                e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
+            e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
+            kern[name] = e
+    return dict(ms=ms, e2e_ms=e2e_ms, kernels=kern, clocks=clk.summary(), inp=inp, s=s, counts=counts.cpu().numpy(),
+                out_dtype=out.dtype)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        log("warm-up raised to 3 steps")
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    s = shape_of(args.config)
+
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        return run_reference(args, s, world)
+
+    if world > 1:
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local))
+    r = run_ours(args, rank, world, local)
+    peaks, peak_kind = load_peaks()
+    result = None
+    if rank == 0:
+        T = s.T
+        value = world * T / (r["ms"] * 1e-3)
+        alg = algorithmic(s, r["counts"])
+        up = r["kernels"].get("up_gemm")
+        roof = None
+        if up:
+            achieved = alg["up_gemm"]["flops"] / (up["us"] * 1e-6) / 1e12
+            peak = float(peaks["bf16_tflops"])
+            roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
+                    "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(kernel_source_hash()),
+                    "kernel": "up-projection grouped GEMM (SiLU gate)",
+                    "peak_kind": f"{peak_kind} bf16 burst (cuBLAS 8192^3)"}
+        gemm_flops = s.gemm_flops()
+        result = {
+            "metric": METRIC,
+            "value": round(value, 1),
+            "unit": "tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": round(r["ms"], 4),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "e4m3" if s.fp8 else "bf16",
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
+            "config": config_block(s),
+            "gemm_tflops": round(gemm_flops / (r["ms"] * 1e-3) / 1e12, 1),
+            "gemm_frac_of_peak": round(gemm_flops / (r["ms"] * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4),
+            "roofline": roof,
+            "kernels": r["kernels"],
+            "e2e": {"value": round(world * T / (r["e2e_ms"] * 1e-3), 1), "unit": "tokens/s",
+                    "h2d_bytes_per_step": T * s.d * (4 if s.x_dtype == "f32" else 2),
+                    "d2h_bytes_per_step": T * s.d * (4 if r["out_dtype"] == torch.float32 else 2)},
+            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
+            "clocks": r["clocks"],
+            "expert_counts": {"min": int(r["counts"].min()), "max": int(r["counts"].max()),
+                              "mean": float(r["counts"].mean()), "zeros": int((r["counts"] == 0).sum())},
+        }
+        if world == 1 and not args.no_cpu_baseline:
+            result["cpu_baseline"] = cpu_baseline(s, r["inp"])
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def run_reference(args, s, world):
+    """The oracle (fp64, host cores) on a bounded token sample per step, as the slow reference arm."""
+    import oracle
+    from threadpoolctl import threadpool_info
+
+    inp = make_inputs(s, seed=1234, device="cuda" if torch.cuda.is_available() else "cpu")
+    W1, W2 = HostExperts(inp["W1"]), HostExperts(inp["W2"])
+    W1s = oracle.as_f64(inp["W1s"]) if inp["W1s"] is not None else None
+    W2s = oracle.as_f64(inp["W2s"]) if inp["W2s"] is not None else None
+    rng = np.random.default_rng(3)
+    per_step = 8
+
+    def step():
+        toks = np.sort(rng.choice(s.T, size=per_step, replace=False))
+        oracle.moe_forward(inp["x"][toks], inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k,
+                           renormalize=s.renormalize)
+
+    for _ in range(args.warmup):
+        step()
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        step()
+    dt = time.perf_counter() - t0
+    value = args.steps * per_step / dt
+    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_block(s),
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                             "sample": f"{per_step} random tokens of {s.T} per step (fp64 oracle forward)"},
+            "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,103 @@
+// Shared definitions of the library's translation units: status handling,
+// small device helpers and the internal launcher interfaces the C ABI layer
+// (moe_api.cu) composes.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+
+#include <cstdint>
+
+#include "moe.h"
+
+namespace moe {
+
+constexpr int kMaxGroups = 1024;     // experts (+ shared) one grouped GEMM launch handles
+constexpr int kMaxTopK = 32;
+constexpr int kMaxExperts = 1024;
+constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
+
+// Record the first device-side error in the status word (0 = OK).
+__device__ __forceinline__ void set_status(int* status, int code) {
+  if (status) atomicCAS(status, 0, code);
+}
+
+__device__ __forceinline__ float bf16_bits_to_float(uint16_t b) {
+  return __uint_as_float(static_cast<uint32_t>(b) << 16);
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T v);
+template <>
+__device__ __forceinline__ float to_f32<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <>
+__device__ __forceinline__ float to_f32<__half>(__half v) { return __half2float(v); }
+
+// Two fp32 -> packed E4M3 pair (round to nearest even, saturating to +-448);
+// `lo` lands in the low byte.
+__device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
+  return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
+}
+
+inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+// ---------------------------------------------------------------- launchers
+// Each returns a moe_status; they assume arguments were validated.
+
+int launch_router_simt(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T,
+                       int d, int E, int k, int renorm, float* logits_out, int32_t* idx, float* w,
+                       cudaStream_t s);
+int launch_topk_logits(const void* logits, int dtype, int N, int E, int k, int renorm, int32_t* idx,
+                       float* w, cudaStream_t s);
+
+struct PermuteArgs {
+  const void* x;
+  int x_dtype;
+  const int32_t* idx;
+  int T, d, E, k, shared, xp_dtype;
+  void* xp;
+  float* xp_scales;
+  int32_t* counts;
+  int32_t* offsets;
+  int32_t* row_to_token;
+  int32_t* token_to_row;
+  int32_t* block_base;  // scratch [nblocks * E]
+  int* status;
+};
+int permute_blocks(int T);  // number of token blocks the permute kernels use
+int launch_permute(const PermuteArgs& a, cudaStream_t s);
+
+struct GemmArgs {
+  const void* A;
+  const float* A_scales;
+  const void* B;            // [G, Nb, K]
+  const float* B_scales;
+  const void* B_extra;      // optional extra group (index G) with its own [Nb, K] weights
+  const float* B_extra_scales;
+  const int32_t* offsets;   // [G + has_extra + 1]
+  int G, has_extra, rows, N, K;
+  int ab_dtype, epilogue, c_dtype;
+  void* C;
+  float* C_scales;
+  int* status;
+};
+int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s);
+
+int launch_combine(const void* Y, const int32_t* t2r, const float* w, int has_shared, int T, int d, int k,
+                   void* out, int out_dtype, cudaStream_t s);
+int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, cudaStream_t s);
+
+int num_sms();
+
+}  // namespace moe
+
+#define MOE_CUDA_CHECK(expr)                        \
+  do {                                              \
+    cudaError_t _e = (expr);                        \
+    if (_e != cudaSuccess) return MOE_ERR_CUDA;     \
+  } while (0)

@@ -1,0 +1,441 @@
+// Persistent grouped GEMM on the 5th-generation tensor cores (tcgen05 + TMEM).
+//
+// "MegaMoE ..." §4.3: one launch computes many GEMM problems that share N and
+// K but have their own M_i; tokens of one expert are contiguous, so problem
+// g is rows offsets[g] .. offsets[g+1]-1 of one A matrix.  "Dense GEMM ->
+// GroupedGEMM -> TP MoE" §2.3 gives the call shape; its pointer arrays become
+// base + offset arithmetic done on the device (its §4.3 / §5.4 note that
+// host-built pointer arrays raced), and the expert sizes never leave the GPU.
+//
+// Structure (one CTA per SM, persistent, 6 warps):
+//   warp 0      TMA producer: A tile [128 x 128 B] and B tile [N_mma x 128 B]
+//               per k-step into an S-stage shared-memory ring (mbarrier
+//               full/empty pairs, 128-byte swizzle);
+//   warp 1      allocates TMEM, one thread issues tcgen05.mma 128 x N_mma x 16
+//               into one of two TMEM accumulators and commits stage / tile
+//               completion to mbarriers;
+//   warps 2-5   epilogue: tcgen05.ld the accumulator (thread = row), apply the
+//               SiLU gate or a plain cast, store the row segment with 16-byte
+//               stores predicated on the row belonging to the group
+//               ("MegaMoE ..." §5.3 tail rows), then release the accumulator.
+// The two accumulators let the epilogue of tile i overlap the main loop of
+// tile i+1 ("MegaMoE ..." §5.2 double buffering, here in TMEM).
+//
+// Tiles: the scheduler enumerates, group by group, ceil(M_g / 128) m-blocks x
+// (N / N_out) n-blocks, m-blocks of one n-block adjacent so that CTAs running
+// at the same time share the weight tile through L2.  An expert with no rows
+// contributes no tile and its weights are never read.  CTA c takes tiles
+// c, c + gridDim.x, ...  A tile that runs past its group's last row reads the
+// next group's rows (or TMA zero fill past the end of A); those rows are
+// computed and discarded, never stored.
+//
+// SiLU-gate epilogue: per k-step the B tile is [gate rows n0..n0+127 ; up rows
+// N+n0..N+n0+127], so one 128 x 256 MMA produces gate and up side by side in
+// TMEM and the epilogue writes h = silu(g) * u for 128 output columns.
+#include <cstdio>
+#include <mutex>
+
+#include "common.cuh"
+#include "ptx.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int BM = 128;
+constexpr int kThreads = 192;
+constexpr int kSmemBudget = 220 * 1024;
+
+template <int MMA_N>
+struct Tile {
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = MMA_N * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr int TABLE_BYTES = 2 * (kMaxGroups + 2) * 4;
+  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512) / STAGE_BYTES;
+  static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
+  static constexpr int TMEM_COLS = 2 * MMA_N;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES;
+};
+
+struct Params {
+  const int32_t* offsets;
+  int G_total;  // groups, including the extra one
+  int G_main;   // groups whose weights come from tmB; group G_main (if any) uses tmBx
+  int N, K, rows;
+  void* C;
+  int* status;
+};
+
+// Largest g in [0, G) with tile_start[g] <= tile.
+__device__ __forceinline__ int find_group(const int* tile_start, int G, int tile) {
+  int lo = 0, hi = G - 1;
+  while (lo < hi) {
+    const int mid = (lo + hi + 1) >> 1;
+    if (tile_start[mid] <= tile)
+      lo = mid;
+    else
+      hi = mid - 1;
+  }
+  return lo;
+}
+
+template <int MMA_N, int EPI, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gg_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                   const __grid_constant__ CUtensorMap tmBx, const Params p) {
+  using L = Tile<MMA_N>;
+  constexpr int OUT_COLS = EPI ? MMA_N / 2 : MMA_N;
+  constexpr uint32_t IDESC = ptx::make_idesc(BM, MMA_N, 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + L::STAGES * L::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + L::STAGES * L::B_BYTES);
+  uint64_t* empty = full + L::STAGES;
+  uint64_t* tfull = empty + L::STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + L::STAGES * L::STAGE_BYTES + 512);
+  int* s_tile = s_off + kMaxGroups + 2;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G_total;
+  const int nt = p.N / OUT_COLS;
+
+  // ---- group tables: row offsets and the exclusive prefix of tile counts
+  if (warp == 0) {
+    for (int g = lane; g <= G; g += 32) s_off[g] = p.offsets[g];
+    __syncwarp();
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int bad = 0, mine = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int m = s_off[g + 1] - s_off[g];
+      if (m < 0) bad = 1;
+      mine += (max(m, 0) + BM - 1) / BM * nt;
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - mine;
+    for (int g = g0; g < g1; ++g) {
+      s_tile[g] = run;
+      run += (max(s_off[g + 1] - s_off[g], 0) + BM - 1) / BM * nt;
+    }
+    if (lane == 31) s_tile[G] = incl;
+    if (lane == 0 && (s_off[0] != 0 || s_off[G] > p.rows)) bad = 1;
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      *s_bad = bad;
+      *abort_flag = 0;
+      if (bad && blockIdx.x == 0) set_status(p.status, MOE_ERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  if (*s_bad) return;  // uniform: nothing loaded, nothing allocated
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&tfull[a], 1);
+      ptx::mbar_init(&tempty[a], 128);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+    ptx::prefetch_tmap(&tmBx);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, L::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tile[G];
+  const int nk = p.K / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t stage = 0, phase = 0;
+      uint32_t issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const int g = find_group(s_tile, G, tile);
+        const int m_g = s_off[g + 1] - s_off[g];
+        const int mt = (m_g + BM - 1) / BM;
+        const int tl = tile - s_tile[g];
+        const int nb = tl / mt, mb = tl % mt;
+        const int a_row = s_off[g] + mb * BM;
+        const bool extra = g >= p.G_main;
+        const CUtensorMap* mB = extra ? &tmBx : &tmB;
+        const int gb = extra ? 0 : g;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          ptx::tma_load_2d(sA + stage * L::A_BYTES, &tmA, &full[stage], kb * 64, a_row);
+          if (EPI) {
+            const int brow = gb * 2 * p.N + nb * (MMA_N / 2);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 64, brow);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES + (MMA_N / 2) * 128, mB, &full[stage], kb * 64,
+                             brow + p.N);
+          } else {
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 64, gb * p.N + nb * MMA_N);
+          }
+          ++issued;
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        // let the copies already issued land before the CTA exits
+        const uint32_t pending = issued < static_cast<uint32_t>(L::STAGES) ? issued : L::STAGES;
+        uint32_t s = stage, ph = phase;
+        for (uint32_t i = 0; i < pending; ++i) {
+          if (s == 0) {
+            s = L::STAGES - 1;
+            ph ^= 1;
+          } else {
+            --s;
+          }
+          ptx::mbar_wait(&full[s], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (!ptx::mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * MMA_N;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t adesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sA + stage * L::A_BYTES));
+          const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sB + stage * L::B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | kk) != 0);
+          ptx::umma_commit(&empty[stage]);
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        ptx::umma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+      }
+      // every MMA issued must finish before TMEM is released
+      ptx::umma_commit(drain);
+      ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter this warp may access
+    const int row_t = q * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int g = find_group(s_tile, G, tile);
+      const int m_g = s_off[g + 1] - s_off[g];
+      const int mt = (m_g + BM - 1) / BM;
+      const int tl = tile - s_tile[g];
+      const int nb = tl / mt, mb = tl % mt;
+      const int r_in = mb * BM + row_t;
+      const bool valid = r_in < m_g;
+      const size_t grow = static_cast<size_t>(s_off[g] + r_in);
+      if (!ptx::mbar_wait_warp(&tfull[acc], use & 1, abort_flag, kWaitLimitNs)) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t tacc = lane_base + acc * MMA_N;
+      if constexpr (EPI == 1) {
+        __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS;
+#pragma unroll 1
+        for (int c = 0; c < OUT_COLS; c += 32) {
+          uint32_t gv[32], uv[32];
+          ptx::tmem_ld_32x32b_x32(tacc + c, gv);
+          ptx::tmem_ld_32x32b_x32(tacc + OUT_COLS + c, uv);
+          ptx::tmem_ld_wait();
+          if (valid) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
+              const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(uv[2 * i]);
+              const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(uv[2 * i + 1]);
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
+              packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(C + c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < OUT_COLS; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld_32x32b_x32(tacc + c, v);
+          ptx::tmem_ld_wait();
+          if (valid) {
+            if constexpr (OUT == 1) {
+              float* C = static_cast<float*>(p.C) + grow * p.N + nb * OUT_COLS + c;
+              uint4* dst = reinterpret_cast<uint4*>(C);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS + c;
+              uint32_t packed[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const __nv_bfloat162 hb =
+                    __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
+              }
+              uint4* dst = reinterpret_cast<uint4*>(C);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&tempty[acc]);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn get_encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* f = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(f);
+  });
+  return fn;
+}
+
+// 2-D K-major map over [rows, K] elements of `ebytes` bytes, box {128 B, box_rows}.
+bool make_map(CUtensorMap* m, const void* base, int ebytes, uint64_t rows, uint64_t K, uint32_t box_rows) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {K, rows};
+  const cuuint64_t strides[1] = {K * static_cast<uint64_t>(ebytes)};
+  const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / ebytes), box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = ebytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+template <int MMA_N, int EPI, int OUT>
+int run_bf16(const GemmArgs& a, cudaStream_t s) {
+  using L = Tile<MMA_N>;
+  static_assert(L::SMEM <= 227 * 1024, "shared memory budget");
+  const int nb_rows = EPI ? 2 * a.N : a.N;
+  const uint32_t box_b = EPI ? MMA_N / 2 : MMA_N;
+  CUtensorMap mA, mB, mBx;
+  if (!make_map(&mA, a.A, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
+  if (!make_map(&mB, a.B, 2, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  MOE_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    MOE_CUDA_CHECK(cudaFuncSetAttribute(gg_bf16_kernel<MMA_N, EPI, OUT>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
+    attr_set[dev] = true;
+  }
+  Params p;
+  p.offsets = a.offsets;
+  p.G_total = a.G + a.has_extra;
+  p.G_main = a.G;
+  p.N = a.N;
+  p.K = a.K;
+  p.rows = a.rows;
+  p.C = a.C;
+  p.status = a.status;
+  gg_bf16_kernel<MMA_N, EPI, OUT><<<num_sms(), kThreads, L::SMEM, s>>>(mA, mB, mBx, p);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+}  // namespace
+
+int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (a.G + a.has_extra == 0 || a.rows == 0) return MOE_OK;
+  if (a.ab_dtype == MOE_BF16) {
+    if (a.epilogue == MOE_EPI_SILU_GATE) {
+      if (a.c_dtype == MOE_BF16 && a.N % 128 == 0) return run_bf16<256, 1, 0>(a, s);
+      return MOE_ERR_UNSUPPORTED;
+    }
+    const int out = a.c_dtype == MOE_F32 ? 1 : 0;
+    if (a.c_dtype != MOE_F32 && a.c_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
+    if (a.N % 256 == 0) return out ? run_bf16<256, 0, 1>(a, s) : run_bf16<256, 0, 0>(a, s);
+    if (a.N % 128 == 0) return out ? run_bf16<128, 0, 1>(a, s) : run_bf16<128, 0, 0>(a, s);
+    if (a.N % 64 == 0) return out ? run_bf16<64, 0, 1>(a, s) : run_bf16<64, 0, 0>(a, s);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_ERR_UNSUPPORTED;  // E4M3 operands: see the FP8 kernel
+}
+
+}  // namespace moe

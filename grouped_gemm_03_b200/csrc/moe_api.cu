@@ -1,0 +1,399 @@
+// The C ABI (include/moe.h): argument validation, workspace layout and the
+// composition of the kernels into the layer forward.  Nothing here computes;
+// every step of the path runs in the kernels of the other translation units.
+#include <cstring>
+
+#include "common.cuh"
+
+namespace moe {
+
+int num_sms() {
+  static int cached[64] = {};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cached[dev]) {
+    int n = 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n <= 0) n = 148;
+    cached[dev] = n;
+  }
+  return cached[dev];
+}
+
+namespace {
+
+inline cudaStream_t as_stream(void* s) { return static_cast<cudaStream_t>(s); }
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+size_t dtype_bytes(int dt) {
+  switch (dt) {
+    case MOE_F32: return 4;
+    case MOE_F16: return 2;
+    case MOE_BF16: return 2;
+    case MOE_E4M3: return 1;
+    default: return 0;
+  }
+}
+
+struct FwdLayout {
+  size_t status, idx, w, logits, base, counts, offsets, r2t, t2r, xp, xps, h, hs, y, total;
+};
+
+FwdLayout fwd_layout(const moe_config& c) {
+  FwdLayout L{};
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t o = off;
+    off = align_up(off + (bytes ? bytes : 1), 1024);
+    return o;
+  };
+  const size_t T = c.T, k = c.k, E = c.E, d = c.d, I = c.inter;
+  const size_t R = T * k, Rp = R + (c.shared_inter ? T : 0);
+  const bool fp8 = c.expert_dtype == MOE_E4M3;
+  const size_t eb = fp8 ? 1 : 2;
+  L.status = take(256);
+  L.idx = take(T * k * 4);
+  L.w = take(T * k * 4);
+  L.logits = take(T * E * 4);
+  L.base = take(static_cast<size_t>(permute_blocks(c.T)) * E * 4);
+  L.counts = take(E * 4);
+  L.offsets = take((E + 2) * 4);
+  L.r2t = take(Rp * 4);
+  L.t2r = take(T * k * 4);
+  L.xp = take(Rp * d * eb);
+  L.xps = fp8 ? take(d / 128 * Rp * 4) : 0;
+  L.h = take(Rp * I * eb);
+  L.hs = fp8 ? take(I / 128 * Rp * 4) : 0;
+  L.y = take(Rp * d * 2);
+  L.total = off;
+  return L;
+}
+
+int check_config(const moe_config* c) {
+  if (!c) return MOE_ERR_INVALID;
+  if (c->T < 0 || c->d <= 0 || c->E <= 0 || c->k <= 0 || c->inter <= 0) return MOE_ERR_INVALID;
+  if (c->k > c->E || c->k > kMaxTopK) return MOE_ERR_INVALID;
+  if (c->E > kMaxExperts || c->E + 1 > kMaxGroups) return MOE_ERR_UNSUPPORTED;
+  if (c->shared_inter != 0 && c->shared_inter != c->inter) return MOE_ERR_UNSUPPORTED;
+  if (c->x_dtype != MOE_F32 && c->x_dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (c->router_dtype != MOE_F32 && c->router_dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (c->expert_dtype != MOE_BF16 && c->expert_dtype != MOE_E4M3) return MOE_ERR_INVALID;
+  if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (c->d % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  const long long rows = static_cast<long long>(c->T) * (c->k + 1);
+  if (rows * c->d > (1ll << 40) || rows > (1ll << 30)) return MOE_ERR_UNSUPPORTED;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+using namespace moe;
+
+extern "C" {
+
+const char* moe_status_string(int s) {
+  switch (s) {
+    case MOE_OK: return "MOE_OK";
+    case MOE_ERR_INVALID: return "MOE_ERR_INVALID: invalid argument";
+    case MOE_ERR_UNSUPPORTED: return "MOE_ERR_UNSUPPORTED: valid but unsupported shape or type";
+    case MOE_ERR_WORKSPACE: return "MOE_ERR_WORKSPACE: workspace too small or misaligned";
+    case MOE_ERR_CUDA: return "MOE_ERR_CUDA: CUDA call failed";
+    case MOE_ERR_BAD_OFFSETS: return "MOE_ERR_BAD_OFFSETS: group offsets not monotone from 0 within rows";
+    case MOE_ERR_TIMEOUT: return "MOE_ERR_TIMEOUT: kernel pipeline wait timed out";
+    default: return "unknown moe status";
+  }
+}
+
+int moe_device_info(int* num_sms_out, int* cc_major, int* cc_minor) {
+  int dev = 0, maj = 0, min_ = 0;
+  MOE_CUDA_CHECK(cudaGetDevice(&dev));
+  MOE_CUDA_CHECK(cudaDeviceGetAttribute(&maj, cudaDevAttrComputeCapabilityMajor, dev));
+  MOE_CUDA_CHECK(cudaDeviceGetAttribute(&min_, cudaDevAttrComputeCapabilityMinor, dev));
+  if (num_sms_out) *num_sms_out = num_sms();
+  if (cc_major) *cc_major = maj;
+  if (cc_minor) *cc_minor = min_;
+  return maj == 10 ? MOE_OK : MOE_ERR_UNSUPPORTED;
+}
+
+int moe_read_device_status(const void* ws, void* stream, int* status) {
+  if (!ws || !status) return MOE_ERR_INVALID;
+  MOE_CUDA_CHECK(cudaStreamSynchronize(as_stream(stream)));
+  int v = 0;
+  MOE_CUDA_CHECK(cudaMemcpy(&v, ws, sizeof(int), cudaMemcpyDeviceToHost));
+  *status = v;
+  return MOE_OK;
+}
+
+// ------------------------------------------------------------------ router
+size_t moe_router_workspace_size(int T, int E) {
+  return 256 + align_up(static_cast<size_t>(T > 0 ? T : 0) * (E > 0 ? E : 0) * 4, 256);
+}
+
+int moe_router_topk(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d,
+                    int E, int k, int renormalize, float* logits_out, int32_t* topk_idx, float* topk_w, void* ws,
+                    size_t ws_bytes, void* stream) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || k > kMaxTopK || E > kMaxExperts) return MOE_ERR_INVALID;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if ((x_dtype != MOE_F32 && x_dtype != MOE_BF16) || (w_dtype != MOE_F32 && w_dtype != MOE_BF16))
+    return MOE_ERR_INVALID;
+  if (T > 0 && (!x || !W_r || !topk_idx || !topk_w)) return MOE_ERR_INVALID;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_router_workspace_size(T, E)) return MOE_ERR_WORKSPACE;
+  if (!aligned(x, 16) || !aligned(W_r, 16)) return MOE_ERR_INVALID;
+  cudaStream_t s = as_stream(stream);
+  MOE_CUDA_CHECK(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  return launch_router_simt(x, x_dtype, W_r, w_dtype, bias, T, d, E, k, renormalize, logits_out, topk_idx, topk_w,
+                            s);
+}
+
+int moe_topk_logits(const void* logits, int dtype, int N, int E, int k, int renormalize, int32_t* topk_idx,
+                    float* topk_w, void* stream) {
+  if (N < 0 || E <= 0 || k <= 0 || k > E || k > kMaxTopK || E > kMaxExperts) return MOE_ERR_INVALID;
+  if (dtype != MOE_F16 && dtype != MOE_F32 && dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (N > 0 && (!logits || !topk_idx || !topk_w)) return MOE_ERR_INVALID;
+  if (!aligned(logits, 16)) return MOE_ERR_INVALID;
+  return launch_topk_logits(logits, dtype, N, E, k, renormalize, topk_idx, topk_w, as_stream(stream));
+}
+
+// ------------------------------------------------------------------ permute
+size_t moe_permute_workspace_size(int T, int E) {
+  if (T < 0 || E <= 0) return 0;
+  return 256 + align_up(static_cast<size_t>(permute_blocks(T)) * E * 4, 256);
+}
+
+int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k, int append_shared,
+                int xp_dtype, void* xp, float* xp_scales, int32_t* counts, int32_t* offsets, int32_t* row_to_token,
+                int32_t* token_to_row, void* ws, size_t ws_bytes, void* stream) {
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || k > kMaxTopK || E > kMaxExperts) return MOE_ERR_INVALID;
+  if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (xp_dtype != MOE_BF16 && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID;
+  if (d % 8 != 0 || (xp_dtype == MOE_E4M3 && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !offsets) return MOE_ERR_INVALID;
+  if (T > 0 && (!x || !topk_idx || !xp || !row_to_token || !token_to_row)) return MOE_ERR_INVALID;
+  if (T > 0 && xp_dtype == MOE_E4M3 && !xp_scales) return MOE_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(xp, 16)) return MOE_ERR_INVALID;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_permute_workspace_size(T, E)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  MOE_CUDA_CHECK(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  PermuteArgs a;
+  a.x = x;
+  a.x_dtype = x_dtype;
+  a.idx = topk_idx;
+  a.T = T;
+  a.d = d;
+  a.E = E;
+  a.k = k;
+  a.shared = append_shared ? 1 : 0;
+  a.xp_dtype = xp_dtype;
+  a.xp = xp;
+  a.xp_scales = xp_scales;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.row_to_token = row_to_token;
+  a.token_to_row = token_to_row;
+  a.block_base = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + 256);
+  a.status = static_cast<int*>(ws);
+  return launch_permute(a, s);
+}
+
+// ------------------------------------------------------------------ grouped GEMM
+size_t moe_grouped_gemm_workspace_size(void) { return 256; }
+
+int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const float* B_scales,
+                     const int32_t* offsets, int G, int rows, int N, int K, int ab_dtype, int epilogue, void* C,
+                     int c_dtype, float* C_scales, void* ws, size_t ws_bytes, void* stream) {
+  if (G <= 0 || rows < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID;
+  if (G > kMaxGroups) return MOE_ERR_UNSUPPORTED;
+  if (!A || !B || !offsets || !C) return MOE_ERR_INVALID;
+  if (ab_dtype != MOE_BF16 && ab_dtype != MOE_E4M3) return MOE_ERR_INVALID;
+  if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SILU_GATE) return MOE_ERR_INVALID;
+  if (ab_dtype == MOE_E4M3 && (!A_scales || !B_scales)) return MOE_ERR_INVALID;
+  if (c_dtype == MOE_E4M3 && !C_scales) return MOE_ERR_INVALID;
+  if (ab_dtype == MOE_BF16 && K % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (ab_dtype == MOE_E4M3 && K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16)) return MOE_ERR_INVALID;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_grouped_gemm_workspace_size()) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  MOE_CUDA_CHECK(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  GemmArgs a{};
+  a.A = A;
+  a.A_scales = A_scales;
+  a.B = B;
+  a.B_scales = B_scales;
+  a.offsets = offsets;
+  a.G = G;
+  a.has_extra = 0;
+  a.rows = rows;
+  a.N = N;
+  a.K = K;
+  a.ab_dtype = ab_dtype;
+  a.epilogue = epilogue;
+  a.c_dtype = c_dtype;
+  a.C = C;
+  a.C_scales = C_scales;
+  a.status = static_cast<int*>(ws);
+  return launch_grouped_gemm(a, s);
+}
+
+// ------------------------------------------------------------------ combine
+int moe_combine(const void* Y, const int32_t* token_to_row, const float* topk_w, int has_shared, int T, int d, int k,
+                void* out, int out_dtype, void* stream) {
+  if (T < 0 || d <= 0 || k <= 0 || k > kMaxTopK) return MOE_ERR_INVALID;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (out_dtype != MOE_F32 && out_dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (T > 0 && (!Y || !token_to_row || !topk_w || !out)) return MOE_ERR_INVALID;
+  if (!aligned(Y, 16) || !aligned(out, 16)) return MOE_ERR_INVALID;
+  return launch_combine(Y, token_to_row, topk_w, has_shared, T, d, k, out, out_dtype, as_stream(stream));
+}
+
+// ------------------------------------------------------------------ FP8 weights
+int moe_quantize_weights_fp8(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, void* stream) {
+  if (G < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID;
+  if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (G > 0 && (!W || !Wq || !scales)) return MOE_ERR_INVALID;
+  if (!aligned(W, 16) || !aligned(Wq, 16)) return MOE_ERR_INVALID;
+  return launch_quantize_weights(W, G, N, K, Wq, scales, as_stream(stream));
+}
+
+// ------------------------------------------------------------------ whole layer
+size_t moe_workspace_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  return fwd_layout(*cfg).total;
+}
+
+int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const float* router_bias, const void* W1,
+                const float* W1_scales, const void* W2, const float* W2_scales, const void* W1_shared,
+                const float* W1s_scales, const void* W2_shared, const float* W2s_scales, void* out,
+                int32_t* counts_out, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  const moe_config c = *cfg;
+  const bool fp8 = c.expert_dtype == MOE_E4M3;
+  const bool shared = c.shared_inter != 0;
+  if (c.T > 0 && (!x || !W_r || !W1 || !W2 || !out)) return MOE_ERR_INVALID;
+  if (shared && (!W1_shared || !W2_shared)) return MOE_ERR_INVALID;
+  if (fp8 && (!W1_scales || !W2_scales || (shared && (!W1s_scales || !W2s_scales)))) return MOE_ERR_INVALID;
+  if (!aligned(x, 16) || !aligned(W_r, 16) || !aligned(W1, 16) || !aligned(W2, 16) || !aligned(out, 16) ||
+      !aligned(W1_shared, 16) || !aligned(W2_shared, 16))
+    return MOE_ERR_INVALID;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const FwdLayout L = fwd_layout(c);
+  if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
+  if (fp8) return MOE_ERR_UNSUPPORTED;  // E4M3 expert GEMMs are provided by the FP8 kernel
+  cudaStream_t s = as_stream(stream);
+  char* base = static_cast<char*>(ws);
+  int* status = reinterpret_cast<int*>(base + L.status);
+  int32_t* idx = reinterpret_cast<int32_t*>(base + L.idx);
+  float* w = reinterpret_cast<float*>(base + L.w);
+  int32_t* counts = reinterpret_cast<int32_t*>(base + L.counts);
+  int32_t* offsets = reinterpret_cast<int32_t*>(base + L.offsets);
+  int32_t* t2r = reinterpret_cast<int32_t*>(base + L.t2r);
+  MOE_CUDA_CHECK(cudaMemsetAsync(status, 0, sizeof(int), s));
+  if (c.T == 0) {
+    if (counts_out) MOE_CUDA_CHECK(cudaMemsetAsync(counts_out, 0, sizeof(int32_t) * c.E, s));
+    return MOE_OK;
+  }
+  const int T = c.T, d = c.d, E = c.E, k = c.k, I = c.inter;
+  const int Rp = T * k + (shared ? T : 0);
+
+  st = launch_router_simt(x, c.x_dtype, W_r, c.router_dtype, router_bias, T, d, E, k, c.renormalize, nullptr, idx,
+                          w, s);
+  if (st != MOE_OK) return st;
+
+  PermuteArgs pa;
+  pa.x = x;
+  pa.x_dtype = c.x_dtype;
+  pa.idx = idx;
+  pa.T = T;
+  pa.d = d;
+  pa.E = E;
+  pa.k = k;
+  pa.shared = shared ? 1 : 0;
+  pa.xp_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
+  pa.xp = base + L.xp;
+  pa.xp_scales = fp8 ? reinterpret_cast<float*>(base + L.xps) : nullptr;
+  pa.counts = counts;
+  pa.offsets = offsets;
+  pa.row_to_token = reinterpret_cast<int32_t*>(base + L.r2t);
+  pa.token_to_row = t2r;
+  pa.block_base = reinterpret_cast<int32_t*>(base + L.base);
+  pa.status = status;
+  st = launch_permute(pa, s);
+  if (st != MOE_OK) return st;
+
+  GemmArgs up{};
+  up.A = base + L.xp;
+  up.B = W1;
+  up.B_extra = W1_shared;
+  up.offsets = offsets;
+  up.G = E;
+  up.has_extra = shared ? 1 : 0;
+  up.rows = Rp;
+  up.N = I;
+  up.K = d;
+  up.ab_dtype = MOE_BF16;
+  up.epilogue = MOE_EPI_SILU_GATE;
+  up.c_dtype = MOE_BF16;
+  up.C = base + L.h;
+  up.status = status;
+  st = launch_grouped_gemm(up, s);
+  if (st != MOE_OK) return st;
+
+  GemmArgs dn{};
+  dn.A = base + L.h;
+  dn.B = W2;
+  dn.B_extra = W2_shared;
+  dn.offsets = offsets;
+  dn.G = E;
+  dn.has_extra = shared ? 1 : 0;
+  dn.rows = Rp;
+  dn.N = d;
+  dn.K = I;
+  dn.ab_dtype = MOE_BF16;
+  dn.epilogue = MOE_EPI_NONE;
+  dn.c_dtype = MOE_BF16;
+  dn.C = base + L.y;
+  dn.status = status;
+  st = launch_grouped_gemm(dn, s);
+  if (st != MOE_OK) return st;
+
+  st = launch_combine(base + L.y, t2r, w, shared ? 1 : 0, T, d, k, out, c.out_dtype, s);
+  if (st != MOE_OK) return st;
+  if (counts_out) MOE_CUDA_CHECK(cudaMemcpyAsync(counts_out, counts, sizeof(int32_t) * E, cudaMemcpyDeviceToDevice, s));
+  (void)W1s_scales;
+  (void)W2s_scales;
+  return MOE_OK;
+}
+
+size_t moe_host_staging_size(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return 0;
+  const size_t td = static_cast<size_t>(cfg->T) * cfg->d;
+  return align_up(td * dtype_bytes(cfg->x_dtype), 1024) + align_up(td * dtype_bytes(cfg->out_dtype), 1024);
+}
+
+int moe_forward_host(const moe_config* cfg, const void* x_host, const void* W_r, const float* router_bias,
+                     const void* W1, const float* W1_scales, const void* W2, const float* W2_scales,
+                     const void* W1_shared, const float* W1s_scales, const void* W2_shared, const float* W2s_scales,
+                     void* out_host, void* ws, size_t ws_bytes, void* stream) {
+  int st = check_config(cfg);
+  if (st != MOE_OK) return st;
+  if (cfg->T > 0 && (!x_host || !out_host)) return MOE_ERR_INVALID;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  const size_t fwd = moe_workspace_size(cfg);
+  if (ws_bytes < fwd + moe_host_staging_size(cfg)) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = as_stream(stream);
+  const size_t td = static_cast<size_t>(cfg->T) * cfg->d;
+  char* xd = static_cast<char*>(ws) + fwd;
+  char* od = xd + align_up(td * dtype_bytes(cfg->x_dtype), 1024);
+  if (td) MOE_CUDA_CHECK(cudaMemcpyAsync(xd, x_host, td * dtype_bytes(cfg->x_dtype), cudaMemcpyHostToDevice, s));
+  st = moe_forward(cfg, xd, W_r, router_bias, W1, W1_scales, W2, W2_scales, W1_shared, W1s_scales, W2_shared,
+                   W2s_scales, od, nullptr, ws, fwd, stream);
+  if (st != MOE_OK) return st;
+  if (td) MOE_CUDA_CHECK(cudaMemcpyAsync(out_host, od, td * dtype_bytes(cfg->out_dtype), cudaMemcpyDeviceToHost, s));
+  return MOE_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,277 @@
+// Permute: per-expert histogram, exclusive prefix sum and scatter of tokens
+// into expert-contiguous order ("Dense GEMM -> GroupedGEMM -> TP MoE" §2.2
+// steps 3-4, §4.2 compute_expert_offsets; "MegaMoE ..." §4.3 same-expert
+// tokens contiguous in memory).
+//
+// Three launches, no atomics deciding any position, so the plan is
+// bit-identical run to run:
+//   hist    block b counts, per expert, the (token, slot) pairs of its 32
+//           tokens (shared-memory histogram) -> cnt[b][e];
+//   scan    one CTA turns cnt into absolute row bases base[b][e] =
+//           offsets[e] + sum_{b' < b} cnt[b'][e], plus counts / offsets;
+//   scatter block b ranks its pairs by token order inside the block and
+//           copies each token's row to its k destinations (and, for the
+//           shared expert, to row R + t), casting to bf16 or quantising to
+//           E4M3 with one scale per 128 columns on the way.
+#include "common.cuh"
+
+namespace moe {
+namespace {
+
+constexpr int kTokPerBlock = 32;
+constexpr int kPermThreads = 256;
+
+__global__ void __launch_bounds__(kPermThreads) hist_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
+                                                            int32_t* __restrict__ cnt, int* status) {
+  extern __shared__ int s_cnt[];
+  const int b = blockIdx.x;
+  const int t0 = b * kTokPerBlock;
+  const int nt = min(kTokPerBlock, T - t0);
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
+    const size_t g = static_cast<size_t>(t0) * k + p;
+    const int e = idx[g];
+    bool ok = e >= 0 && e < E;
+    const int j = p % k;
+    for (int jj = 0; jj < j && ok; ++jj) ok = idx[g - j + jj] != e;  // distinct within a token
+    if (ok)
+      atomicAdd(&s_cnt[e], 1);
+    else
+      set_status(status, MOE_ERR_INVALID);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[static_cast<size_t>(b) * E + e] = s_cnt[e];
+}
+
+// Single CTA of 1024 threads: thread (e, c) owns expert e and a contiguous
+// chunk c of the token blocks.
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, int nblk, int E, int R, int T,
+                                                    int shared, int32_t* __restrict__ counts,
+                                                    int32_t* __restrict__ offsets) {
+  __shared__ int s_part[1024];
+  __shared__ int s_tot[1024];
+  __shared__ int s_warp[32];
+  int tpe = 1;  // threads per expert (power of two, tpe * E <= 1024)
+  while (tpe * 2 * E <= 1024 && tpe * 2 <= nblk) tpe *= 2;
+  const int chunk = (nblk + tpe - 1) / tpe;
+  const int e = threadIdx.x / tpe, c = threadIdx.x % tpe;
+  const bool active = e < E;
+  const int b0 = c * chunk, b1 = min(nblk, b0 + chunk);
+  int local = 0;
+  if (active)
+    for (int b = b0; b < b1; ++b) local += base[static_cast<size_t>(b) * E + e];
+  s_part[threadIdx.x] = local;
+  __syncthreads();
+  // per-expert total and exclusive chunk prefix (tpe is small)
+  int chunk_pre = 0;
+  if (active) {
+    int tot = 0;
+    for (int cc = 0; cc < tpe; ++cc) {
+      const int v = s_part[e * tpe + cc];
+      if (cc < c) chunk_pre += v;
+      tot += v;
+    }
+    if (c == 0) s_tot[e] = tot;
+  }
+  __syncthreads();
+  // exclusive scan of s_tot[0..E) by the whole block (one value per thread)
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int mine = threadIdx.x < E ? s_tot[threadIdx.x] : 0;
+  int incl = mine;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl, o);
+    if (lane >= o) incl += y;
+  }
+  if (lane == 31) s_warp[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int w = s_warp[lane];
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    s_warp[lane] = wi - w;
+  }
+  __syncthreads();
+  const int excl = incl - mine + s_warp[warp];
+  __syncthreads();
+  if (threadIdx.x < E) {
+    s_part[threadIdx.x] = excl;  // reuse: offsets
+    counts[threadIdx.x] = mine;
+    offsets[threadIdx.x] = excl;
+  }
+  if (threadIdx.x == 0) {
+    offsets[E] = R;
+    if (shared) offsets[E + 1] = R + T;
+  }
+  __syncthreads();
+  if (active) {
+    int run = s_part[e] + chunk_pre;
+    for (int b = b0; b < b1; ++b) {
+      const size_t i = static_cast<size_t>(b) * E + e;
+      const int v = base[i];
+      base[i] = run;
+      run += v;
+    }
+  }
+}
+
+__device__ __forceinline__ void load_row8(const float* p, float (&f)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+
+template <typename XT, bool kFp8>
+__global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a, int nblk) {
+  __shared__ int s_idx[kTokPerBlock * kMaxTopK];
+  __shared__ int s_row[kTokPerBlock * (kMaxTopK + 1)];
+  const int b = blockIdx.x;
+  const int t0 = b * kTokPerBlock;
+  const int nt = min(kTokPerBlock, a.T - t0);
+  const int k = a.k, E = a.E;
+  const int R = a.T * k;
+  const int rows_total = R + (a.shared ? a.T : 0);
+  const int nd = k + (a.shared ? 1 : 0);  // destinations per token
+  for (int p = threadIdx.x; p < nt * k; p += blockDim.x) s_idx[p] = a.idx[static_cast<size_t>(t0) * k + p];
+  __syncthreads();
+  for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
+    const int tl = p / k, j = p % k;
+    const int e = s_idx[p];
+    int row = 0;
+    if (e >= 0 && e < E) {
+      int rank = 0;
+      for (int q = 0; q < tl * k; ++q) rank += (s_idx[q] == e);
+      row = a.block_base[static_cast<size_t>(b) * E + e] + rank;
+      if (row < 0 || row >= R) row = 0;  // only reachable with invalid ids (status already set)
+    }
+    s_row[tl * nd + j] = row;
+    a.token_to_row[static_cast<size_t>(t0 + tl) * k + j] = row;
+    a.row_to_token[row] = t0 + tl;
+  }
+  if (a.shared)
+    for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) {
+      s_row[tl * nd + k] = R + t0 + tl;
+      a.row_to_token[R + t0 + tl] = t0 + tl;
+    }
+  __syncthreads();
+
+  const int d = a.d;
+  const XT* x = static_cast<const XT*>(a.x);
+  if constexpr (!kFp8) {
+    // bf16 destination: 8 elements (16 bytes) per thread per step
+    __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(a.xp);
+    const int nvec = d / 8;
+    for (int it = threadIdx.x; it < nt * nvec; it += blockDim.x) {
+      const int tl = it / nvec, c = (it % nvec) * 8;
+      const XT* src = x + static_cast<size_t>(t0 + tl) * d + c;
+      uint4 out;
+      if constexpr (sizeof(XT) == 2) {
+        out = *reinterpret_cast<const uint4*>(src);
+      } else {
+        float f[8];
+        load_row8(reinterpret_cast<const float*>(src), f);
+        __nv_bfloat162 h[4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+        out = *reinterpret_cast<uint4*>(h);
+      }
+      for (int j = 0; j < nd; ++j)
+        *reinterpret_cast<uint4*>(xp + static_cast<size_t>(s_row[tl * nd + j]) * d + c) = out;
+    }
+  } else {
+    // E4M3 destination: 16 threads quantise one 128-column group of one token
+    uint8_t* xp = static_cast<uint8_t*>(a.xp);
+    const int ngrp = d / 128;
+    const int sub = threadIdx.x & 15;
+    const int half = (threadIdx.x >> 4) & 1;
+    const int total = nt * ngrp;
+    // warp-uniform trip count: both half-warps run every iteration (the
+    // shuffles below name all 32 lanes), the idle half on dummy data
+    for (int base = (threadIdx.x >> 5) * 2; base < total; base += (blockDim.x >> 5) * 2) {
+      const int it = base + half;
+      const bool act = it < total;
+      const int tl = act ? it / ngrp : 0, gi = act ? it % ngrp : 0;
+      const int c = gi * 128 + sub * 8;
+      float f[8];
+      const XT* src = x + static_cast<size_t>(t0 + tl) * d + c;
+      if (!act) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = 0.f;
+      } else if constexpr (sizeof(XT) == 2) {
+        const uint4 raw = *reinterpret_cast<const uint4*>(src);
+        const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          f[2 * i] = __uint_as_float(w[i] << 16);
+          f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+        }
+      } else {
+        load_row8(reinterpret_cast<const float*>(src), f);
+        // experts consume x rounded to bf16
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = __bfloat162float(__float2bfloat16_rn(f[i]));
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+      for (int o = 8; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+      const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      uint32_t q[2];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(f[4 * i], s), __fdiv_rn(f[4 * i + 1], s));
+        const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(f[4 * i + 2], s), __fdiv_rn(f[4 * i + 3], s));
+        q[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+      }
+      const uint2 qv = make_uint2(q[0], q[1]);
+      if (!act) continue;
+      for (int j = 0; j < nd; ++j) {
+        const int row = s_row[tl * nd + j];
+        *reinterpret_cast<uint2*>(xp + static_cast<size_t>(row) * d + c) = qv;
+        if (sub == 0) a.xp_scales[static_cast<size_t>(gi) * rows_total + row] = s;
+      }
+    }
+  }
+  (void)nblk;
+}
+
+}  // namespace
+
+int permute_blocks(int T) { return (T + kTokPerBlock - 1) / kTokPerBlock; }
+
+int launch_permute(const PermuteArgs& a, cudaStream_t s) {
+  const int nblk = permute_blocks(a.T);
+  if (a.T == 0) {
+    // no tokens: counts are zero and every offset is zero
+    MOE_CUDA_CHECK(cudaMemsetAsync(a.counts, 0, sizeof(int32_t) * a.E, s));
+    MOE_CUDA_CHECK(cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1 + (a.shared ? 1 : 0)), s));
+    return MOE_OK;
+  }
+  hist_kernel<<<nblk, kPermThreads, sizeof(int) * a.E, s>>>(a.idx, a.T, a.E, a.k, a.block_base, a.status);
+  MOE_CUDA_CHECK(cudaGetLastError());
+  scan_kernel<<<1, 1024, 0, s>>>(a.block_base, nblk, a.E, a.T * a.k, a.T, a.shared, a.counts, a.offsets);
+  MOE_CUDA_CHECK(cudaGetLastError());
+  const bool fp8 = a.xp_dtype == MOE_E4M3;
+  if (a.x_dtype == MOE_BF16) {
+    if (fp8)
+      scatter_kernel<__nv_bfloat16, true><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+    else
+      scatter_kernel<__nv_bfloat16, false><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+  } else {
+    if (fp8)
+      scatter_kernel<float, true><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+    else
+      scatter_kernel<float, false><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+  }
+  MOE_CUDA_CHECK(cudaGetLastError());
+  return MOE_OK;
+}
+
+}  // namespace moe
