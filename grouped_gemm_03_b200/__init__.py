@@ -59,6 +59,7 @@ _SIGS = {
     "moe_topk_logits": (_i, [_vp, _i, _i, _i, _i, _i, _ip, _fp, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i]),
     "moe_permute": (_i, [_vp, _i, _ip, _i, _i, _i, _i, _i, _i, _vp, _fp, _ip, _ip, _ip, _ip, _vp, _sz, _vp]),
+    "moe_permute_noalloc": (_i, [_vp, _i, _ip, _i, _i, _i, _i, _i, _i, _vp, _fp, _ip, _ip, _ip, _ip, _vp]),
     "moe_grouped_gemm_workspace_size": (_sz, []),
     "moe_grouped_gemm": (_i, [_vp, _fp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _vp, _i, _fp, _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _ip, _fp, _i, _i, _i, _i, _vp, _i, _vp]),

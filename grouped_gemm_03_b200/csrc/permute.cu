@@ -13,6 +13,8 @@
 //           copies each token's row to its k destinations (and, for the
 //           shared expert, to row R + t), casting to bf16 or quantising to
 //           E4M3 with one scale per 128 columns on the way.
+#include <mutex>
+
 #include "common.cuh"
 
 namespace moe {
@@ -275,3 +277,90 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
 }
 
 }  // namespace moe
+
+// ---------------------------------------------------------------------------
+// Allocation-free permute (moe_permute_noalloc).
+//
+// Some callers cannot hand this library a workspace: a plugin whose host
+// runtime owns all device memory and offers none, code that must not call
+// cudaMalloc while a stream capture is in progress, or a serving loop whose
+// memory plan is frozen at start-up.  For them the permute's scratch (the
+// status word and the per-block expert counts) lives in this file-scope
+// device array instead of a caller workspace.  Every GPU that loads the
+// library keeps the array (1 MiB + 256 bytes) until the process exits; all
+// calls on a device share it, so calls whose kernels overlap on the GPU (two
+// streams, say) race on it and must be ordered by the caller.  A call
+// rewrites every count it reads and clears the status word first, so what
+// a previous call left there does not matter.
+namespace moe {
+namespace {
+
+constexpr int kNoAllocStatusWords = 64;          // status word, padded to 256 bytes
+constexpr size_t kNoAllocCountWords = 262144;    // per-block expert counts (1 MiB of int32)
+
+static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocStatusWords + kNoAllocCountWords];
+
+std::mutex g_scratch_mu;
+int32_t* g_scratch_dev[64] = {};
+
+// Device address of g_permute_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so it must never be passed
+// to a kernel; the address is looked up once per device (with that device
+// current) and cached.
+int noalloc_scratch(int32_t** out) {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  if (!g_scratch_dev[dev]) {
+    void* p = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    if (e != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
+    g_scratch_dev[dev] = static_cast<int32_t*>(p);
+  }
+  *out = g_scratch_dev[dev];
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moe
+
+extern "C" int moe_permute_noalloc(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k,
+                                   int append_shared, int xp_dtype, void* xp, float* xp_scales, int32_t* counts,
+                                   int32_t* offsets, int32_t* row_to_token, int32_t* token_to_row, void* stream) {
+  using namespace moe;
+  if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || k > kMaxTopK || E > kMaxExperts) return MOE_ERR_INVALID;
+  if (static_cast<size_t>(permute_blocks(T)) * static_cast<size_t>(E) > kNoAllocCountWords)
+    return MOE_ERR_UNSUPPORTED;  // beyond the built-in scratch: use moe_permute with a workspace
+  if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (xp_dtype != MOE_BF16 && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID;
+  if (d % 8 != 0 || (xp_dtype == MOE_E4M3 && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (!counts || !offsets) return MOE_ERR_INVALID;
+  if (T > 0 && (!x || !topk_idx || !xp || !row_to_token || !token_to_row)) return MOE_ERR_INVALID;
+  if (T > 0 && xp_dtype == MOE_E4M3 && !xp_scales) return MOE_ERR_INVALID;
+  if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(xp) % 16) return MOE_ERR_INVALID;
+  int32_t* scratch = nullptr;
+  const int st = noalloc_scratch(&scratch);
+  if (st != MOE_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaMemsetAsync(scratch, 0, sizeof(int32_t), s) != cudaSuccess) return MOE_ERR_CUDA;
+  PermuteArgs a;
+  a.x = x;
+  a.x_dtype = x_dtype;
+  a.idx = topk_idx;
+  a.T = T;
+  a.d = d;
+  a.E = E;
+  a.k = k;
+  a.shared = append_shared ? 1 : 0;
+  a.xp_dtype = xp_dtype;
+  a.xp = xp;
+  a.xp_scales = xp_scales;
+  a.counts = counts;
+  a.offsets = offsets;
+  a.row_to_token = row_to_token;
+  a.token_to_row = token_to_row;
+  a.block_base = scratch + kNoAllocStatusWords;
+  a.status = scratch;
+  return launch_permute(a, s);
+}

@@ -130,6 +130,31 @@ int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int 
                 int32_t* offsets, int32_t* row_to_token, int32_t* token_to_row, void* ws, size_t ws_bytes,
                 void* stream);
 
+/* Allocation-free variant of moe_permute, for callers that cannot give the
+ * library any device memory of its own: a plugin whose host runtime owns all
+ * allocations and offers no workspace, code that runs while a stream capture
+ * is in progress (where cudaMalloc is not allowed), or a serving loop whose
+ * memory plan is fixed at start-up.  The source pages have no counterpart;
+ * the operation and the arguments are those of moe_permute, minus `ws`.
+ *   Scratch (status word + per-block expert counts) lives in a 1 MiB + 256 B
+ *   array of static device memory inside the library, which every GPU that
+ *   loads the library keeps until the process exits.  Limit:
+ *   ceil(T / 32) * E <= 262144 (e.g. T <= 32768 at E = 256, T <= 65536 at
+ *   E = 128); larger calls return MOE_ERR_UNSUPPORTED before launching.
+ *   The first call on a device looks up the array's device address (once per
+ *   device, with that device current); make that first call before any
+ *   stream capture begins.
+ *   All calls on a device share the one array and leave their contents
+ *   there; each call clears the status word and rewrites every count it
+ *   reads.  Calls whose kernels overlap on the GPU (e.g. on two streams)
+ *   race on it: order them.  There is no status read-back: invalid expert
+ *   ids are skipped (nothing out of bounds is written) and leave the outputs
+ *   unspecified; use moe_permute + moe_read_device_status to detect them.
+ * Never calls cudaMalloc / cudaFree or any allocating routine. */
+int moe_permute_noalloc(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k,
+                        int append_shared, int xp_dtype, void* xp, float* xp_scales, int32_t* counts,
+                        int32_t* offsets, int32_t* row_to_token, int32_t* token_to_row, void* stream);
+
 /* ---------------------------------------------------------------- grouped GEMM
  * One persistent launch computes, for every group g (an expert) with rows
  * offsets[g] .. offsets[g+1]-1 of A:
