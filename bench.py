@@ -217,13 +217,21 @@ class Staged:
                                   gg.MOE_BF16, None, P(self.gws), self.gws.numel(), st)
 
 
-def time_steps(fn, steps, warmup, flush, stream):
+HOLD_CYCLES = 2_000_000  # ~1 ms spin queued ahead of each timed step
+
+
+def time_steps(fn, steps, warmup, flush, stream, hold=True):
+    """Per-step device time.  With hold, a short spin kernel is queued after the
+    L2 flush so the step's launches are already enqueued when its start event
+    fires: the events then bracket device work, not host enqueue latency."""
     for _ in range(warmup):
         fn()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     for a, b in ev:
         flush()
+        if hold:
+            torch.cuda._sleep(HOLD_CYCLES)
         a.record(stream)
         fn()
         b.record(stream)
@@ -240,6 +248,7 @@ def time_staged(staged, steps, flush, stream):
     per = {n: [] for n, _ in st}
     for _ in range(steps):
         flush()
+        torch.cuda._sleep(HOLD_CYCLES)
         evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(st) + 1)]
         evs[0].record(stream)
         for i, (_, f) in enumerate(st):
@@ -384,7 +393,7 @@ def run_ours(args, rank, world, dev):
     def step_host():
         gg.moe_forward_host(cfg, xh, inp["W_r"], inp["bias"], weights, oh, ws)
 
-    e2e_times = time_steps(step_host, max(3, args.steps // 2), 2, flush, stream)
+    e2e_times = time_steps(step_host, max(3, args.steps // 2), 2, flush, stream, hold=False)
     e2e_ms = float(np.mean(e2e_times))
     if world > 1:
         t = torch.tensor([e2e_ms], device=dev)

@@ -62,8 +62,14 @@ struct Params {
   int G_total;  // groups, including the extra one
   int G_main;   // groups whose weights come from tmB; group G_main (if any) uses tmBx
   int N, K, rows;
+  int ksplit;          // K is split into this many slices (fp32 partial outputs, no gate)
+  size_t split_stride; // elements between the partial outputs of consecutive slices
   void* C;
   int* status;
+};
+
+struct TileCoord {
+  int g, mb, nb, ks, m_g;
 };
 
 // Largest g in [0, G) with tile_start[g] <= tile.
@@ -77,6 +83,20 @@ __device__ __forceinline__ int find_group(const int* tile_start, int G, int tile
       hi = mid - 1;
   }
   return lo;
+}
+
+// Tile t of group g: m-block fastest, then n-block, then K slice.
+__device__ __forceinline__ TileCoord decode_tile(const int* s_tile, const int* s_off, int G, int nt, int tile) {
+  TileCoord c;
+  c.g = find_group(s_tile, G, tile);
+  c.m_g = s_off[c.g + 1] - s_off[c.g];
+  const int mt = (c.m_g + BM - 1) / BM;
+  const int tl = tile - s_tile[c.g];
+  const int q = tl / mt;
+  c.mb = tl % mt;
+  c.ks = q / nt;
+  c.nb = q % nt;
+  return c;
 }
 
 template <int MMA_N, int EPI, int OUT>
@@ -105,10 +125,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G_total;
   const int nt = p.N / OUT_COLS;
+  const int ntk = nt * p.ksplit;  // tiles per m-block
 
   // ---- group tables: row offsets and the exclusive prefix of tile counts
   if (warp == 0) {
-    for (int g = lane; g <= G; g += 32) s_off[g] = p.offsets[g];
+    // no offsets array: a single group spanning every row of A
+    for (int g = lane; g <= G; g += 32) s_off[g] = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
     __syncwarp();
     const int per = (G + 31) / 32;
     const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
@@ -116,7 +138,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int g = g0; g < g1; ++g) {
       const int m = s_off[g + 1] - s_off[g];
       if (m < 0) bad = 1;
-      mine += (max(m, 0) + BM - 1) / BM * nt;
+      mine += (max(m, 0) + BM - 1) / BM * ntk;
     }
     int incl = mine;
 #pragma unroll
@@ -127,7 +149,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     int run = incl - mine;
     for (int g = g0; g < g1; ++g) {
       s_tile[g] = run;
-      run += (max(s_off[g + 1] - s_off[g], 0) + BM - 1) / BM * nt;
+      run += (max(s_off[g + 1] - s_off[g], 0) + BM - 1) / BM * ntk;
     }
     if (lane == 31) s_tile[G] = incl;
     if (lane == 0 && (s_off[0] != 0 || s_off[G] > p.rows)) bad = 1;
@@ -174,16 +196,14 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued = 0;
       bool ok = true;
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
-        const int g = find_group(s_tile, G, tile);
-        const int m_g = s_off[g + 1] - s_off[g];
-        const int mt = (m_g + BM - 1) / BM;
-        const int tl = tile - s_tile[g];
-        const int nb = tl / mt, mb = tl % mt;
-        const int a_row = s_off[g] + mb * BM;
+        const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+        const int g = tc.g, nb = tc.nb;
+        const int a_row = s_off[g] + tc.mb * BM;
         const bool extra = g >= p.G_main;
         const CUtensorMap* mB = extra ? &tmBx : &tmB;
         const int gb = extra ? 0 : g;
-        for (int kb = 0; kb < nk; ++kb) {
+        const int kb0 = tc.ks * nk / p.ksplit, kb1 = (tc.ks + 1) * nk / p.ksplit;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
@@ -237,7 +257,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MMA_N;
-        for (int kb = 0; kb < nk; ++kb) {
+        const int ks = decode_tile(s_tile, s_off, G, nt, tile).ks;
+        const int kb0 = ks * nk / p.ksplit, kb1 = (ks + 1) * nk / p.ksplit;
+        for (int kb = kb0; kb < kb1; ++kb) {
           if (!ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
@@ -247,7 +269,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sB + stage * L::B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | kk) != 0);
+            ptx::umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb > kb0) || (kk > 0));
           ptx::umma_commit(&empty[stage]);
           if (++stage == L::STAGES) {
             stage = 0;
@@ -274,12 +296,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
       const int acc = it & 1;
       const uint32_t use = static_cast<uint32_t>(it >> 1);
-      const int g = find_group(s_tile, G, tile);
-      const int m_g = s_off[g + 1] - s_off[g];
-      const int mt = (m_g + BM - 1) / BM;
-      const int tl = tile - s_tile[g];
-      const int nb = tl / mt, mb = tl % mt;
-      const int r_in = mb * BM + row_t;
+      const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+      const int g = tc.g, nb = tc.nb, m_g = tc.m_g;
+      const int r_in = tc.mb * BM + row_t;
       const bool valid = r_in < m_g;
       const size_t grow = static_cast<size_t>(s_off[g] + r_in);
       if (!ptx::mbar_wait_warp(&tfull[acc], use & 1, abort_flag, kWaitLimitNs)) {
@@ -321,7 +340,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           ptx::tmem_ld_wait();
           if (valid) {
             if constexpr (OUT == 1) {
-              float* C = static_cast<float*>(p.C) + grow * p.N + nb * OUT_COLS + c;
+              float* C = static_cast<float*>(p.C) + tc.ks * p.split_stride + grow * p.N + nb * OUT_COLS + c;
               uint4* dst = reinterpret_cast<uint4*>(C);
 #pragma unroll
               for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
@@ -413,6 +432,8 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   p.N = a.N;
   p.K = a.K;
   p.rows = a.rows;
+  p.ksplit = a.ksplit > 1 ? a.ksplit : 1;
+  p.split_stride = static_cast<size_t>(a.rows) * a.N;
   p.C = a.C;
   p.status = a.status;
   gg_bf16_kernel<MMA_N, EPI, OUT><<<num_sms(), kThreads, L::SMEM, s>>>(mA, mB, mBx, p);
@@ -425,14 +446,16 @@ int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.G + a.has_extra == 0 || a.rows == 0) return MOE_OK;
   if (a.ab_dtype == MOE_BF16) {
     if (a.epilogue == MOE_EPI_SILU_GATE) {
-      if (a.c_dtype == MOE_BF16 && a.N % 128 == 0) return run_bf16<256, 1, 0>(a, s);
+      if (a.c_dtype == MOE_BF16 && a.N % 128 == 0 && a.ksplit <= 1) return run_bf16<256, 1, 0>(a, s);
       return MOE_ERR_UNSUPPORTED;
     }
     const int out = a.c_dtype == MOE_F32 ? 1 : 0;
     if (a.c_dtype != MOE_F32 && a.c_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    if (a.N % 256 == 0) return out ? run_bf16<256, 0, 1>(a, s) : run_bf16<256, 0, 0>(a, s);
-    if (a.N % 128 == 0) return out ? run_bf16<128, 0, 1>(a, s) : run_bf16<128, 0, 0>(a, s);
-    if (a.N % 64 == 0) return out ? run_bf16<64, 0, 1>(a, s) : run_bf16<64, 0, 0>(a, s);
+    if (a.ksplit > 1 && (!out || a.ksplit > a.K / 64)) return MOE_ERR_UNSUPPORTED;
+    const int want = a.mma_n;
+    if ((want == 0 || want == 256) && a.N % 256 == 0) return out ? run_bf16<256, 0, 1>(a, s) : run_bf16<256, 0, 0>(a, s);
+    if ((want == 0 || want == 128) && a.N % 128 == 0) return out ? run_bf16<128, 0, 1>(a, s) : run_bf16<128, 0, 0>(a, s);
+    if ((want == 0 || want == 64) && a.N % 64 == 0) return out ? run_bf16<64, 0, 1>(a, s) : run_bf16<64, 0, 0>(a, s);
     return MOE_ERR_UNSUPPORTED;
   }
   return MOE_ERR_UNSUPPORTED;  // E4M3 operands: see the FP8 kernel

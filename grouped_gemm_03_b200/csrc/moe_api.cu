@@ -54,7 +54,7 @@ FwdLayout fwd_layout(const moe_config& c) {
   L.status = take(256);
   L.idx = take(T * k * 4);
   L.w = take(T * k * 4);
-  L.logits = take(T * E * 4);
+  L.logits = take(kRouterMaxSplit * T * E * 4);
   L.base = take(static_cast<size_t>(permute_blocks(c.T)) * E * 4);
   L.counts = take(E * 4);
   L.offsets = take((E + 2) * 4);
@@ -127,7 +127,7 @@ int moe_read_device_status(const void* ws, void* stream, int* status) {
 
 // ------------------------------------------------------------------ router
 size_t moe_router_workspace_size(int T, int E) {
-  return 256 + align_up(static_cast<size_t>(T > 0 ? T : 0) * (E > 0 ? E : 0) * 4, 256);
+  return 256 + align_up(static_cast<size_t>(kRouterMaxSplit) * (T > 0 ? T : 0) * (E > 0 ? E : 0) * 4, 256);
 }
 
 int moe_router_topk(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d,
@@ -143,8 +143,8 @@ int moe_router_topk(const void* x, int x_dtype, const void* W_r, int w_dtype, co
   if (!aligned(x, 16) || !aligned(W_r, 16)) return MOE_ERR_INVALID;
   cudaStream_t s = as_stream(stream);
   MOE_CUDA_CHECK(cudaMemsetAsync(ws, 0, sizeof(int), s));
-  return launch_router_simt(x, x_dtype, W_r, w_dtype, bias, T, d, E, k, renormalize, logits_out, topk_idx, topk_w,
-                            s);
+  return launch_router(x, x_dtype, W_r, w_dtype, bias, T, d, E, k, renormalize, logits_out, topk_idx, topk_w,
+                       reinterpret_cast<float*>(static_cast<char*>(ws) + 256), static_cast<int*>(ws), s);
 }
 
 int moe_topk_logits(const void* logits, int dtype, int N, int E, int k, int renormalize, int32_t* topk_idx,
@@ -299,8 +299,8 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   const int T = c.T, d = c.d, E = c.E, k = c.k, I = c.inter;
   const int Rp = T * k + (shared ? T : 0);
 
-  st = launch_router_simt(x, c.x_dtype, W_r, c.router_dtype, router_bias, T, d, E, k, c.renormalize, nullptr, idx,
-                          w, s);
+  st = launch_router(x, c.x_dtype, W_r, c.router_dtype, router_bias, T, d, E, k, c.renormalize, nullptr, idx, w,
+                     reinterpret_cast<float*>(base + L.logits), status, s);
   if (st != MOE_OK) return st;
 
   PermuteArgs pa;

@@ -2,12 +2,17 @@
 //
 // "MegaMoE math model -> DeepGEMM source walk-through" §2.1 (p = Softmax(W_r x_t),
 // keep the k best) and "Dense GEMM -> GroupedGEMM -> TP MoE" §4.2 (route_tokens).
-// One warp owns one token: the dot products are split over the lanes along d
-// and reduced with shuffles, then k rounds of a warp-wide arg-max on
-// (logit descending, expert index ascending) pick the experts.  Selection
-// compares logits, so equal probabilities never reorder it; the weight of a
-// selected expert is its softmax value (or that value over the sum of the
-// selected ones when renormalising).
+// Two launches:
+//   logits  either the grouped-GEMM kernel on the tensor cores (bf16, large
+//           E and d: the logits GEMM is then near the compute ridge), split
+//           along K into fp32 partial products, or a SIMT kernel that keeps
+//           a block's W_r rows in shared memory (small E or d, fp32 inputs);
+//   finish  one warp per token sums the partials in a fixed order, adds the
+//           bias, and runs k rounds of a warp-wide arg-max on (logit
+//           descending, expert index ascending) for the softmax + top-k.
+// Selection compares logits, so equal probabilities never reorder it; the
+// weight of a selected expert is its softmax value (or that value over the
+// sum of the selected ones when renormalising).
 #include <cfloat>
 #include <climits>
 
@@ -81,7 +86,8 @@ __device__ __forceinline__ void warp_select(float (&v)[V], const int (&ix)[V], i
   }
 }
 
-// 8 consecutive elements as fp32 (16- or 32-byte vector loads).
+
+// 8 consecutive elements as fp32.
 __device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
   const float4 a = __ldg(reinterpret_cast<const float4*>(p));
   const float4 b = __ldg(reinterpret_cast<const float4*>(p) + 1);
@@ -97,174 +103,223 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
     f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
   }
 }
-constexpr int kRouterWarps = 8;
 
-// Fused logits + softmax + top-k, one warp per token.
-template <typename XT, typename WT, int V>
-__global__ void __launch_bounds__(kRouterWarps * 32) router_simt_kernel(
-    const XT* __restrict__ x, const WT* __restrict__ Wr, const float* __restrict__ bias, int T, int d, int E,
-    int k, int renorm, float* __restrict__ logits_out, int32_t* __restrict__ idx_out,
-    float* __restrict__ w_out) {
-  extern __shared__ float s_logit[];  // [kRouterWarps][E]
+// ------------------------------------------------------------------ SIMT logits
+// Block = 32 tokens x 8 experts; each warp owns 4 tokens.  W_r rows of the
+// block's experts are staged (as fp32) in shared memory 512 columns at a time,
+// so every block reads them once from L2 while x streams from HBM once per
+// expert block.  Used when E or d is small (the logits are then bound by
+// reading x) and for fp32 operands.
+constexpr int kRTok = 32;
+constexpr int kREC = 8;
+constexpr int kRDC = 512;
+
+template <typename XT, typename WT>
+__global__ void __launch_bounds__(256) logits_simt_kernel(const XT* __restrict__ x, const WT* __restrict__ Wr,
+                                                          int T, int d, int E, float* __restrict__ logits) {
+  __shared__ __align__(16) float s_w[kREC][kRDC];
+  const int t0 = blockIdx.x * kRTok, e0 = blockIdx.y * kREC;
+  const int ne = min(kREC, E - e0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  float* lg = s_logit + warp * E;
-  for (int t = blockIdx.x * kRouterWarps + warp; t < T; t += gridDim.x * kRouterWarps) {
-    const XT* xr = x + static_cast<size_t>(t) * d;
-    for (int e0 = 0; e0 < E; e0 += 8) {
-      const int ne = min(8, E - e0);
-      float acc[8];
+  const int tw = t0 + warp * 4;
+  float acc[4][kREC];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = 0.f;
-      for (int c = lane * 8; c < d; c += 32 * 8) {
-        float xv[8];
-        load8(xr + c, xv);
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          if (j < ne) {
-            float wv[8];
-            load8(Wr + static_cast<size_t>(e0 + j) * d + c, wv);
+    for (int e = 0; e < kREC; ++e) acc[i][e] = 0.f;
+  for (int c0 = 0; c0 < d; c0 += kRDC) {
+    const int dc = min(kRDC, d - c0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < kREC * (kRDC / 8); i += blockDim.x) {
+      const int e = i / (kRDC / 8), c = (i % (kRDC / 8)) * 8;
+      float f[8];
+      if (e < ne && c < dc) {
+        load8(Wr + static_cast<size_t>(e0 + e) * d + c0 + c, f);
+      } else {
 #pragma unroll
-            for (int q = 0; q < 8; ++q) acc[j] = fmaf(xv[q], wv[q], acc[j]);
-          }
+        for (int q = 0; q < 8; ++q) f[q] = 0.f;
+      }
+      float4* dst = reinterpret_cast<float4*>(&s_w[e][c]);
+      dst[0] = make_float4(f[0], f[1], f[2], f[3]);
+      dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+    }
+    __syncthreads();
+    for (int c = lane * 8; c < dc; c += 256) {
+      float xv[4][8];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        if (tw + i < T) {
+          load8(x + static_cast<size_t>(tw + i) * d + c0 + c, xv[i]);
+        } else {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) xv[i][q] = 0.f;
         }
       }
 #pragma unroll
-      for (int j = 0; j < 8; ++j) acc[j] = warp_sum(acc[j]);
-      if (lane < ne) {
-        float a = acc[0];
+      for (int e = 0; e < kREC; ++e) {
+        const float4 wa = *reinterpret_cast<const float4*>(&s_w[e][c]);
+        const float4 wb = *reinterpret_cast<const float4*>(&s_w[e][c + 4]);
+        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
 #pragma unroll
-        for (int j = 1; j < 8; ++j)
-          if (lane == j) a = acc[j];
-        lg[e0 + lane] = a + (bias ? bias[e0 + lane] : 0.f);
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int q = 0; q < 8; ++q) acc[i][e] = fmaf(xv[i][q], wv[q], acc[i][e]);
       }
     }
-    __syncwarp();
+  }
+  float mine = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int e = 0; e < kREC; ++e) {
+      const float v = warp_sum(acc[i][e]);
+      if (lane == i * kREC + e) mine = v;
+    }
+  const int t = tw + lane / kREC, e = lane % kREC;
+  if (t < T && e < ne) logits[static_cast<size_t>(t) * E + e0 + e] = mine;
+}
+
+// ------------------------------------------------------------------ finish
+// Sum the K-slice partial logits in slice order, add the bias, optionally
+// store the logits, then softmax + top-k.  One warp per token; lane l holds
+// experts l*V .. l*V+V-1.
+template <typename LT, int V>
+__global__ void __launch_bounds__(256) finish_kernel(const LT* __restrict__ parts, int nsplit, size_t split_stride,
+                                                     const float* __restrict__ bias, int N, int E, int k, int renorm,
+                                                     float* __restrict__ logits_out, int32_t* __restrict__ idx_out,
+                                                     float* __restrict__ w_out) {
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
+  const bool vec = (E == 32 * V) && ((V * sizeof(LT)) % 8 == 0) && ((V * sizeof(LT)) <= 32);
+  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < N; t += warps) {
     float v[V];
     int ix[V];
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-      const int e = lane + 32 * i;
-      ix[i] = e < E ? e : INT_MAX;
-      v[i] = e < E ? lg[e] : -INFINITY;
+      v[i] = 0.f;
+      ix[i] = lane * V + i < E ? lane * V + i : INT_MAX;
     }
-    if (logits_out)
-      for (int e = lane; e < E; e += 32) logits_out[static_cast<size_t>(t) * E + e] = lg[e];
-    warp_select<V>(v, ix, k, renorm, lane, idx_out + static_cast<size_t>(t) * k,
-                   w_out + static_cast<size_t>(t) * k);
-    __syncwarp();
-  }
-}
-
-// Softmax + top-k of stored logits, one warp per token; lane l holds the
-// V consecutive experts l*V .. l*V+V-1.
-template <typename LT, int V>
-__global__ void __launch_bounds__(256) topk_logits_kernel(const LT* __restrict__ logits, int N, int E, int k,
-                                                          int renorm, int32_t* __restrict__ idx_out,
-                                                          float* __restrict__ w_out) {
-  const int lane = threadIdx.x & 31;
-  const int warps = gridDim.x * (blockDim.x >> 5);
-  const bool vec = (E == 32 * V) && (V * sizeof(LT)) % 8 == 0;
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < N; t += warps) {
-    const LT* row = logits + static_cast<size_t>(t) * E;
-    float v[V];
-    int ix[V];
-    if (vec && V * sizeof(LT) == 8) {
-      const uint2 raw = __ldg(reinterpret_cast<const uint2*>(row) + lane);
-      const LT* pv = reinterpret_cast<const LT*>(&raw);
+    for (int sp = 0; sp < nsplit; ++sp) {
+      const LT* row = parts + sp * split_stride + static_cast<size_t>(t) * E;
+      if (vec) {
+        constexpr int kWords = (V * sizeof(LT) + 7) / 8;  // 8-byte words per lane
+        uint2 raw[kWords > 0 ? kWords : 1];
 #pragma unroll
-      for (int i = 0; i < V; ++i) {
-        v[i] = to_f32(pv[i]);
-        ix[i] = lane * V + i;
+        for (int wd = 0; wd < kWords; ++wd) raw[wd] = __ldg(reinterpret_cast<const uint2*>(row + lane * V) + wd);
+        const LT* pv = reinterpret_cast<const LT*>(raw);
+#pragma unroll
+        for (int i = 0; i < V; ++i) v[i] += to_f32(pv[i]);
+      } else {
+#pragma unroll
+        for (int i = 0; i < V; ++i)
+          if (ix[i] != INT_MAX) v[i] += to_f32(row[ix[i]]);
       }
-    } else if (vec && V * sizeof(LT) == 16) {
-      const uint4 raw = __ldg(reinterpret_cast<const uint4*>(row) + lane);
-      const LT* pv = reinterpret_cast<const LT*>(&raw);
+    }
 #pragma unroll
-      for (int i = 0; i < V; ++i) {
-        v[i] = to_f32(pv[i]);
-        ix[i] = lane * V + i;
-      }
-    } else {
-#pragma unroll
-      for (int i = 0; i < V; ++i) {
-        const int e = lane * V + i;
-        ix[i] = e < E ? e : INT_MAX;
-        v[i] = e < E ? to_f32(row[e]) : -INFINITY;
+    for (int i = 0; i < V; ++i) {
+      if (ix[i] == INT_MAX) {
+        v[i] = -INFINITY;
+      } else {
+        if (bias) v[i] += bias[ix[i]];
+        if (logits_out) logits_out[static_cast<size_t>(t) * E + ix[i]] = v[i];
       }
     }
     warp_select<V>(v, ix, k, renorm, lane, idx_out + static_cast<size_t>(t) * k,
                    w_out + static_cast<size_t>(t) * k);
   }
-}
-
-template <typename XT, typename WT>
-int router_dispatch(const void* x, const void* Wr, const float* bias, int T, int d, int E, int k, int renorm,
-                    float* lo, int32_t* idx, float* w, cudaStream_t s) {
-  const int blocks = min((T + kRouterWarps - 1) / kRouterWarps, num_sms() * 8);
-  const size_t smem = static_cast<size_t>(kRouterWarps) * E * sizeof(float);
-  const XT* xp = static_cast<const XT*>(x);
-  const WT* wp = static_cast<const WT*>(Wr);
-  const int v = (E + 31) / 32;
-#define MOE_ROUTER_CASE(VV)                                                                                  \
-  if (v <= VV) {                                                                                            \
-    router_simt_kernel<XT, WT, VV><<<blocks, kRouterWarps * 32, smem, s>>>(xp, wp, bias, T, d, E, k, renorm, \
-                                                                          lo, idx, w);                     \
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;                                       \
-  }
-  MOE_ROUTER_CASE(1)
-  MOE_ROUTER_CASE(2)
-  MOE_ROUTER_CASE(4)
-  MOE_ROUTER_CASE(8)
-  MOE_ROUTER_CASE(16)
-  MOE_ROUTER_CASE(32)
-#undef MOE_ROUTER_CASE
-  return MOE_ERR_UNSUPPORTED;
 }
 
 template <typename LT>
-int topk_dispatch(const void* logits, int N, int E, int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
+int finish_dispatch(const void* parts, int nsplit, size_t stride, const float* bias, int N, int E, int k,
+                    int renorm, float* lo, int32_t* idx, float* w, cudaStream_t s) {
   const int warps_per_block = 8;
   const int blocks = max(1, min((N + warps_per_block - 1) / warps_per_block, num_sms() * 16));
-  const LT* lp = static_cast<const LT*>(logits);
+  const LT* lp = static_cast<const LT*>(parts);
   const int v = (E + 31) / 32;
-#define MOE_TOPK_CASE(VV)                                                                                    \
-  if (v <= VV) {                                                                                            \
-    topk_logits_kernel<LT, VV><<<blocks, warps_per_block * 32, 0, s>>>(lp, N, E, k, renorm, idx, w);         \
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;                                       \
+#define MOE_FINISH_CASE(VV)                                                                                   \
+  if (v <= VV) {                                                                                             \
+    finish_kernel<LT, VV><<<blocks, warps_per_block * 32, 0, s>>>(lp, nsplit, stride, bias, N, E, k, renorm, lo, \
+                                                                 idx, w);                                    \
+    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;                                        \
   }
-  MOE_TOPK_CASE(1)
-  MOE_TOPK_CASE(2)
-  MOE_TOPK_CASE(4)
-  MOE_TOPK_CASE(8)
-  MOE_TOPK_CASE(16)
-  MOE_TOPK_CASE(32)
-#undef MOE_TOPK_CASE
+  MOE_FINISH_CASE(1)
+  MOE_FINISH_CASE(2)
+  MOE_FINISH_CASE(4)
+  MOE_FINISH_CASE(8)
+  MOE_FINISH_CASE(16)
+  MOE_FINISH_CASE(32)
+#undef MOE_FINISH_CASE
   return MOE_ERR_UNSUPPORTED;
+}
+
+template <typename XT, typename WT>
+int simt_logits(const void* x, const void* Wr, int T, int d, int E, float* logits, cudaStream_t s) {
+  dim3 grid((T + kRTok - 1) / kRTok, (E + kREC - 1) / kREC);
+  logits_simt_kernel<XT, WT><<<grid, 256, 0, s>>>(static_cast<const XT*>(x), static_cast<const WT*>(Wr), T, d, E,
+                                                  logits);
+  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
 }
 
 }  // namespace
 
-int launch_router_simt(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T,
-                       int d, int E, int k, int renorm, float* logits_out, int32_t* idx, float* w,
-                       cudaStream_t s) {
+// Tensor-core router: x [T, d] x W_r[E, d]^T on the grouped GEMM kernel (one
+// group, fp32 output), split along K so that about one tile per SM is
+// in flight; the slices' partial logits are summed in slice order by the
+// finish kernel, so the result does not depend on scheduling.
+bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E) {
+  return x_dtype == MOE_BF16 && w_dtype == MOE_BF16 && E % 64 == 0 && d % 64 == 0 && T >= 256 && E >= 64 &&
+         d >= 1024;
+}
+
+int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d, int E,
+                  int k, int renorm, float* logits_out, int32_t* idx, float* w, float* parts, int* status,
+                  cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  if (x_dtype == MOE_BF16 && w_dtype == MOE_BF16)
-    return router_dispatch<__nv_bfloat16, __nv_bfloat16>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
-  if (x_dtype == MOE_F32 && w_dtype == MOE_F32)
-    return router_dispatch<float, float>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
-  if (x_dtype == MOE_F32 && w_dtype == MOE_BF16)
-    return router_dispatch<float, __nv_bfloat16>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
-  if (x_dtype == MOE_BF16 && w_dtype == MOE_F32)
-    return router_dispatch<__nv_bfloat16, float>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
-  return MOE_ERR_UNSUPPORTED;
+  int nsplit = 1;
+  int st;
+  if (router_uses_tensor_cores(x_dtype, w_dtype, T, d, E)) {
+    const int mma_n = E % 256 == 0 ? 256 : (E % 128 == 0 ? 128 : 64);
+    const int tiles = (T + 127) / 128 * (E / mma_n);
+    nsplit = max(1, min(kRouterMaxSplit, min(num_sms() / max(tiles, 1), d / 64 / 4)));
+    GemmArgs g{};
+    g.A = x;
+    g.B = W_r;
+    g.offsets = nullptr;  // one group: all T rows
+    g.G = 1;
+    g.rows = T;
+    g.N = E;
+    g.K = d;
+    g.ksplit = nsplit;
+    g.mma_n = mma_n;
+    g.ab_dtype = MOE_BF16;
+    g.epilogue = MOE_EPI_NONE;
+    g.c_dtype = MOE_F32;
+    g.C = parts;
+    g.status = status;
+    st = launch_grouped_gemm(g, s);
+  } else if (x_dtype == MOE_BF16 && w_dtype == MOE_BF16) {
+    st = simt_logits<__nv_bfloat16, __nv_bfloat16>(x, W_r, T, d, E, parts, s);
+  } else if (x_dtype == MOE_F32 && w_dtype == MOE_F32) {
+    st = simt_logits<float, float>(x, W_r, T, d, E, parts, s);
+  } else if (x_dtype == MOE_F32 && w_dtype == MOE_BF16) {
+    st = simt_logits<float, __nv_bfloat16>(x, W_r, T, d, E, parts, s);
+  } else if (x_dtype == MOE_BF16 && w_dtype == MOE_F32) {
+    st = simt_logits<__nv_bfloat16, float>(x, W_r, T, d, E, parts, s);
+  } else {
+    return MOE_ERR_UNSUPPORTED;
+  }
+  if (st != MOE_OK) return st;
+  return finish_dispatch<float>(parts, nsplit, static_cast<size_t>(T) * E, bias, T, E, k, renorm, logits_out, idx, w,
+                                s);
 }
 
 int launch_topk_logits(const void* logits, int dtype, int N, int E, int k, int renorm, int32_t* idx, float* w,
                        cudaStream_t s) {
   if (N == 0) return MOE_OK;
-  if (dtype == MOE_F16) return topk_dispatch<__half>(logits, N, E, k, renorm, idx, w, s);
-  if (dtype == MOE_F32) return topk_dispatch<float>(logits, N, E, k, renorm, idx, w, s);
-  if (dtype == MOE_BF16) return topk_dispatch<__nv_bfloat16>(logits, N, E, k, renorm, idx, w, s);
+  if (dtype == MOE_F16) return finish_dispatch<__half>(logits, 1, 0, nullptr, N, E, k, renorm, nullptr, idx, w, s);
+  if (dtype == MOE_F32) return finish_dispatch<float>(logits, 1, 0, nullptr, N, E, k, renorm, nullptr, idx, w, s);
+  if (dtype == MOE_BF16)
+    return finish_dispatch<__nv_bfloat16>(logits, 1, 0, nullptr, N, E, k, renorm, nullptr, idx, w, s);
   return MOE_ERR_UNSUPPORTED;
 }
 

@@ -66,7 +66,8 @@ def test_topk_k1_renormalised_is_one():
 
 
 # ---------------------------------------------------------------- router
-@pytest.mark.parametrize("name,T", [("tiny", 256), ("mixtral", 512), ("decode", 128), ("fine", 256)])
+@pytest.mark.parametrize("name,T", [("tiny", 256), ("mixtral", 512), ("decode", 128), ("fine", 256), ("fine", 1000),
+                                    ("fine", 4096), ("mixtral", 4096), ("tiny", 77)])
 @pytest.mark.parametrize("renorm", [False, True])
 def test_router_topk(name, T, renorm):
     s = shape_of(name, T=T)
