@@ -356,7 +356,15 @@ def run_ours(args, rank, world, dev):
     inp = make_inputs(s, seed=1234 + rank, device=dev)
     cfg = make_cfg(gg, s)
     ws = torch.empty(gg.workspace_size(cfg) + gg.host_staging_size(cfg), dtype=torch.uint8, device=dev)
-    weights = gg.ExpertWeights(W1=inp["W1"], W2=inp["W2"], W1s=inp["W1s"], W2s=inp["W2s"])
+    if s.fp8:  # weights quantised once per 128x128 block (offline, outside the timed region)
+        W1q, W1sc = gg.quantize_weights_fp8(inp["W1"])
+        W2q, W2sc = gg.quantize_weights_fp8(inp["W2"])
+        weights = gg.ExpertWeights(W1=W1q, W2=W2q, W1_scales=W1sc, W2_scales=W2sc)
+        if s.shared_inter:
+            weights.W1s, weights.W1s_scales = gg.quantize_weights_fp8(inp["W1s"])
+            weights.W2s, weights.W2s_scales = gg.quantize_weights_fp8(inp["W2s"])
+    else:
+        weights = gg.ExpertWeights(W1=inp["W1"], W2=inp["W2"], W1s=inp["W1s"], W2s=inp["W2s"])
     out = torch.empty((s.T, s.d), dtype=torch.bfloat16 if s.x_dtype != "f32" else torch.float32, device=dev)
     counts = torch.empty(s.E, dtype=torch.int32, device=dev)
     l2 = torch.cuda.get_device_properties(dev).L2_cache_size

@@ -52,6 +52,7 @@ _CFG = ctypes.POINTER(MoEConfig)
 # name -> (restype, argtypes); the full C ABI of include/moe.h
 _SIGS = {
     "moe_status_string": (ctypes.c_char_p, [_i]),
+    "moe_last_error_string": (ctypes.c_char_p, []),
     "moe_device_info": (_i, [ctypes.POINTER(_i), ctypes.POINTER(_i), ctypes.POINTER(_i)]),
     "moe_read_device_status": (_i, [_vp, _vp, ctypes.POINTER(_i)]),
     "moe_router_workspace_size": (_sz, [_i, _i]),
@@ -101,6 +102,8 @@ def status_string(status: int) -> str:
 
 def _check(status: int, what: str) -> None:
     if status != 0:
+        if status == -4:
+            what = f"{what} [{lib().moe_last_error_string().decode()}]"
         raise MoEError(status, what)
 
 

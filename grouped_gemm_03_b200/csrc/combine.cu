@@ -72,7 +72,7 @@ int launch_combine(const void* Y, const int32_t* t2r, const float* w, int has_sh
   else
     combine_kernel<__nv_bfloat16>
         <<<T, kCombThreads, 0, s>>>(y, t2r, w, has_shared, T, d, k, static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_status(__func__);
 }
 
 }  // namespace moe

@@ -101,8 +101,18 @@ int num_sms();
 
 }  // namespace moe
 
-#define MOE_CUDA_CHECK(expr)                        \
-  do {                                              \
-    cudaError_t _e = (expr);                        \
-    if (_e != cudaSuccess) return MOE_ERR_CUDA;     \
+namespace moe {
+// Remember the last failing CUDA call (per host thread) for moe_last_error_string.
+int record_cuda_error(cudaError_t e, const char* where);
+// Status of the kernel launch just made.
+inline int launch_status(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : record_cuda_error(e, where);
+}
+}  // namespace moe
+
+#define MOE_CUDA_CHECK(expr)                                            \
+  do {                                                                  \
+    cudaError_t _e = (expr);                                            \
+    if (_e != cudaSuccess) return ::moe::record_cuda_error(_e, #expr);  \
   } while (0)

@@ -51,10 +51,11 @@ struct Tile {
   static constexpr int B_BYTES = MMA_N * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TABLE_BYTES = 2 * (kMaxGroups + 2) * 4;
-  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512) / STAGE_BYTES;
+  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512 - 2048) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = 2 * MMA_N;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES;
+  static constexpr int EXTRA_BYTES = 2048;  // amax exchange of the E4M3 epilogue
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES + EXTRA_BYTES;
 };
 
 struct Params {
@@ -66,6 +67,11 @@ struct Params {
   size_t split_stride; // elements between the partial outputs of consecutive slices
   void* C;
   int* status;
+  // E4M3 operands only
+  const float* A_scales;   // [K/128][rows]
+  const float* B_scales;   // [G_main][Nb/128][K/128]
+  const float* Bx_scales;  // [Nb/128][K/128] of the extra group
+  float* C_scales;         // [N/128][rows] when C is E4M3
 };
 
 struct TileCoord {
@@ -374,6 +380,329 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ FP8 (E4M3) kernel
+// Same persistent structure; operands are E4M3 with fp32 scales that vary
+// along K ("MegaMoE ..." §2.3 / §5.1: 1x128 per token, 128x128 per weight
+// block), so one K block of 128 is one pipeline stage and the scales are
+// applied per K block ("promotion"): the MMA warp writes each block's partial
+// product A_kb B_kb^T into one of two TMEM buffers (kind::f8f6f4, 128 x 256
+// x 32 per instruction) and eight epilogue warps fold it into fp32 registers,
+//     acc[m][n] += partial[m][n] * sa[m, kb] * sb[n/128, kb],
+// while the MMA fills the other buffer.  Epilogue thread = one row and half
+// of the tile's 256 columns: with the SiLU gate, half h owns gate columns
+// [64h, 64h+64) and the matching up columns, so silu(g)*u stays in-thread;
+// the E4M3 output (per row per 128 columns) exchanges the two halves' amax
+// through shared memory under an mbarrier.
+constexpr int kThreadsF8 = 320;
+
+template <int EPI, int OUT>  // EPI 1: SiLU gate (OUT 0 bf16 / 2 e4m3); EPI 0: OUT 0 bf16
+__global__ void __launch_bounds__(kThreadsF8, 1)
+    gg_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                  const __grid_constant__ CUtensorMap tmBx, const Params p) {
+  constexpr int MMA_N = 256;
+  using L = Tile<MMA_N>;
+  constexpr int OUT_COLS = EPI ? 128 : 256;
+  constexpr uint32_t IDESC = ptx::make_idesc(BM, MMA_N, 0);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + L::STAGES * L::A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + L::STAGES * L::B_BYTES);
+  uint64_t* empty = full + L::STAGES;
+  uint64_t* pfull = empty + L::STAGES;
+  uint64_t* pempty = pfull + 2;
+  uint64_t* xchg = pempty + 2;
+  uint64_t* drain = xchg + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + L::STAGES * L::STAGE_BYTES + 512);
+  int* s_tile = s_off + kMaxGroups + 2;
+  float* s_amax = reinterpret_cast<float*>(s_tile + kMaxGroups + 2);  // [2 parity][2 halves][128 rows]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G_total;
+  const int nt = p.N / OUT_COLS;
+
+  if (warp == 0) {
+    for (int g = lane; g <= G; g += 32) s_off[g] = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
+    __syncwarp();
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int bad = 0, mine = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int m = s_off[g + 1] - s_off[g];
+      if (m < 0) bad = 1;
+      mine += (max(m, 0) + BM - 1) / BM * nt;
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - mine;
+    for (int g = g0; g < g1; ++g) {
+      s_tile[g] = run;
+      run += (max(s_off[g + 1] - s_off[g], 0) + BM - 1) / BM * nt;
+    }
+    if (lane == 31) s_tile[G] = incl;
+    if (lane == 0 && (s_off[0] != 0 || s_off[G] > p.rows)) bad = 1;
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      *s_bad = bad;
+      *abort_flag = 0;
+      if (bad && blockIdx.x == 0) set_status(p.status, MOE_ERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  if (*s_bad) return;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&pfull[a], 1);
+      ptx::mbar_init(&pempty[a], 256);
+    }
+    ptx::mbar_init(xchg, 256);
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+    ptx::prefetch_tmap(&tmBx);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, L::TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tile[G];
+  const int nk = p.K / 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+        const int g = tc.g, nb = tc.nb;
+        const int a_row = s_off[g] + tc.mb * BM;
+        const bool extra = g >= p.G_main;
+        const CUtensorMap* mB = extra ? &tmBx : &tmB;
+        const int gb = extra ? 0 : g;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+          ptx::tma_load_2d(sA + stage * L::A_BYTES, &tmA, &full[stage], kb * 128, a_row);
+          if (EPI) {
+            const int brow = gb * 2 * p.N + nb * 128;
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, brow);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES + 128 * 128, mB, &full[stage], kb * 128, brow + p.N);
+          } else {
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, gb * p.N + nb * 256);
+          }
+          ++issued;
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        const uint32_t pending = issued < static_cast<uint32_t>(L::STAGES) ? issued : L::STAGES;
+        uint32_t s = stage, ph = phase;
+        for (uint32_t i = 0; i < pending; ++i) {
+          if (s == 0) {
+            s = L::STAGES - 1;
+            ph ^= 1;
+          } else {
+            --s;
+          }
+          ptx::mbar_wait(&full[s], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t stage = 0, phase = 0;
+      uint32_t pb = 0, puse = 0;  // partial buffer and how many times the pair was cycled
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&pempty[pb], (puse & 1) ^ 1, abort_flag, kWaitLimitNs) ||
+              !ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t d_tmem = tmem_base + pb * MMA_N;
+          const uint64_t adesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sA + stage * L::A_BYTES));
+          const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sB + stage * L::B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk) ptx::umma_f8(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, kk > 0);
+          ptx::umma_commit(&empty[stage]);
+          ptx::umma_commit(&pfull[pb]);
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+          pb ^= 1;
+          if (pb == 0) ++puse;
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+      }
+      ptx::umma_commit(drain);
+      ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (8 warps)
+    const int q = warp & 3;
+    const int h = (warp - 2) >> 2;  // column half
+    const int row_t = q * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    // TMEM column offsets of this thread's two 64-column pieces (gate, up) or its 128 columns
+    const int c_lo = EPI ? h * 64 : h * 128;
+    const int c_hi = EPI ? 128 + h * 64 : h * 128 + 64;
+    const int nbk = p.K / 128;
+    uint32_t pb = 0, puse = 0;
+    int it = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+      const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+      const int g = tc.g, nb = tc.nb;
+      const int r_in = tc.mb * BM + row_t;
+      const bool valid = r_in < tc.m_g;
+      const size_t grow = static_cast<size_t>(s_off[g] + r_in);
+      const bool extra = g >= p.G_main;
+      const float* bsc = extra ? p.Bx_scales : p.B_scales + static_cast<size_t>(g) * ((EPI ? 2 : 1) * p.N / 128) * nbk;
+      // weight-block rows of the two column pieces
+      const int nblk_lo = EPI ? nb : 2 * nb + h;
+      const int nblk_hi = EPI ? p.N / 128 + nb : 2 * nb + h;
+      const float* sb_lo = bsc + static_cast<size_t>(nblk_lo) * nbk;
+      const float* sb_hi = bsc + static_cast<size_t>(nblk_hi) * nbk;
+      const float* sa_row = p.A_scales + grow;
+      float acc[128];
+#pragma unroll
+      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
+      float sa_next = valid ? __ldg(sa_row) : 0.f;
+      for (int kb = 0; kb < nbk; ++kb) {
+        const float sa = sa_next;
+        if (kb + 1 < nbk) sa_next = valid ? __ldg(sa_row + static_cast<size_t>(kb + 1) * p.rows) : 0.f;
+        const float m_lo = sa * __ldg(sb_lo + kb);
+        const float m_hi = sa * __ldg(sb_hi + kb);
+        if (!ptx::mbar_wait_warp(&pfull[pb], puse & 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t t0 = lane_base + pb * MMA_N;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          uint32_t v[16];
+          ptx::tmem_ld_32x32b_x16(t0 + (j < 4 ? c_lo : c_hi) + (j & 3) * 16, v);
+          ptx::tmem_ld_wait();
+          const float m = j < 4 ? m_lo : m_hi;
+#pragma unroll
+          for (int i = 0; i < 16; ++i) acc[16 * j + i] = fmaf(__uint_as_float(v[i]), m, acc[16 * j + i]);
+        }
+        ptx::tc_fence_before();
+        ptx::mbar_arrive(&pempty[pb]);
+        pb ^= 1;
+        if (pb == 0) ++puse;
+      }
+      if (!ok) break;
+      if constexpr (EPI == 1) {
+#pragma unroll
+        for (int i = 0; i < 64; ++i) {
+          const float gt = acc[i];
+          acc[i] = gt / (1.0f + __expf(-gt)) * acc[64 + i];
+        }
+        if constexpr (OUT == 2) {
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+          float* xa = s_amax + (it & 1) * 256;
+          xa[h * 128 + row_t] = amax;
+          ptx::mbar_arrive(xchg);
+          if (!ptx::mbar_wait_warp(xchg, it & 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          amax = fmaxf(xa[row_t], xa[128 + row_t]);
+          const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+          if (valid) {
+            uint32_t qw[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc));
+              const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc));
+              qw[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.C) + grow * p.N + nb * 128 + h * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(qw[4 * v], qw[4 * v + 1], qw[4 * v + 2], qw[4 * v + 3]);
+            if (h == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
+          }
+        } else {
+          if (valid) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
+              pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 128 + h * 64);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+          }
+        }
+      } else {
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 256 + h * 128);
+#pragma unroll
+          for (int v = 0; v < 16; ++v) {
+            uint32_t pk[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(acc[8 * v + 2 * i], acc[8 * v + 2 * i + 1]);
+              pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
+            }
+            dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+          }
+        }
+      }
+    }
+    if (!ok) {
+      *abort_flag = 1;
+      set_status(p.status, MOE_ERR_TIMEOUT);
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, L::TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -395,15 +724,23 @@ EncodeTiledFn get_encode_fn() {
 // 2-D K-major map over [rows, K] elements of `ebytes` bytes, box {128 B, box_rows}.
 bool make_map(CUtensorMap* m, const void* base, int ebytes, uint64_t rows, uint64_t K, uint32_t box_rows) {
   EncodeTiledFn enc = get_encode_fn();
-  if (!enc) return false;
+  if (!enc) {
+    record_cuda_error(cudaErrorNotSupported, "cuTensorMapEncodeTiled unavailable from the driver");
+    return false;
+  }
   const cuuint64_t dims[2] = {K, rows};
   const cuuint64_t strides[1] = {K * static_cast<uint64_t>(ebytes)};
   const cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / ebytes), box_rows};
   const cuuint32_t estr[2] = {1, 1};
   const CUtensorMapDataType dt = ebytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
-  return enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-             CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+  const CUresult r = enc(m, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    record_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled rejected the operand layout");
+    return false;
+  }
+  return true;
 }
 
 template <int MMA_N, int EPI, int OUT>
@@ -425,7 +762,7 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
                                         cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
     attr_set[dev] = true;
   }
-  Params p;
+  Params p{};
   p.offsets = a.offsets;
   p.G_total = a.G + a.has_extra;
   p.G_main = a.G;
@@ -437,7 +774,43 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   p.C = a.C;
   p.status = a.status;
   gg_bf16_kernel<MMA_N, EPI, OUT><<<num_sms(), kThreads, L::SMEM, s>>>(mA, mB, mBx, p);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_status(__func__);
+}
+
+template <int EPI, int OUT>
+int run_fp8(const GemmArgs& a, cudaStream_t s) {
+  using L = Tile<256>;
+  static_assert(L::SMEM <= 227 * 1024, "shared memory budget");
+  const int nb_rows = EPI ? 2 * a.N : a.N;
+  const uint32_t box_b = EPI ? 128 : 256;
+  CUtensorMap mA, mB, mBx;
+  if (!make_map(&mA, a.A, 1, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
+  if (!make_map(&mB, a.B, 1, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 1, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  MOE_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    MOE_CUDA_CHECK(cudaFuncSetAttribute(gg_fp8_kernel<EPI, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
+    attr_set[dev] = true;
+  }
+  Params p{};
+  p.offsets = a.offsets;
+  p.G_total = a.G + a.has_extra;
+  p.G_main = a.G;
+  p.N = a.N;
+  p.K = a.K;
+  p.rows = a.rows;
+  p.ksplit = 1;
+  p.C = a.C;
+  p.status = a.status;
+  p.A_scales = a.A_scales;
+  p.B_scales = a.B_scales;
+  p.Bx_scales = a.has_extra ? a.B_extra_scales : a.B_scales;
+  p.C_scales = a.C_scales;
+  gg_fp8_kernel<EPI, OUT><<<num_sms(), kThreadsF8, L::SMEM, s>>>(mA, mB, mBx, p);
+  return launch_status(__func__);
 }
 
 }  // namespace
@@ -458,7 +831,17 @@ int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
     if ((want == 0 || want == 64) && a.N % 64 == 0) return out ? run_bf16<64, 0, 1>(a, s) : run_bf16<64, 0, 0>(a, s);
     return MOE_ERR_UNSUPPORTED;
   }
-  return MOE_ERR_UNSUPPORTED;  // E4M3 operands: see the FP8 kernel
+  if (a.ab_dtype == MOE_E4M3) {
+    if (a.ksplit > 1 || !a.A_scales || !a.B_scales || (a.has_extra && !a.B_extra_scales)) return MOE_ERR_UNSUPPORTED;
+    if (a.epilogue == MOE_EPI_SILU_GATE && a.N % 128 == 0) {
+      if (a.c_dtype == MOE_E4M3) return a.C_scales ? run_fp8<1, 2>(a, s) : MOE_ERR_INVALID;
+      if (a.c_dtype == MOE_BF16) return run_fp8<1, 0>(a, s);
+      return MOE_ERR_UNSUPPORTED;
+    }
+    if (a.epilogue == MOE_EPI_NONE && a.N % 256 == 0 && a.c_dtype == MOE_BF16) return run_fp8<0, 0>(a, s);
+    return MOE_ERR_UNSUPPORTED;
+  }
+  return MOE_ERR_UNSUPPORTED;
 }
 
 }  // namespace moe

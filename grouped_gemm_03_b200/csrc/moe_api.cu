@@ -1,11 +1,21 @@
 // The C ABI (include/moe.h): argument validation, workspace layout and the
 // composition of the kernels into the layer forward.  Nothing here computes;
 // every step of the path runs in the kernels of the other translation units.
+#include <cstdio>
 #include <cstring>
 
 #include "common.cuh"
 
 namespace moe {
+
+namespace {
+thread_local char g_last_error[256] = "no error";
+}
+
+int record_cuda_error(cudaError_t e, const char* where) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s: %s (%d)", where, cudaGetErrorString(e), static_cast<int>(e));
+  return MOE_ERR_CUDA;
+}
 
 int num_sms() {
   static int cached[64] = {};
@@ -80,6 +90,7 @@ int check_config(const moe_config* c) {
   if (c->expert_dtype != MOE_BF16 && c->expert_dtype != MOE_E4M3) return MOE_ERR_INVALID;
   if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID;
   if (c->d % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->expert_dtype == MOE_E4M3 && c->d % 256 != 0) return MOE_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(c->T) * (c->k + 1);
   if (rows * c->d > (1ll << 40) || rows > (1ll << 30)) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -104,6 +115,8 @@ const char* moe_status_string(int s) {
     default: return "unknown moe status";
   }
 }
+
+const char* moe_last_error_string(void) { return g_last_error; }
 
 int moe_device_info(int* num_sms_out, int* cc_major, int* cc_minor) {
   int dev = 0, maj = 0, min_ = 0;
@@ -282,7 +295,6 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
   const FwdLayout L = fwd_layout(c);
   if (ws_bytes < L.total) return MOE_ERR_WORKSPACE;
-  if (fp8) return MOE_ERR_UNSUPPORTED;  // E4M3 expert GEMMs are provided by the FP8 kernel
   cudaStream_t s = as_stream(stream);
   char* base = static_cast<char*>(ws);
   int* status = reinterpret_cast<int*>(base + L.status);
@@ -334,11 +346,17 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   up.rows = Rp;
   up.N = I;
   up.K = d;
-  up.ab_dtype = MOE_BF16;
+  up.ab_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
   up.epilogue = MOE_EPI_SILU_GATE;
-  up.c_dtype = MOE_BF16;
+  up.c_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
   up.C = base + L.h;
   up.status = status;
+  if (fp8) {
+    up.A_scales = reinterpret_cast<const float*>(base + L.xps);
+    up.B_scales = W1_scales;
+    up.B_extra_scales = W1s_scales;
+    up.C_scales = reinterpret_cast<float*>(base + L.hs);
+  }
   st = launch_grouped_gemm(up, s);
   if (st != MOE_OK) return st;
 
@@ -352,19 +370,22 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   dn.rows = Rp;
   dn.N = d;
   dn.K = I;
-  dn.ab_dtype = MOE_BF16;
+  dn.ab_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
   dn.epilogue = MOE_EPI_NONE;
   dn.c_dtype = MOE_BF16;
   dn.C = base + L.y;
   dn.status = status;
+  if (fp8) {
+    dn.A_scales = reinterpret_cast<const float*>(base + L.hs);
+    dn.B_scales = W2_scales;
+    dn.B_extra_scales = W2s_scales;
+  }
   st = launch_grouped_gemm(dn, s);
   if (st != MOE_OK) return st;
 
   st = launch_combine(base + L.y, t2r, w, shared ? 1 : 0, T, d, k, out, c.out_dtype, s);
   if (st != MOE_OK) return st;
   if (counts_out) MOE_CUDA_CHECK(cudaMemcpyAsync(counts_out, counts, sizeof(int32_t) * E, cudaMemcpyDeviceToDevice, s));
-  (void)W1s_scales;
-  (void)W2s_scales;
   return MOE_OK;
 }
 

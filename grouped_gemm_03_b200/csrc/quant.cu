@@ -60,7 +60,7 @@ int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, flo
   if (G == 0) return MOE_OK;
   dim3 grid(K / 128, N / 128, G);
   quant_block_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(W), N, K, Wq, scales);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_status(__func__);
 }
 
 }  // namespace moe

@@ -240,7 +240,7 @@ int finish_dispatch(const void* parts, int nsplit, size_t stride, const float* b
   if (v <= VV) {                                                                                             \
     finish_kernel<LT, VV><<<blocks, warps_per_block * 32, 0, s>>>(lp, nsplit, stride, bias, N, E, k, renorm, lo, \
                                                                  idx, w);                                    \
-    return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;                                        \
+    return launch_status(__func__);                                        \
   }
   MOE_FINISH_CASE(1)
   MOE_FINISH_CASE(2)
@@ -257,7 +257,7 @@ int simt_logits(const void* x, const void* Wr, int T, int d, int E, float* logit
   dim3 grid((T + kRTok - 1) / kRTok, (E + kREC - 1) / kREC);
   logits_simt_kernel<XT, WT><<<grid, 256, 0, s>>>(static_cast<const XT*>(x), static_cast<const WT*>(Wr), T, d, E,
                                                   logits);
-  return cudaGetLastError() == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+  return launch_status(__func__);
 }
 
 }  // namespace

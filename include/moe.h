@@ -61,6 +61,7 @@ typedef enum moe_epilogue {
  * MOE_F32 | MOE_BF16 (an fp32 router needs fp32 x).  expert_dtype: MOE_BF16 |
  * MOE_E4M3 (the expert GEMMs run in E4M3 with fp32 scales).  out_dtype:
  * MOE_F32 | MOE_BF16.  shared_inter is 0 (no shared expert) or equal to inter.
+ * d and inter are multiples of 128 (E4M3 experts: d a multiple of 256).
  * renormalize = 0 weights each expert by its softmax value p_i (MegaMoE §2.1);
  * 1 divides by the sum over the selected experts (route_tokens in
  * Dense GEMM -> GroupedGEMM -> TP MoE §4.2). */
@@ -72,6 +73,10 @@ typedef struct moe_config {
 
 /* Human-readable name of a status code (static string). */
 const char* moe_status_string(int status);
+
+/* Description of the last CUDA runtime / driver failure on this host thread
+ * (the call that made an entry point return MOE_ERR_CUDA); static storage. */
+const char* moe_last_error_string(void);
 
 /* Multiprocessor count and compute capability of the current device; returns
  * MOE_ERR_UNSUPPORTED when it is not an sm_100 part. */
@@ -176,8 +181,13 @@ int moe_permute_noalloc(const void* x, int x_dtype, const int32_t* topk_idx, int
  *            MOE_BF16 | MOE_E4M3 (SILU_GATE); rows outside every group untouched
  *   C_scales [N/128][rows] fp32 when c_dtype == MOE_E4M3 (per row per 128 columns)
  *   ws       moe_grouped_gemm_workspace_size() bytes (status word)
- * Supported: K % 64 == 0 (bf16) / K % 128 == 0 (E4M3); N % 128 == 0
- * (SILU_GATE) or N % 64 == 0 (NONE); G <= 1024. */
+ * E4M3 operands: the scales vary along K, so each 128-wide K block's partial
+ * product is scaled by sa[row, kb] * sb[n/128, kb] and accumulated in fp32
+ * ("MegaMoE ..." §5.1); an E4M3 C is quantised per row per 128 columns
+ * (s = amax/448, q = e4m3_rn_satfinite(c/s)) like the permute's activations.
+ * Supported: bf16: K % 64 == 0, N % 128 == 0 (SILU_GATE) or N % 64 == 0
+ * (NONE); E4M3: K % 128 == 0, N % 128 == 0 (SILU_GATE, C bf16 or E4M3) or
+ * N % 256 == 0 (NONE, C bf16); G <= 1024. */
 size_t moe_grouped_gemm_workspace_size(void);
 int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const float* B_scales,
                      const int32_t* offsets, int G, int rows, int N, int K, int ab_dtype, int epilogue,
