@@ -337,7 +337,8 @@ def cpu_baseline(s, inp, budget_s=12.0):
         W1.stage(need)
         W2.stage(need)
         t0 = time.perf_counter()
-        oracle.moe_forward(xs, inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k, renormalize=s.renormalize)
+        fwd = oracle.moe_forward_fp8 if s.fp8 else oracle.moe_forward
+        fwd(xs, inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k, renormalize=s.renormalize)
         spent += time.perf_counter() - t0
         done_tokens += n
         n *= 2
@@ -350,7 +351,7 @@ def cpu_baseline(s, inp, budget_s=12.0):
 
 def run_ours(args, rank, world, dev):
     gg = build_lib()
-    s = shape_of(args.config)
+    s = shape_of(args.config, **args.overrides)
     torch.cuda.set_device(dev)
     stream = torch.cuda.current_stream()
     inp = make_inputs(s, seed=1234 + rank, device=dev)
@@ -434,7 +435,12 @@ def main():
     ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--set", default="", help="shape overrides for profiling runs, e.g. E=32,T=512")
     args = ap.parse_args()
+    args.overrides = {}
+    for kv in filter(None, args.set.split(",")):
+        key, val = kv.split("=")
+        args.overrides[key.strip()] = int(val)
     if args.warmup < 3:
         log("warm-up raised to 3 steps")
         args.warmup = 3
@@ -442,7 +448,7 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    s = shape_of(args.config)
+    s = shape_of(args.config, **args.overrides)
 
     if args.impl == "reference":
         if rank != 0:
@@ -519,8 +525,8 @@ def run_reference(args, s, world):
 
     def step():
         toks = np.sort(rng.choice(s.T, size=per_step, replace=False))
-        oracle.moe_forward(inp["x"][toks], inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k,
-                           renormalize=s.renormalize)
+        fwd = oracle.moe_forward_fp8 if s.fp8 else oracle.moe_forward
+        fwd(inp["x"][toks], inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k, renormalize=s.renormalize)
 
     for _ in range(args.warmup):
         step()

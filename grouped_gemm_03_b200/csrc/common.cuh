@@ -86,6 +86,7 @@ struct GemmArgs {
   int G, has_extra, rows, N, K;
   int ksplit;               // > 1: fp32 partial products of K slices at C + s * rows * N (no epilogue)
   int mma_n;                // 0 = widest tile that divides N; else 64 / 128 / 256 (no-gate GEMMs)
+  int pair_tiles;           // 256-row tiles on CTA pairs: 0 = by average group size, 1 = always, -1 = never
   int ab_dtype, epilogue, c_dtype;
   void* C;
   float* C_scales;

@@ -380,6 +380,285 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ CTA-pair bf16 kernel
+// For large groups (the compute-bound Mixtral-shaped layer) two SMs of a
+// cluster share one 256-row tile: each CTA stages its own 128 rows of A and
+// one half of the 256 B columns (with the SiLU gate: CTA 0 the gate rows, CTA 1
+// the up rows), and the pair's leader issues tcgen05.mma.cta_group::2
+// 256 x 256 x 16, which reads both CTAs' shared memory and accumulates each
+// CTA's 128 rows in its own TMEM.  Per FLOP each SM now moves two thirds of
+// the operand bytes of the single-CTA kernel.  Barriers: both CTAs' TMA loads
+// count their bytes on the leader's full[stage]; the leader's commits arrive
+// on empty[stage] / tfull[acc] in both CTAs; both epilogues release an
+// accumulator on the leader's tempty[acc].
+constexpr int kPairStages = 6;
+constexpr int kPairSmem = 1024 + kPairStages * 32768 + 512 + 2 * (kMaxGroups + 2) * 4;
+
+template <int EPI, int OUT>
+__global__ void __launch_bounds__(kThreads, 1)
+    gg_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                        const __grid_constant__ CUtensorMap tmBx, const Params p) {
+  constexpr int MMA_N = 256;
+  constexpr int BM2 = 256;
+  constexpr int A_BYTES = 128 * 128;
+  constexpr int B_BYTES = 128 * 128;
+  constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  constexpr int STAGES = kPairStages;
+  constexpr int TMEM_COLS = 512;
+  constexpr int OUT_COLS = EPI ? 128 : 256;
+  constexpr uint32_t IDESC = ptx::make_idesc(BM2, MMA_N, 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + STAGES * A_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sB + STAGES * B_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + STAGES * STAGE_BYTES + 512);
+  int* s_tile = s_off + kMaxGroups + 2;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = ptx::cluster_ctarank();
+  const bool leader = rank == 0;
+  const int pair = blockIdx.x >> 1, npairs = gridDim.x >> 1;
+  const int G = p.G_total;
+  const int nt = p.N / OUT_COLS;
+
+  if (warp == 0) {
+    for (int g = lane; g <= G; g += 32) s_off[g] = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
+    __syncwarp();
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int bad = 0, mine = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int m = s_off[g + 1] - s_off[g];
+      if (m < 0) bad = 1;
+      mine += (max(m, 0) + BM2 - 1) / BM2 * nt;
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - mine;
+    for (int g = g0; g < g1; ++g) {
+      s_tile[g] = run;
+      run += (max(s_off[g + 1] - s_off[g], 0) + BM2 - 1) / BM2 * nt;
+    }
+    if (lane == 31) s_tile[G] = incl;
+    if (lane == 0 && (s_off[0] != 0 || s_off[G] > p.rows)) bad = 1;
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      *s_bad = bad;
+      *abort_flag = 0;
+      if (bad && blockIdx.x == 0) set_status(p.status, MOE_ERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  if (*s_bad) return;  // both CTAs of the pair read the same offsets: uniform
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&tfull[a], 1);
+      ptx::mbar_init(&tempty[a], 256);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+    ptx::prefetch_tmap(&tmBx);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc_pair(tmem_slot, TMEM_COLS);
+    ptx::tmem_relinquish_pair();
+  }
+  ptx::tc_fence_before();
+  ptx::cluster_sync();  // barrier inits of both CTAs visible to the pair
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tile[G];
+  const int nk = p.K / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer (both CTAs)
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      for (int tile = pair; tile < total && ok; tile += npairs) {
+        const int g = find_group(s_tile, G, tile);
+        const int m_g = s_off[g + 1] - s_off[g];
+        const int mt = (m_g + BM2 - 1) / BM2;
+        const int tl = tile - s_tile[g];
+        const int nb = tl / mt, mb = tl % mt;
+        const int a_row = s_off[g] + mb * BM2 + static_cast<int>(rank) * 128;
+        const bool extra = g >= p.G_main;
+        const CUtensorMap* mB = extra ? &tmBx : &tmB;
+        const int gb = extra ? 0 : g;
+        const int brow = EPI ? gb * 2 * p.N + static_cast<int>(rank) * p.N + nb * 128
+                             : gb * p.N + nb * 256 + static_cast<int>(rank) * 128;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          const uint32_t fb = ptx::map_to_rank(ptx::smem_u32(&full[stage]), 0);
+          if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
+          ptx::tma_load_2d_pair(sA + stage * A_BYTES, &tmA, fb, kb * 64, a_row);
+          ptx::tma_load_2d_pair(sB + stage * B_BYTES, mB, fb, kb * 64, brow);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        for (int i = 0; i < 20; ++i) __nanosleep(50000);  // let copies in flight land (~1 ms)
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0 && leader) {
+      // ------------------------------------------------------------ MMA issuer (leader CTA)
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = pair; tile < total && ok; tile += npairs, ++it) {
+        const int acc = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (!ptx::mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * MMA_N;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t adesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sA + stage * A_BYTES));
+          const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sB + stage * B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_f16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | kk) != 0);
+          ptx::umma_commit_pair_both(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        ptx::umma_commit_pair_both(&tfull[acc]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+      }
+      ptx::umma_commit_pair_both(drain);
+      ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (both CTAs)
+    const int q = warp & 3;
+    const int row_t = q * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    int it = 0;
+    for (int tile = pair; tile < total; tile += npairs, ++it) {
+      const int acc = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int g = find_group(s_tile, G, tile);
+      const int m_g = s_off[g + 1] - s_off[g];
+      const int mt = (m_g + BM2 - 1) / BM2;
+      const int tl = tile - s_tile[g];
+      const int nb = tl / mt, mb = tl % mt;
+      const int r_in = mb * BM2 + static_cast<int>(rank) * 128 + row_t;
+      const bool valid = r_in < m_g;
+      const size_t grow = static_cast<size_t>(s_off[g] + r_in);
+      if (!ptx::mbar_wait_warp(&tfull[acc], use & 1, abort_flag, kWaitLimitNs)) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        break;
+      }
+      ptx::tc_fence_after();
+      const uint32_t tacc = lane_base + acc * MMA_N;
+      if constexpr (EPI == 1) {
+        __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS;
+#pragma unroll 1
+        for (int c = 0; c < OUT_COLS; c += 32) {
+          uint32_t gv[32], uv[32];
+          ptx::tmem_ld_32x32b_x32(tacc + c, gv);
+          ptx::tmem_ld_32x32b_x32(tacc + OUT_COLS + c, uv);
+          ptx::tmem_ld_wait();
+          if (valid) {
+            uint32_t packed[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
+              const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(uv[2 * i]);
+              const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(uv[2 * i + 1]);
+              const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
+              packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(C + c);
+#pragma unroll
+            for (int v = 0; v < 4; ++v)
+              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < OUT_COLS; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld_32x32b_x32(tacc + c, v);
+          ptx::tmem_ld_wait();
+          if (valid) {
+            if constexpr (OUT == 1) {
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.C) + grow * p.N + nb * OUT_COLS + c);
+#pragma unroll
+              for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            } else {
+              uint32_t packed[16];
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const __nv_bfloat162 hb =
+                    __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
+              }
+              uint4* dst =
+                  reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS + c);
+#pragma unroll
+              for (int i = 0; i < 4; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            }
+          }
+        }
+      }
+      ptx::tc_fence_before();
+      ptx::mbar_arrive_cluster(ptx::map_to_rank(ptx::smem_u32(&tempty[acc]), 0));
+    }
+  }
+
+  ptx::tc_fence_before();
+  ptx::cluster_sync();  // neither CTA leaves while the pair still uses its memory
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc_pair(tmem_base, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ FP8 (E4M3) kernel
 // Same persistent structure; operands are E4M3 with fp32 scales that vary
 // along K ("MegaMoE ..." §2.3 / §5.1: 1x128 per token, 128x128 per weight
@@ -601,12 +880,36 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
       float acc[128];
 #pragma unroll
       for (int i = 0; i < 128; ++i) acc[i] = 0.f;
-      float sa_next = valid ? __ldg(sa_row) : 0.f;
+      // Scales are fetched well ahead of use so that no K block waits on a
+      // global load: this row's sa[kb] runs through a 4-deep register queue;
+      // the tile's weight-block scales sb[kb] are spread over the lanes in
+      // windows of 32 K blocks (lane j holds block w + j) and broadcast with
+      // a shuffle, the next window being loaded halfway through the current.
+      const size_t rstride = static_cast<size_t>(p.rows);
+      float sa0 = (valid && 0 < nbk) ? __ldg(sa_row) : 0.f;
+      float sa1 = (valid && 1 < nbk) ? __ldg(sa_row + rstride) : 0.f;
+      float sa2 = (valid && 2 < nbk) ? __ldg(sa_row + 2 * rstride) : 0.f;
+      float sa3 = (valid && 3 < nbk) ? __ldg(sa_row + 3 * rstride) : 0.f;
+      float wl = lane < nbk ? __ldg(sb_lo + lane) : 0.f;
+      float wh = lane < nbk ? __ldg(sb_hi + lane) : 0.f;
+      float nwl = 0.f, nwh = 0.f;
       for (int kb = 0; kb < nbk; ++kb) {
-        const float sa = sa_next;
-        if (kb + 1 < nbk) sa_next = valid ? __ldg(sa_row + static_cast<size_t>(kb + 1) * p.rows) : 0.f;
-        const float m_lo = sa * __ldg(sb_lo + kb);
-        const float m_hi = sa * __ldg(sb_hi + kb);
+        if ((kb & 31) == 0 && kb > 0) {
+          wl = nwl;
+          wh = nwh;
+        }
+        if ((kb & 31) == 16) {
+          const int kw = (kb & ~31) + 32 + lane;
+          nwl = kw < nbk ? __ldg(sb_lo + kw) : 0.f;
+          nwh = kw < nbk ? __ldg(sb_hi + kw) : 0.f;
+        }
+        const float sa = sa0;
+        sa0 = sa1;
+        sa1 = sa2;
+        sa2 = sa3;
+        sa3 = (valid && kb + 4 < nbk) ? __ldg(sa_row + static_cast<size_t>(kb + 4) * rstride) : 0.f;
+        const float m_lo = sa * __shfl_sync(0xffffffffu, wl, kb & 31);
+        const float m_hi = sa * __shfl_sync(0xffffffffu, wh, kb & 31);
         if (!ptx::mbar_wait_warp(&pfull[pb], puse & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
@@ -614,13 +917,13 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
         ptx::tc_fence_after();
         const uint32_t t0 = lane_base + pb * MMA_N;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          uint32_t v[16];
-          ptx::tmem_ld_32x32b_x16(t0 + (j < 4 ? c_lo : c_hi) + (j & 3) * 16, v);
+        for (int j = 0; j < 16; ++j) {
+          uint32_t v[8];
+          ptx::tmem_ld_32x32b_x8(t0 + (j < 8 ? c_lo : c_hi) + (j & 7) * 8, v);
           ptx::tmem_ld_wait();
-          const float m = j < 4 ? m_lo : m_hi;
+          const float m = j < 8 ? m_lo : m_hi;
 #pragma unroll
-          for (int i = 0; i < 16; ++i) acc[16 * j + i] = fmaf(__uint_as_float(v[i]), m, acc[16 * j + i]);
+          for (int i = 0; i < 8; ++i) acc[8 * j + i] = fmaf(__uint_as_float(v[i]), m, acc[8 * j + i]);
         }
         ptx::tc_fence_before();
         ptx::mbar_arrive(&pempty[pb]);
@@ -778,6 +1081,53 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
 }
 
 template <int EPI, int OUT>
+int run_bf16_pair(const GemmArgs& a, cudaStream_t s) {
+  static_assert(kPairSmem <= 227 * 1024, "shared memory budget");
+  const int nb_rows = EPI ? 2 * a.N : a.N;
+  CUtensorMap mA, mB, mBx;
+  if (!make_map(&mA, a.A, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, 128)) return MOE_ERR_CUDA;
+  if (!make_map(&mB, a.B, 2, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, 128)) return MOE_ERR_CUDA;
+  if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, 128)) return MOE_ERR_CUDA;
+  static int clusters[64] = {};
+  int dev = 0;
+  MOE_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  cudaLaunchConfig_t cfg = {};
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kPairSmem;
+  cfg.stream = s;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (!clusters[dev]) {
+    MOE_CUDA_CHECK(cudaFuncSetAttribute(gg_bf16_pair_kernel<EPI, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        kPairSmem));
+    // persistent grid: as many CTA pairs as can be resident at once
+    cfg.gridDim = dim3(num_sms() & ~1);
+    int n = 0;
+    MOE_CUDA_CHECK(cudaOccupancyMaxActiveClusters(&n, gg_bf16_pair_kernel<EPI, OUT>, &cfg));
+    clusters[dev] = n > 0 ? n : 1;
+  }
+  cfg.gridDim = dim3(2 * clusters[dev]);
+  Params p{};
+  p.offsets = a.offsets;
+  p.G_total = a.G + a.has_extra;
+  p.G_main = a.G;
+  p.N = a.N;
+  p.K = a.K;
+  p.rows = a.rows;
+  p.ksplit = 1;
+  p.C = a.C;
+  p.status = a.status;
+  MOE_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gg_bf16_pair_kernel<EPI, OUT>, mA, mB, mBx, p));
+  return MOE_OK;
+}
+
+template <int EPI, int OUT>
 int run_fp8(const GemmArgs& a, cudaStream_t s) {
   using L = Tile<256>;
   static_assert(L::SMEM <= 227 * 1024, "shared memory budget");
@@ -818,10 +1168,14 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
 int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.G + a.has_extra == 0 || a.rows == 0) return MOE_OK;
   if (a.ab_dtype == MOE_BF16) {
+    // CTA pairs pay off when tiles of 256 rows are mostly full: large groups on average
+    const bool pairs = a.pair_tiles > 0 || (a.pair_tiles == 0 && a.rows >= 512 * (a.G + a.has_extra));
     if (a.epilogue == MOE_EPI_SILU_GATE) {
-      if (a.c_dtype == MOE_BF16 && a.N % 128 == 0 && a.ksplit <= 1) return run_bf16<256, 1, 0>(a, s);
-      return MOE_ERR_UNSUPPORTED;
+      if (a.c_dtype != MOE_BF16 || a.N % 128 != 0 || a.ksplit > 1) return MOE_ERR_UNSUPPORTED;
+      return pairs ? run_bf16_pair<1, 0>(a, s) : run_bf16<256, 1, 0>(a, s);
     }
+    if (pairs && a.ksplit <= 1 && a.N % 256 == 0 && (a.mma_n == 0 || a.mma_n == 256))
+      return a.c_dtype == MOE_F32 ? run_bf16_pair<0, 1>(a, s) : run_bf16_pair<0, 0>(a, s);
     const int out = a.c_dtype == MOE_F32 ? 1 : 0;
     if (a.c_dtype != MOE_F32 && a.c_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
     if (a.ksplit > 1 && (!out || a.ksplit > a.K / 64)) return MOE_ERR_UNSUPPORTED;

@@ -177,6 +177,11 @@ GEMM_CASES = [
     ([128], 128, 64, gg.EPI_SILU_GATE, torch.bfloat16),
     ([0, 250, 1, 128, 513], 256, 384, gg.EPI_SILU_GATE, torch.bfloat16),
     ([1000, 24, 0, 0, 333], 512, 1024, gg.EPI_NONE, torch.bfloat16),
+    # groups of >= 512 rows on average run on CTA pairs (256-row tiles split over two SMs)
+    ([1024, 700, 513], 256, 256, gg.EPI_NONE, torch.bfloat16),
+    ([2000, 0, 129], 512, 128, gg.EPI_NONE, torch.float32),
+    ([257, 1600, 0, 255], 128, 320, gg.EPI_SILU_GATE, torch.bfloat16),
+    ([1536, 1], 256, 512, gg.EPI_SILU_GATE, torch.bfloat16),
 ]
 
 
