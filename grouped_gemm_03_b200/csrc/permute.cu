@@ -129,8 +129,12 @@ __device__ __forceinline__ void load_row8(const float* p, float (&f)[8]) {
   f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
 }
 
+// Columns of x one scatter block copies: the grid is (token blocks) x (d /
+// kScatterCols) so that even a few hundred tokens keep every SM busy.
+constexpr int kScatterCols = 512;
+
 template <typename XT, bool kFp8>
-__global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a, int nblk) {
+__global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   __shared__ int s_idx[kTokPerBlock * kMaxTopK];
   __shared__ int s_row[kTokPerBlock * (kMaxTopK + 1)];
   const int b = blockIdx.x;
@@ -140,6 +144,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a, in
   const int R = a.T * k;
   const int rows_total = R + (a.shared ? a.T : 0);
   const int nd = k + (a.shared ? 1 : 0);  // destinations per token
+  const bool writer = blockIdx.y == 0;   // one column block writes the index maps
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) s_idx[p] = a.idx[static_cast<size_t>(t0) * k + p];
   __syncthreads();
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
@@ -153,43 +158,59 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a, in
       if (row < 0 || row >= R) row = 0;  // only reachable with invalid ids (status already set)
     }
     s_row[tl * nd + j] = row;
-    a.token_to_row[static_cast<size_t>(t0 + tl) * k + j] = row;
-    a.row_to_token[row] = t0 + tl;
+    if (writer) {
+      a.token_to_row[static_cast<size_t>(t0 + tl) * k + j] = row;
+      a.row_to_token[row] = t0 + tl;
+    }
   }
   if (a.shared)
     for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) {
       s_row[tl * nd + k] = R + t0 + tl;
-      a.row_to_token[R + t0 + tl] = t0 + tl;
+      if (writer) a.row_to_token[R + t0 + tl] = t0 + tl;
     }
   __syncthreads();
 
   const int d = a.d;
+  const int cbeg = blockIdx.y * kScatterCols;
+  const int cw = min(kScatterCols, d - cbeg);
   const XT* x = static_cast<const XT*>(a.x);
   if constexpr (!kFp8) {
-    // bf16 destination: 8 elements (16 bytes) per thread per step
+    // bf16 destination: 8 elements (16 bytes) per thread per item, 4 items in flight
     __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(a.xp);
-    const int nvec = d / 8;
-    for (int it = threadIdx.x; it < nt * nvec; it += blockDim.x) {
-      const int tl = it / nvec, c = (it % nvec) * 8;
-      const XT* src = x + static_cast<size_t>(t0 + tl) * d + c;
-      uint4 out;
-      if constexpr (sizeof(XT) == 2) {
-        out = *reinterpret_cast<const uint4*>(src);
-      } else {
-        float f[8];
-        load_row8(reinterpret_cast<const float*>(src), f);
-        __nv_bfloat162 h[4];
+    const int nvec = cw / 8;
+    const int items = nt * nvec;
+    for (int base = threadIdx.x; base < items; base += 4 * blockDim.x) {
+      uint4 v[4];
+      int tl[4], c[4];
 #pragma unroll
-        for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
-        out = *reinterpret_cast<uint4*>(h);
+      for (int u = 0; u < 4; ++u) {
+        const int it = base + u * blockDim.x;
+        tl[u] = it < items ? it / nvec : -1;
+        c[u] = it < items ? cbeg + (it % nvec) * 8 : 0;
+        if (tl[u] < 0) continue;
+        const XT* src = x + static_cast<size_t>(t0 + tl[u]) * d + c[u];
+        if constexpr (sizeof(XT) == 2) {
+          v[u] = *reinterpret_cast<const uint4*>(src);
+        } else {
+          float f[8];
+          load_row8(reinterpret_cast<const float*>(src), f);
+          __nv_bfloat162 h[4];
+#pragma unroll
+          for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+          v[u] = *reinterpret_cast<uint4*>(h);
+        }
       }
-      for (int j = 0; j < nd; ++j)
-        *reinterpret_cast<uint4*>(xp + static_cast<size_t>(s_row[tl * nd + j]) * d + c) = out;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        if (tl[u] < 0) continue;
+        for (int j = 0; j < nd; ++j)
+          *reinterpret_cast<uint4*>(xp + static_cast<size_t>(s_row[tl[u] * nd + j]) * d + c[u]) = v[u];
+      }
     }
   } else {
     // E4M3 destination: 16 threads quantise one 128-column group of one token
     uint8_t* xp = static_cast<uint8_t*>(a.xp);
-    const int ngrp = d / 128;
+    const int ngrp = cw / 128;
     const int sub = threadIdx.x & 15;
     const int half = (threadIdx.x >> 4) & 1;
     const int total = nt * ngrp;
@@ -198,7 +219,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a, in
     for (int base = (threadIdx.x >> 5) * 2; base < total; base += (blockDim.x >> 5) * 2) {
       const int it = base + half;
       const bool act = it < total;
-      const int tl = act ? it / ngrp : 0, gi = act ? it % ngrp : 0;
+      const int tl = act ? it / ngrp : 0, gi = act ? cbeg / 128 + it % ngrp : 0;
       const int c = gi * 128 + sub * 8;
       float f[8];
       const XT* src = x + static_cast<size_t>(t0 + tl) * d + c;
@@ -241,7 +262,6 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a, in
       }
     }
   }
-  (void)nblk;
 }
 
 }  // namespace
@@ -261,16 +281,17 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
   scan_kernel<<<1, 1024, 0, s>>>(a.block_base, nblk, a.E, a.T * a.k, a.T, a.shared, a.counts, a.offsets);
   MOE_CUDA_CHECK(cudaGetLastError());
   const bool fp8 = a.xp_dtype == MOE_E4M3;
+  const dim3 grid(nblk, (a.d + kScatterCols - 1) / kScatterCols);
   if (a.x_dtype == MOE_BF16) {
     if (fp8)
-      scatter_kernel<__nv_bfloat16, true><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+      scatter_kernel<__nv_bfloat16, true><<<grid, kPermThreads, 0, s>>>(a);
     else
-      scatter_kernel<__nv_bfloat16, false><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+      scatter_kernel<__nv_bfloat16, false><<<grid, kPermThreads, 0, s>>>(a);
   } else {
     if (fp8)
-      scatter_kernel<float, true><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+      scatter_kernel<float, true><<<grid, kPermThreads, 0, s>>>(a);
     else
-      scatter_kernel<float, false><<<nblk, kPermThreads, 0, s>>>(a, nblk);
+      scatter_kernel<float, false><<<grid, kPermThreads, 0, s>>>(a);
   }
   MOE_CUDA_CHECK(cudaGetLastError());
   return MOE_OK;

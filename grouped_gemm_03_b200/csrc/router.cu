@@ -105,78 +105,111 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
 }
 
 // ------------------------------------------------------------------ SIMT logits
-// Block = 32 tokens x 8 experts; each warp owns 4 tokens.  W_r rows of the
-// block's experts are staged (as fp32) in shared memory 512 columns at a time,
-// so every block reads them once from L2 while x streams from HBM once per
-// expert block.  Used when E or d is small (the logits are then bound by
-// reading x) and for fp32 operands.
-constexpr int kRTok = 32;
+// Block = 16 tokens x 8 experts; each warp owns 2 tokens.  The block's W_r
+// rows are staged in shared memory 32 KB at a time (2048 bf16 / 1024 fp32
+// columns), so each block reads them once from L2 while x streams from HBM
+// once per expert block; every lane keeps the next 8 columns of its tokens
+// in flight while it multiplies the current ones.  Used when E or d is small
+// (the logits are then bound by reading x) and for fp32 operands.
 constexpr int kREC = 8;
-constexpr int kRDC = 512;
+constexpr int kTPW = 2;
+constexpr int kRTok = 8 * kTPW;
+
+template <typename T>
+__device__ __forceinline__ void load8_any(const T* p, float (&f)[8]) {
+  load8(p, f);
+}
+
+// 8 consecutive shared-memory elements as fp32.
+__device__ __forceinline__ void smem8(const float* p, float (&f)[8]) {
+  const float4 a = *reinterpret_cast<const float4*>(p);
+  const float4 b = *(reinterpret_cast<const float4*>(p) + 1);
+  f[0] = a.x; f[1] = a.y; f[2] = a.z; f[3] = a.w;
+  f[4] = b.x; f[5] = b.y; f[6] = b.z; f[7] = b.w;
+}
+__device__ __forceinline__ void smem8(const __nv_bfloat16* p, float (&f)[8]) {
+  const uint4 a = *reinterpret_cast<const uint4*>(p);
+  const uint32_t w[4] = {a.x, a.y, a.z, a.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = __uint_as_float(w[i] << 16);
+    f[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u);
+  }
+}
 
 template <typename XT, typename WT>
 __global__ void __launch_bounds__(256) logits_simt_kernel(const XT* __restrict__ x, const WT* __restrict__ Wr,
                                                           int T, int d, int E, float* __restrict__ logits) {
-  __shared__ __align__(16) float s_w[kREC][kRDC];
+  constexpr int DC = 32768 / (kREC * static_cast<int>(sizeof(WT)));  // columns per staged chunk
+  constexpr int VPE = 16 / static_cast<int>(sizeof(WT));            // elements per 16-byte copy
+  __shared__ __align__(16) WT s_w[kREC][DC];
   const int t0 = blockIdx.x * kRTok, e0 = blockIdx.y * kREC;
   const int ne = min(kREC, E - e0);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tw = t0 + warp * 4;
-  float acc[4][kREC];
+  const int tw = t0 + warp * kTPW;
+  float acc[kTPW][kREC];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < kTPW; ++i)
 #pragma unroll
     for (int e = 0; e < kREC; ++e) acc[i][e] = 0.f;
-  for (int c0 = 0; c0 < d; c0 += kRDC) {
-    const int dc = min(kRDC, d - c0);
+  for (int c0 = 0; c0 < d; c0 += DC) {
+    const int dc = min(DC, d - c0);
     __syncthreads();
-    for (int i = threadIdx.x; i < kREC * (kRDC / 8); i += blockDim.x) {
-      const int e = i / (kRDC / 8), c = (i % (kRDC / 8)) * 8;
-      float f[8];
-      if (e < ne && c < dc) {
-        load8(Wr + static_cast<size_t>(e0 + e) * d + c0 + c, f);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) f[q] = 0.f;
-      }
-      float4* dst = reinterpret_cast<float4*>(&s_w[e][c]);
-      dst[0] = make_float4(f[0], f[1], f[2], f[3]);
-      dst[1] = make_float4(f[4], f[5], f[6], f[7]);
+    for (int i = threadIdx.x; i < kREC * (DC / VPE); i += blockDim.x) {
+      const int e = i / (DC / VPE), c = (i % (DC / VPE)) * VPE;
+      uint4 v = make_uint4(0, 0, 0, 0);
+      if (e < ne && c < dc) v = __ldg(reinterpret_cast<const uint4*>(Wr + static_cast<size_t>(e0 + e) * d + c0 + c));
+      *reinterpret_cast<uint4*>(&s_w[e][c]) = v;
     }
     __syncthreads();
-    for (int c = lane * 8; c < dc; c += 256) {
-      float xv[4][8];
+    float xv[kTPW][8];
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (tw + i < T) {
-          load8(x + static_cast<size_t>(tw + i) * d + c0 + c, xv[i]);
+    for (int i = 0; i < kTPW; ++i) {
+      const int c = lane * 8;
+      if (tw + i < T && c < dc) {
+        load8_any(x + static_cast<size_t>(tw + i) * d + c0 + c, xv[i]);
+      } else {
+#pragma unroll
+        for (int q = 0; q < 8; ++q) xv[i][q] = 0.f;
+      }
+    }
+    for (int c = lane * 8; c < dc; c += 256) {
+      float xn[kTPW][8];
+      const int cn = c + 256;
+#pragma unroll
+      for (int i = 0; i < kTPW; ++i) {
+        if (tw + i < T && cn < dc) {
+          load8_any(x + static_cast<size_t>(tw + i) * d + c0 + cn, xn[i]);
         } else {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) xv[i][q] = 0.f;
+          for (int q = 0; q < 8; ++q) xn[i][q] = 0.f;
         }
       }
 #pragma unroll
       for (int e = 0; e < kREC; ++e) {
-        const float4 wa = *reinterpret_cast<const float4*>(&s_w[e][c]);
-        const float4 wb = *reinterpret_cast<const float4*>(&s_w[e][c + 4]);
-        const float wv[8] = {wa.x, wa.y, wa.z, wa.w, wb.x, wb.y, wb.z, wb.w};
+        float wv[8];
+        smem8(&s_w[e][c], wv);
 #pragma unroll
-        for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < kTPW; ++i)
 #pragma unroll
           for (int q = 0; q < 8; ++q) acc[i][e] = fmaf(xv[i][q], wv[q], acc[i][e]);
       }
+#pragma unroll
+      for (int i = 0; i < kTPW; ++i)
+#pragma unroll
+        for (int q = 0; q < 8; ++q) xv[i][q] = xn[i][q];
     }
   }
   float mine = 0.f;
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < kTPW; ++i)
 #pragma unroll
     for (int e = 0; e < kREC; ++e) {
       const float v = warp_sum(acc[i][e]);
       if (lane == i * kREC + e) mine = v;
     }
   const int t = tw + lane / kREC, e = lane % kREC;
-  if (t < T && e < ne) logits[static_cast<size_t>(t) * E + e0 + e] = mine;
+  if (lane < kTPW * kREC && t < T && e < ne) logits[static_cast<size_t>(t) * E + e0 + e] = mine;
 }
 
 // ------------------------------------------------------------------ finish
