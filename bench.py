@@ -41,7 +41,8 @@ import torch
 ROOT = os.path.dirname(os.path.abspath(__file__))
 sys.path.insert(0, ROOT)
 
-from workload import CONFIGS, make_inputs, shape_of  # noqa: E402
+from workload import CONFIGS, make_inputs, make_router_logits, shape_of  # noqa: E402
+from workload.gen import ROUTER_MICRO  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200; grouped-GEMM TFLOP/s as % of dense tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
@@ -432,7 +433,7 @@ def main():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=3)
-    ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS))
+    ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS) + ["router_micro"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--set", default="", help="shape overrides for profiling runs, e.g. E=32,T=512")
@@ -448,6 +449,8 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.config == "router_micro":
+        return run_router_micro(args, rank, world, local)
     s = shape_of(args.config, **args.overrides)
 
     if args.impl == "reference":
@@ -506,6 +509,91 @@ def main():
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(result), flush=True)
+    return 0
+
+
+def run_router_micro(args, rank, world, local):
+    """Router-only microbenchmark: softmax + top-k of N fp16 logits rows (moe_topk_logits)."""
+    N, E, k = (args.overrides.get(key, ROUTER_MICRO[key]) for key in ("N", "E", "k"))
+    desc = {"workload": f"router_micro: N={N} tokens, E={E} experts, top-{k}, fp16 logits ~ N(0,1)",
+            "tokens_per_step": N, "seed": 1234,
+            "l2": "flushed between timed steps (2x L2 buffer rewrite, outside the events)"}
+    bytes_per_step = N * E * 2 + N * k * 8
+    if args.impl == "reference":
+        if rank != 0:
+            return 0
+        import oracle
+        from threadpoolctl import threadpool_info
+        logits = make_router_logits(N, E, seed=1234, device="cpu")
+        lf = oracle.as_f64(logits)
+        per_step = min(N, 4096)
+        rng = np.random.default_rng(3)
+
+        def step():
+            rows = rng.choice(N, size=per_step, replace=False)
+            oracle.gate_weights(oracle.softmax(lf[rows]), oracle.topk_select(lf[rows], k))
+
+        for _ in range(args.warmup):
+            step()
+        t0 = time.perf_counter()
+        for _ in range(args.steps):
+            step()
+        dt = time.perf_counter() - t0
+        value = args.steps * per_step / dt
+        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        print(json.dumps({"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                          "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                          "config": desc,
+                          "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": threads,
+                                           "kind": "oracle", "sample": f"{per_step} random rows of {N} per step"},
+                          "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                                  "d2h_bytes_per_step": 0}}), flush=True)
+        return 0
+    gg = build_lib()
+    dev = local
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream()
+    logits = make_router_logits(N, E, seed=1234 + rank, device=dev)
+    idx = torch.empty((N, k), dtype=torch.int32, device=dev)
+    w = torch.empty((N, k), dtype=torch.float32, device=dev)
+    scrub = torch.empty(max(2 * torch.cuda.get_device_properties(dev).L2_cache_size, 256 << 20), dtype=torch.uint8,
+                        device=dev)
+
+    def step():
+        gg.topk_logits(logits, k, out_idx=idx, out_w=w)
+
+    with ClockSampler(dev) as clk:
+        times = time_steps(step, args.steps, args.warmup, lambda: scrub.fill_(1), stream)
+    ms = float(np.mean(times))
+    lh = logits.cpu().pin_memory()
+    ih = torch.empty((N, k), dtype=torch.int32).pin_memory()
+    wh = torch.empty((N, k), dtype=torch.float32).pin_memory()
+
+    def step_host():
+        logits.copy_(lh, non_blocking=True)
+        gg.topk_logits(logits, k, out_idx=idx, out_w=w)
+        ih.copy_(idx, non_blocking=True)
+        wh.copy_(w, non_blocking=True)
+
+    e2e_ms = float(np.mean(time_steps(step_host, max(3, args.steps // 2), 2, lambda: scrub.fill_(1), stream,
+                                      hold=False)))
+    peaks, kind = load_peaks()
+    achieved = bytes_per_step / (ms * 1e-3) / 1e9
+    result = {"metric": METRIC, "value": round(world * N / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
+              "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
+              "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": desc,
+              "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": float(peaks["hbm_gbs"]),
+                           "unit": "GB/s", "frac": round(achieved / float(peaks["hbm_gbs"]), 4), "traffic": None,
+                           "kernel": "finish_kernel (softmax + top-k of stored logits)",
+                           "peak_kind": f"{kind} HBM copy bandwidth"},
+              "kernel_us": round(ms * 1e3, 2),
+              "e2e": {"value": round(world * N / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+                      "h2d_bytes_per_step": N * E * 2, "d2h_bytes_per_step": N * k * 8},
+              "gpu_launches": args.steps, "clocks": clk.summary()}
     if rank == 0:
         print(json.dumps(result), flush=True)
     return 0
