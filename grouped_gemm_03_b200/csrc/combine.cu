@@ -19,55 +19,13 @@ __device__ __forceinline__ void unpack8(const uint4& r, float (&f)[8]) {
   }
 }
 
-// Grid = tokens x (d / 1024): each thread owns 8 columns of one token and
-// issues the k + 1 row loads for them at once.
-constexpr int kCombCols = kCombThreads * 8;
+// Grid = tokens x (d / 2048): each thread owns 16 columns (two 16-byte
+// pieces) of one token and issues the loads of all k + 1 rows for them before
+// it accumulates.
+constexpr int kCombCols = kCombThreads * 16;
 
 template <typename OT>
-__global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat16* __restrict__ Y,
-                                                              const int32_t* __restrict__ t2r,
-                                                              const float* __restrict__ w, int has_shared,
-                                                              int T, int d, int k, OT* __restrict__ out) {
-  __shared__ int s_row[kMaxTopK];
-  __shared__ float s_w[kMaxTopK];
-  const int t = blockIdx.x;
-  if (threadIdx.x < k) {
-    s_row[threadIdx.x] = t2r[static_cast<size_t>(t) * k + threadIdx.x];
-    s_w[threadIdx.x] = w[static_cast<size_t>(t) * k + threadIdx.x];
-  }
-  __syncthreads();
-  const int c = blockIdx.y * kCombCols + threadIdx.x * 8;
-  if (c >= d) return;
-  const size_t R = static_cast<size_t>(T) * k;
-  float acc[8];
-  if (has_shared) {
-    unpack8(__ldg(reinterpret_cast<const uint4*>(Y + (R + t) * d + c)), acc);
-  } else {
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  }
-  int j = 0;
-  for (; j + 4 <= k; j += 4) {  // four rows in flight
-    uint4 r[4];
-#pragma unroll
-    for (int u = 0; u < 4; ++u) r[u] = __ldg(reinterpret_cast<const uint4*>(Y + static_cast<size_t>(s_row[j + u]) * d + c));
-#pragma unroll
-    for (int u = 0; u < 4; ++u) {
-      float f[8];
-      unpack8(r[u], f);
-      const float wj = s_w[j + u];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
-    }
-  }
-  for (; j < k; ++j) {
-    float f[8];
-    unpack8(__ldg(reinterpret_cast<const uint4*>(Y + static_cast<size_t>(s_row[j]) * d + c)), f);
-    const float wj = s_w[j];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = fmaf(wj, f[i], acc[i]);
-  }
-  OT* o = out + static_cast<size_t>(t) * d + c;
+__device__ __forceinline__ void store8(OT* o, const float (&acc)[8]) {
   if constexpr (sizeof(OT) == 4) {
     reinterpret_cast<float4*>(o)[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
     reinterpret_cast<float4*>(o)[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
@@ -77,6 +35,70 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat
     for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
     *reinterpret_cast<uint4*>(o) = *reinterpret_cast<uint4*>(h);
   }
+}
+
+template <typename OT>
+__global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat16* __restrict__ Y,
+                                                              const int32_t* __restrict__ t2r,
+                                                              const float* __restrict__ w, int has_shared,
+                                                              int T, int d, int k, OT* __restrict__ out) {
+  const int t = blockIdx.x;
+  const int c0 = blockIdx.y * kCombCols + threadIdx.x * 8;               // first piece
+  const int c1 = c0 + kCombThreads * 8;                                   // second piece
+  const bool p0 = c0 < d, p1 = c1 < d;
+  if (!p0) return;
+  const size_t R = static_cast<size_t>(T) * k;
+  float a0[8], a1[8];
+  if (has_shared) {
+    const __nv_bfloat16* ys = Y + (R + t) * d;
+    unpack8(__ldg(reinterpret_cast<const uint4*>(ys + c0)), a0);
+    if (p1) unpack8(__ldg(reinterpret_cast<const uint4*>(ys + c1)), a1);
+  } else {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a0[i] = a1[i] = 0.f;
+  }
+  const int32_t* rows = t2r + static_cast<size_t>(t) * k;
+  const float* ws = w + static_cast<size_t>(t) * k;
+  int j = 0;
+  for (; j + 4 <= k; j += 4) {  // four rows x two pieces in flight
+    uint4 r0[4], r1[4];
+    float wj[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const __nv_bfloat16* yr = Y + static_cast<size_t>(__ldg(rows + j + u)) * d;
+      wj[u] = __ldg(ws + j + u);
+      r0[u] = __ldg(reinterpret_cast<const uint4*>(yr + c0));
+      if (p1) r1[u] = __ldg(reinterpret_cast<const uint4*>(yr + c1));
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      float f[8];
+      unpack8(r0[u], f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a0[i] = fmaf(wj[u], f[i], a0[i]);
+      if (p1) {
+        unpack8(r1[u], f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) a1[i] = fmaf(wj[u], f[i], a1[i]);
+      }
+    }
+  }
+  for (; j < k; ++j) {
+    const __nv_bfloat16* yr = Y + static_cast<size_t>(__ldg(rows + j)) * d;
+    const float wj = __ldg(ws + j);
+    float f[8];
+    unpack8(__ldg(reinterpret_cast<const uint4*>(yr + c0)), f);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) a0[i] = fmaf(wj, f[i], a0[i]);
+    if (p1) {
+      unpack8(__ldg(reinterpret_cast<const uint4*>(yr + c1)), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) a1[i] = fmaf(wj, f[i], a1[i]);
+    }
+  }
+  OT* o = out + static_cast<size_t>(t) * d;
+  store8(o + c0, a0);
+  if (p1) store8(o + c1, a1);
 }
 
 }  // namespace

@@ -50,11 +50,12 @@ inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 // Each returns a moe_status; they assume arguments were validated.
 
 constexpr int kRouterMaxSplit = 8;  // K slices of the tensor-core router
-// parts: scratch of kRouterMaxSplit * T * E fp32 (partial logits)
+// parts: scratch of kRouterMaxSplit * T * router_padded_experts(E) fp32 (partial logits)
 int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d, int E,
                   int k, int renorm, float* logits_out, int32_t* idx, float* w, float* parts, int* status,
                   cudaStream_t s);
 bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E);
+int router_padded_experts(int E);  // logits columns the tensor-core router computes
 int launch_topk_logits(const void* logits, int dtype, int N, int E, int k, int renorm, int32_t* idx,
                        float* w, cudaStream_t s);
 
@@ -84,6 +85,7 @@ struct GemmArgs {
   const float* B_extra_scales;
   const int32_t* offsets;   // [G + has_extra + 1]
   int G, has_extra, rows, N, K;
+  int B_rows;               // > 0: rows of B actually present (G == 1); rows past it read as zero
   int ksplit;               // > 1: fp32 partial products of K slices at C + s * rows * N (no epilogue)
   int mma_n;                // 0 = widest tile that divides N; else 64 / 128 / 256 (no-gate GEMMs)
   int pair_tiles;           // 256-row tiles on CTA pairs: 0 = by average group size, 1 = always, -1 = never

@@ -1054,7 +1054,9 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   const uint32_t box_b = EPI ? MMA_N / 2 : MMA_N;
   CUtensorMap mA, mB, mBx;
   if (!make_map(&mA, a.A, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
-  if (!make_map(&mB, a.B, 2, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  const uint64_t b_rows = a.B_rows > 0 ? static_cast<uint64_t>(a.B_rows)
+                                       : static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows;
+  if (!make_map(&mB, a.B, 2, b_rows, a.K, box_b)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   static bool attr_set[64] = {};
   int dev = 0;

@@ -64,7 +64,7 @@ FwdLayout fwd_layout(const moe_config& c) {
   L.status = take(256);
   L.idx = take(T * k * 4);
   L.w = take(T * k * 4);
-  L.logits = take(kRouterMaxSplit * T * E * 4);
+  L.logits = take(kRouterMaxSplit * T * static_cast<size_t>(router_padded_experts(c.E)) * 4);
   L.base = take(static_cast<size_t>(permute_blocks(c.T)) * E * 4);
   L.counts = take(E * 4);
   L.offsets = take((E + 2) * 4);
@@ -140,7 +140,9 @@ int moe_read_device_status(const void* ws, void* stream, int* status) {
 
 // ------------------------------------------------------------------ router
 size_t moe_router_workspace_size(int T, int E) {
-  return 256 + align_up(static_cast<size_t>(kRouterMaxSplit) * (T > 0 ? T : 0) * (E > 0 ? E : 0) * 4, 256);
+  return 256 + align_up(static_cast<size_t>(kRouterMaxSplit) * (T > 0 ? T : 0) *
+                            static_cast<size_t>(E > 0 ? router_padded_experts(E) : 0) * 4,
+                        256);
 }
 
 int moe_router_topk(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d,

@@ -175,15 +175,16 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   const int cw = min(kScatterCols, d - cbeg);
   const XT* x = static_cast<const XT*>(a.x);
   if constexpr (!kFp8) {
-    // bf16 destination: 8 elements (16 bytes) per thread per item, 4 items in flight
+    // bf16 destination: 8 elements (16 bytes) per item, 4 items in flight per thread
+    constexpr int U = 4;
     __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(a.xp);
     const int nvec = cw / 8;
     const int items = nt * nvec;
-    for (int base = threadIdx.x; base < items; base += 4 * blockDim.x) {
-      uint4 v[4];
-      int tl[4], c[4];
+    for (int base = threadIdx.x; base < items; base += U * blockDim.x) {
+      uint4 v[U];
+      int tl[U], c[U];
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         const int it = base + u * blockDim.x;
         tl[u] = it < items ? it / nvec : -1;
         c[u] = it < items ? cbeg + (it % nvec) * 8 : 0;
@@ -201,7 +202,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
         }
       }
 #pragma unroll
-      for (int u = 0; u < 4; ++u) {
+      for (int u = 0; u < U; ++u) {
         if (tl[u] < 0) continue;
         for (int j = 0; j < nd; ++j)
           *reinterpret_cast<uint4*>(xp + static_cast<size_t>(s_row[tl[u] * nd + j]) * d + c[u]) = v[u];

@@ -33,60 +33,6 @@ __device__ __forceinline__ float warp_sum(float v) {
   return v;
 }
 
-// Softmax + top-k over the values a warp holds in registers: lane `lane`
-// holds v[i] for expert ix[i] (ix = INT_MAX marks padding, v = -inf).
-template <int V>
-__device__ __forceinline__ void warp_select(float (&v)[V], const int (&ix)[V], int k, int renorm, int lane,
-                                            int32_t* idx_out, float* w_out) {
-  float m = -FLT_MAX;
-#pragma unroll
-  for (int i = 0; i < V; ++i) m = fmaxf(m, v[i]);
-  m = warp_max(m);
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < V; ++i)
-    if (ix[i] != INT_MAX) s += expf(v[i] - m);
-  s = warp_sum(s);
-
-  float my_p = 0.f;
-  int my_i = 0;
-  for (int j = 0; j < k; ++j) {
-    float bv = -INFINITY;
-    int bi = INT_MAX;
-#pragma unroll
-    for (int i = 0; i < V; ++i)
-      if (v[i] > bv || (v[i] == bv && ix[i] < bi)) {
-        bv = v[i];
-        bi = ix[i];
-      }
-#pragma unroll
-    for (int o = 16; o; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xffffffffu, bv, o);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, o);
-      if (ov > bv || (ov == bv && oi < bi)) {
-        bv = ov;
-        bi = oi;
-      }
-    }
-    if (lane == j) {
-      my_i = bi;
-      my_p = expf(bv - m) / s;
-    }
-#pragma unroll
-    for (int i = 0; i < V; ++i)
-      if (ix[i] == bi) v[i] = -INFINITY;
-  }
-  if (renorm) {
-    const float ps = warp_sum(lane < k ? my_p : 0.f);
-    my_p = my_p / ps;
-  }
-  if (lane < k) {
-    idx_out[lane] = my_i;
-    w_out[lane] = my_p;
-  }
-}
-
-
 // 8 consecutive elements as fp32.
 __device__ __forceinline__ void load8(const float* p, float (&f)[8]) {
   const float4 a = __ldg(reinterpret_cast<const float4*>(p));
@@ -105,15 +51,16 @@ __device__ __forceinline__ void load8(const __nv_bfloat16* p, float (&f)[8]) {
 }
 
 // ------------------------------------------------------------------ SIMT logits
-// Block = 16 tokens x 8 experts; each warp owns 2 tokens.  The block's W_r
-// rows are staged in shared memory 32 KB at a time (2048 bf16 / 1024 fp32
+// Block = 8 tokens x 8 experts (4 warps of 2 tokens).  The block's W_r rows
+// are staged in shared memory 32 KB at a time (2048 bf16 / 1024 fp32
 // columns), so each block reads them once from L2 while x streams from HBM
-// once per expert block; every lane keeps the next 8 columns of its tokens
-// in flight while it multiplies the current ones.  Used when E or d is small
+// once per expert block; every lane keeps the next two steps of its tokens'
+// columns in flight while it multiplies the current ones.  Used when E or d is small
 // (the logits are then bound by reading x) and for fp32 operands.
 constexpr int kREC = 8;
 constexpr int kTPW = 2;
-constexpr int kRTok = 8 * kTPW;
+constexpr int kRWarps = 4;
+constexpr int kRTok = kRWarps * kTPW;
 
 template <typename T>
 __device__ __forceinline__ void load8_any(const T* p, float (&f)[8]) {
@@ -138,7 +85,7 @@ __device__ __forceinline__ void smem8(const __nv_bfloat16* p, float (&f)[8]) {
 }
 
 template <typename XT, typename WT>
-__global__ void __launch_bounds__(256) logits_simt_kernel(const XT* __restrict__ x, const WT* __restrict__ Wr,
+__global__ void __launch_bounds__(kRWarps * 32) logits_simt_kernel(const XT* __restrict__ x, const WT* __restrict__ Wr,
                                                           int T, int d, int E, float* __restrict__ logits) {
   constexpr int DC = 32768 / (kREC * static_cast<int>(sizeof(WT)));  // columns per staged chunk
   constexpr int VPE = 16 / static_cast<int>(sizeof(WT));            // elements per 16-byte copy
@@ -162,29 +109,24 @@ __global__ void __launch_bounds__(256) logits_simt_kernel(const XT* __restrict__
       *reinterpret_cast<uint4*>(&s_w[e][c]) = v;
     }
     __syncthreads();
-    float xv[kTPW][8];
-#pragma unroll
-    for (int i = 0; i < kTPW; ++i) {
-      const int c = lane * 8;
-      if (tw + i < T && c < dc) {
-        load8_any(x + static_cast<size_t>(tw + i) * d + c0 + c, xv[i]);
-      } else {
-#pragma unroll
-        for (int q = 0; q < 8; ++q) xv[i][q] = 0.f;
-      }
-    }
-    for (int c = lane * 8; c < dc; c += 256) {
-      float xn[kTPW][8];
-      const int cn = c + 256;
+    // three steps of 8 columns in flight per lane: current (xa), next (xb), after next (xc)
+    auto fetch = [&](float (&dst)[kTPW][8], int c) {
 #pragma unroll
       for (int i = 0; i < kTPW; ++i) {
-        if (tw + i < T && cn < dc) {
-          load8_any(x + static_cast<size_t>(tw + i) * d + c0 + cn, xn[i]);
+        if (tw + i < T && c < dc) {
+          load8_any(x + static_cast<size_t>(tw + i) * d + c0 + c, dst[i]);
         } else {
 #pragma unroll
-          for (int q = 0; q < 8; ++q) xn[i][q] = 0.f;
+          for (int q = 0; q < 8; ++q) dst[i][q] = 0.f;
         }
       }
+    };
+    float xa[kTPW][8], xb[kTPW][8];
+    fetch(xa, lane * 8);
+    fetch(xb, lane * 8 + 256);
+    for (int c = lane * 8; c < dc; c += 256) {
+      float xc[kTPW][8];
+      fetch(xc, c + 512);
 #pragma unroll
       for (int e = 0; e < kREC; ++e) {
         float wv[8];
@@ -192,12 +134,15 @@ __global__ void __launch_bounds__(256) logits_simt_kernel(const XT* __restrict__
 #pragma unroll
         for (int i = 0; i < kTPW; ++i)
 #pragma unroll
-          for (int q = 0; q < 8; ++q) acc[i][e] = fmaf(xv[i][q], wv[q], acc[i][e]);
+          for (int q = 0; q < 8; ++q) acc[i][e] = fmaf(xa[i][q], wv[q], acc[i][e]);
       }
 #pragma unroll
       for (int i = 0; i < kTPW; ++i)
 #pragma unroll
-        for (int q = 0; q < 8; ++q) xv[i][q] = xn[i][q];
+        for (int q = 0; q < 8; ++q) {
+          xa[i][q] = xb[i][q];
+          xb[i][q] = xc[i][q];
+        }
     }
   }
   float mine = 0.f;
@@ -214,81 +159,201 @@ __global__ void __launch_bounds__(256) logits_simt_kernel(const XT* __restrict__
 
 // ------------------------------------------------------------------ finish
 // Sum the K-slice partial logits in slice order, add the bias, optionally
-// store the logits, then softmax + top-k.  One warp per token; lane l holds
-// experts l*V .. l*V+V-1.
-template <typename LT, int V>
+// store the logits, then softmax + top-k.  A group of G lanes owns one token
+// (each lane V consecutive experts, 16- or 32-byte loads), so a warp handles
+// 32/G tokens at once; max, sum and the k arg-max rounds are reduced over the
+// group with xor shuffles on (logit descending, expert index ascending).
+// (logit, expert) as one 64-bit key whose unsigned order is "larger logit,
+// then lower expert index": the float's bits mapped to an order-preserving
+// unsigned integer in the high word, the complemented index in the low word.
+__device__ __forceinline__ uint64_t sel_key(float v, int e) {
+  const uint32_t u = __float_as_uint(v);
+  const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+  return (static_cast<uint64_t>(o) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(e));
+}
+__device__ __forceinline__ float key_value(uint64_t key) {
+  const uint32_t o = static_cast<uint32_t>(key >> 32);
+  return __uint_as_float((o & 0x80000000u) ? (o & 0x7fffffffu) : ~o);
+}
+__device__ __forceinline__ int key_index(uint64_t key) {
+  return static_cast<int>(~static_cast<uint32_t>(key));
+}
+
+// 16-bit logits taken as stored (no partial sums, no bias): the same order in
+// one 32-bit key, 16-bit order-preserving value over the complemented index.
+template <typename LT>
+__device__ __forceinline__ uint32_t sel_key16(LT v, int e) {
+  const uint16_t u = *reinterpret_cast<const uint16_t*>(&v);
+  const uint16_t o = (u & 0x8000u) ? static_cast<uint16_t>(~u) : static_cast<uint16_t>(u | 0x8000u);
+  return (static_cast<uint32_t>(o) << 16) | static_cast<uint32_t>(0xffffu - e);
+}
+template <typename LT>
+__device__ __forceinline__ float key16_value(uint32_t key) {
+  const uint16_t o = static_cast<uint16_t>(key >> 16);
+  const uint16_t u = (o & 0x8000u) ? static_cast<uint16_t>(o & 0x7fffu) : static_cast<uint16_t>(~o);
+  return to_f32(*reinterpret_cast<const LT*>(&u));
+}
+
+template <typename LT, int V, int G, bool K16>
 __global__ void __launch_bounds__(256) finish_kernel(const LT* __restrict__ parts, int nsplit, size_t split_stride,
-                                                     const float* __restrict__ bias, int N, int E, int k, int renorm,
-                                                     float* __restrict__ logits_out, int32_t* __restrict__ idx_out,
-                                                     float* __restrict__ w_out) {
+                                                     int pstride, const float* __restrict__ bias, int N, int E,
+                                                     int k, int renorm, float* __restrict__ logits_out,
+                                                     int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  constexpr int TPW = 32 / G;
+  constexpr int kBytes = V * static_cast<int>(sizeof(LT));
+  constexpr float kLog2e = 1.4426950408889634f;
   const int lane = threadIdx.x & 31;
+  const int gl = lane % G, gw = lane / G;
+  const int e_base = gl * V;
   const int warps = gridDim.x * (blockDim.x >> 5);
-  const bool vec = (E == 32 * V) && ((V * sizeof(LT)) % 8 == 0) && ((V * sizeof(LT)) <= 32);
-  for (int t = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < N; t += warps) {
+  const int warp_id = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const bool vec = (E == G * V) && (pstride == E) && (kBytes % 16 == 0);
+  for (int t0 = warp_id * TPW; t0 < N; t0 += warps * TPW) {  // warp-uniform trip count
+    const int t = t0 + gw;
+    const bool tok = t < N;
     float v[V];
-    int ix[V];
+    [[maybe_unused]] uint32_t key16[K16 ? V : 1];
 #pragma unroll
-    for (int i = 0; i < V; ++i) {
-      v[i] = 0.f;
-      ix[i] = lane * V + i < E ? lane * V + i : INT_MAX;
-    }
-    for (int sp = 0; sp < nsplit; ++sp) {
-      const LT* row = parts + sp * split_stride + static_cast<size_t>(t) * E;
-      if (vec) {
-        constexpr int kWords = (V * sizeof(LT) + 7) / 8;  // 8-byte words per lane
-        uint2 raw[kWords > 0 ? kWords : 1];
+    for (int i = 0; i < V; ++i) v[i] = 0.f;
+    if constexpr (K16) {
+      // single stored 16-bit row: keys straight from the raw values
+      LT raw[V];
 #pragma unroll
-        for (int wd = 0; wd < kWords; ++wd) raw[wd] = __ldg(reinterpret_cast<const uint2*>(row + lane * V) + wd);
-        const LT* pv = reinterpret_cast<const LT*>(raw);
+      for (int i = 0; i < V; ++i) raw[i] = LT();
+      if (tok) {
+        const LT* row = parts + static_cast<size_t>(t) * pstride;
+        if (vec) {
 #pragma unroll
-        for (int i = 0; i < V; ++i) v[i] += to_f32(pv[i]);
-      } else {
+          for (int q = 0; q < kBytes / 16; ++q)
+            reinterpret_cast<uint4*>(raw)[q] = __ldg(reinterpret_cast<const uint4*>(row + e_base) + q);
+        } else {
 #pragma unroll
-        for (int i = 0; i < V; ++i)
-          if (ix[i] != INT_MAX) v[i] += to_f32(row[ix[i]]);
+          for (int i = 0; i < V; ++i)
+            if (e_base + i < E) raw[i] = row[e_base + i];
+        }
+      }
+#pragma unroll
+      for (int i = 0; i < V; ++i) {
+        v[i] = to_f32(raw[i]);
+        key16[i] = (tok && e_base + i < E) ? sel_key16(raw[i], e_base + i) : 0u;
+      }
+    } else if (tok) {
+      for (int sp = 0; sp < nsplit; ++sp) {
+        const LT* row = parts + sp * split_stride + static_cast<size_t>(t) * pstride;
+        if (vec) {
+          uint4 raw[kBytes / 16 > 0 ? kBytes / 16 : 1];
+#pragma unroll
+          for (int q = 0; q < kBytes / 16; ++q) raw[q] = __ldg(reinterpret_cast<const uint4*>(row + e_base) + q);
+          const LT* pv = reinterpret_cast<const LT*>(raw);
+#pragma unroll
+          for (int i = 0; i < V; ++i) v[i] += to_f32(pv[i]);
+        } else {
+#pragma unroll
+          for (int i = 0; i < V; ++i)
+            if (e_base + i < E) v[i] += to_f32(row[e_base + i]);
+        }
       }
     }
+    float m = -INFINITY;
 #pragma unroll
     for (int i = 0; i < V; ++i) {
-      if (ix[i] == INT_MAX) {
+      const int e = e_base + i;
+      if (!tok || e >= E) {
         v[i] = -INFINITY;
       } else {
-        if (bias) v[i] += bias[ix[i]];
-        if (logits_out) logits_out[static_cast<size_t>(t) * E + ix[i]] = v[i];
+        if (bias) v[i] += bias[e];
+        if (logits_out) logits_out[static_cast<size_t>(t) * E + e] = v[i];
+      }
+      m = fmaxf(m, v[i]);
+    }
+#pragma unroll
+    for (int o = G / 2; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < V; ++i)
+      if (e_base + i < E) sum += exp2f((v[i] - m) * kLog2e);
+#pragma unroll
+    for (int o = G / 2; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv_sum = 1.0f / sum;
+    float psum = 0.f;
+    if constexpr (K16) {
+      for (int r = 0; r < k; ++r) {
+        uint32_t best = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) best = max(best, key16[i]);
+#pragma unroll
+        for (int o = G / 2; o; o >>= 1) best = max(best, __shfl_xor_sync(0xffffffffu, best, o));
+        const float pr = exp2f((key16_value<LT>(best) - m) * kLog2e) * inv_sum;
+        psum += pr;
+        if (tok && gl == 0) {
+          idx_out[static_cast<size_t>(t) * k + r] = static_cast<int>(0xffffu - (best & 0xffffu));
+          w_out[static_cast<size_t>(t) * k + r] = pr;
+        }
+#pragma unroll
+        for (int i = 0; i < V; ++i) key16[i] = key16[i] == best ? 0u : key16[i];
+      }
+    } else {
+      uint64_t key[V];
+#pragma unroll
+      for (int i = 0; i < V; ++i) key[i] = (e_base + i < E && tok) ? sel_key(v[i], e_base + i) : 0ull;
+      for (int r = 0; r < k; ++r) {
+        uint64_t best = 0;
+#pragma unroll
+        for (int i = 0; i < V; ++i) best = key[i] > best ? key[i] : best;
+#pragma unroll
+        for (int o = G / 2; o; o >>= 1) {
+          const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+          best = other > best ? other : best;
+        }
+        const float pr = exp2f((key_value(best) - m) * kLog2e) * inv_sum;
+        psum += pr;
+        if (tok && gl == 0) {
+          idx_out[static_cast<size_t>(t) * k + r] = key_index(best);
+          w_out[static_cast<size_t>(t) * k + r] = pr;
+        }
+#pragma unroll
+        for (int i = 0; i < V; ++i) key[i] = key[i] == best ? 0ull : key[i];
       }
     }
-    warp_select<V>(v, ix, k, renorm, lane, idx_out + static_cast<size_t>(t) * k,
-                   w_out + static_cast<size_t>(t) * k);
+    if (renorm && tok && gl == 0)
+      for (int r = 0; r < k; ++r) w_out[static_cast<size_t>(t) * k + r] /= psum;
   }
 }
 
+template <typename LT, int V, int G>
+int finish_launch(const void* parts, int nsplit, size_t stride, int pstride, const float* bias, int N, int E, int k,
+                  int renorm, float* lo, int32_t* idx, float* w, cudaStream_t s) {
+  constexpr int TPB = 8 * (32 / G);  // tokens per 256-thread block
+  const int blocks = max(1, min((N + TPB - 1) / TPB, num_sms() * 32));
+  const LT* pp = static_cast<const LT*>(parts);
+  if (sizeof(LT) == 2 && nsplit == 1 && bias == nullptr && E <= 65535)
+    finish_kernel<LT, V, G, sizeof(LT) == 2><<<blocks, 256, 0, s>>>(pp, nsplit, stride, pstride, bias, N, E, k, renorm,
+                                                                     lo, idx, w);
+  else
+    finish_kernel<LT, V, G, false><<<blocks, 256, 0, s>>>(pp, nsplit, stride, pstride, bias, N, E, k, renorm, lo,
+                                                          idx, w);
+  return launch_status(__func__);
+}
+
 template <typename LT>
-int finish_dispatch(const void* parts, int nsplit, size_t stride, const float* bias, int N, int E, int k,
+int finish_dispatch(const void* parts, int nsplit, size_t stride, int pstride, const float* bias, int N, int E, int k,
                     int renorm, float* lo, int32_t* idx, float* w, cudaStream_t s) {
-  const int warps_per_block = 8;
-  const int blocks = max(1, min((N + warps_per_block - 1) / warps_per_block, num_sms() * 16));
-  const LT* lp = static_cast<const LT*>(parts);
-  const int v = (E + 31) / 32;
-#define MOE_FINISH_CASE(VV)                                                                                   \
-  if (v <= VV) {                                                                                             \
-    finish_kernel<LT, VV><<<blocks, warps_per_block * 32, 0, s>>>(lp, nsplit, stride, bias, N, E, k, renorm, lo, \
-                                                                 idx, w);                                    \
-    return launch_status(__func__);                                        \
-  }
-  MOE_FINISH_CASE(1)
-  MOE_FINISH_CASE(2)
-  MOE_FINISH_CASE(4)
-  MOE_FINISH_CASE(8)
-  MOE_FINISH_CASE(16)
-  MOE_FINISH_CASE(32)
-#undef MOE_FINISH_CASE
+#define MOE_FINISH(VV, GG) finish_launch<LT, VV, GG>(parts, nsplit, stride, pstride, bias, N, E, k, renorm, lo, idx, w, s)
+  if (E <= 16) return MOE_FINISH(16, 1);
+  if (E <= 32) return MOE_FINISH(16, 2);
+  if (E <= 64) return MOE_FINISH(16, 4);
+  if (E <= 128) return MOE_FINISH(16, 8);
+  if (E <= 256) return MOE_FINISH(16, 16);
+  if (E <= 512) return MOE_FINISH(16, 32);
+  if (E <= 1024) return MOE_FINISH(32, 32);
+#undef MOE_FINISH
   return MOE_ERR_UNSUPPORTED;
 }
 
 template <typename XT, typename WT>
 int simt_logits(const void* x, const void* Wr, int T, int d, int E, float* logits, cudaStream_t s) {
   dim3 grid((T + kRTok - 1) / kRTok, (E + kREC - 1) / kREC);
-  logits_simt_kernel<XT, WT><<<grid, 256, 0, s>>>(static_cast<const XT*>(x), static_cast<const WT*>(Wr), T, d, E,
+  logits_simt_kernel<XT, WT><<<grid, kRWarps * 32, 0, s>>>(static_cast<const XT*>(x), static_cast<const WT*>(Wr), T, d, E,
                                                   logits);
   return launch_status(__func__);
 }
@@ -300,19 +365,24 @@ int simt_logits(const void* x, const void* Wr, int T, int d, int E, float* logit
 // in flight; the slices' partial logits are summed in slice order by the
 // finish kernel, so the result does not depend on scheduling.
 bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E) {
-  return x_dtype == MOE_BF16 && w_dtype == MOE_BF16 && E % 64 == 0 && d % 64 == 0 && T >= 256 && E >= 64 &&
-         d >= 1024;
+  return x_dtype == MOE_BF16 && w_dtype == MOE_BF16 && d % 64 == 0 && T >= 256 && d >= 512;
 }
+
+int router_padded_experts(int E) { return (E + 63) / 64 * 64; }
 
 int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d, int E,
                   int k, int renorm, float* logits_out, int32_t* idx, float* w, float* parts, int* status,
                   cudaStream_t s) {
   if (T == 0) return MOE_OK;
   int nsplit = 1;
+  int pstride = E;
   int st;
   if (router_uses_tensor_cores(x_dtype, w_dtype, T, d, E)) {
-    const int mma_n = E % 256 == 0 ? 256 : (E % 128 == 0 ? 128 : 64);
-    const int tiles = (T + 127) / 128 * (E / mma_n);
+    // N = E rounded up to 64: the weight rows past E are read as zeros (TMA
+    // fill beyond the tensor) and their logits columns are ignored
+    pstride = router_padded_experts(E);
+    const int mma_n = pstride % 256 == 0 ? 256 : (pstride % 128 == 0 ? 128 : 64);
+    const int tiles = (T + 127) / 128 * (pstride / mma_n);
     nsplit = max(1, min(kRouterMaxSplit, min(num_sms() / max(tiles, 1), d / 64 / 4)));
     GemmArgs g{};
     g.A = x;
@@ -320,10 +390,12 @@ int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, cons
     g.offsets = nullptr;  // one group: all T rows
     g.G = 1;
     g.rows = T;
-    g.N = E;
+    g.N = pstride;
+    g.B_rows = E;
     g.K = d;
     g.ksplit = nsplit;
     g.mma_n = mma_n;
+    g.pair_tiles = -1;
     g.ab_dtype = MOE_BF16;
     g.epilogue = MOE_EPI_NONE;
     g.c_dtype = MOE_F32;
@@ -342,17 +414,17 @@ int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, cons
     return MOE_ERR_UNSUPPORTED;
   }
   if (st != MOE_OK) return st;
-  return finish_dispatch<float>(parts, nsplit, static_cast<size_t>(T) * E, bias, T, E, k, renorm, logits_out, idx, w,
-                                s);
+  return finish_dispatch<float>(parts, nsplit, static_cast<size_t>(T) * pstride, pstride, bias, T, E, k, renorm,
+                                logits_out, idx, w, s);
 }
 
 int launch_topk_logits(const void* logits, int dtype, int N, int E, int k, int renorm, int32_t* idx, float* w,
                        cudaStream_t s) {
   if (N == 0) return MOE_OK;
-  if (dtype == MOE_F16) return finish_dispatch<__half>(logits, 1, 0, nullptr, N, E, k, renorm, nullptr, idx, w, s);
-  if (dtype == MOE_F32) return finish_dispatch<float>(logits, 1, 0, nullptr, N, E, k, renorm, nullptr, idx, w, s);
+  if (dtype == MOE_F16) return finish_dispatch<__half>(logits, 1, 0, E, nullptr, N, E, k, renorm, nullptr, idx, w, s);
+  if (dtype == MOE_F32) return finish_dispatch<float>(logits, 1, 0, E, nullptr, N, E, k, renorm, nullptr, idx, w, s);
   if (dtype == MOE_BF16)
-    return finish_dispatch<__nv_bfloat16>(logits, 1, 0, nullptr, N, E, k, renorm, nullptr, idx, w, s);
+    return finish_dispatch<__nv_bfloat16>(logits, 1, 0, E, nullptr, N, E, k, renorm, nullptr, idx, w, s);
   return MOE_ERR_UNSUPPORTED;
 }
 
