@@ -51,10 +51,10 @@ struct Tile {
   static constexpr int B_BYTES = MMA_N * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TABLE_BYTES = 2 * (kMaxGroups + 2) * 4;
-  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512 - 2048) / STAGE_BYTES;
+  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512 - 4096) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = 2 * MMA_N;
-  static constexpr int EXTRA_BYTES = 2048;  // amax exchange of the E4M3 epilogue
+  static constexpr int EXTRA_BYTES = 4096;  // amax exchange of the E4M3 epilogue
   static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES + EXTRA_BYTES;
 };
 
@@ -665,14 +665,17 @@ __global__ void __launch_bounds__(kThreads, 1)
 // block), so one K block of 128 is one pipeline stage and the scales are
 // applied per K block ("promotion"): the MMA warp writes each block's partial
 // product A_kb B_kb^T into one of two TMEM buffers (kind::f8f6f4, 128 x 256
-// x 32 per instruction) and eight epilogue warps fold it into fp32 registers,
+// x 32 per instruction) and sixteen epilogue warps fold it into fp32
+// registers,
 //     acc[m][n] += partial[m][n] * sa[m, kb] * sb[n/128, kb],
-// while the MMA fills the other buffer.  Epilogue thread = one row and half
-// of the tile's 256 columns: with the SiLU gate, half h owns gate columns
-// [64h, 64h+64) and the matching up columns, so silu(g)*u stays in-thread;
-// the E4M3 output (per row per 128 columns) exchanges the two halves' amax
-// through shared memory under an mbarrier.
-constexpr int kThreadsF8 = 320;
+// while the MMA fills the other buffer.  Epilogue thread = one row and a
+// quarter c of the tile's 256 columns (64 accumulators, so four warps share
+// each TMEM lane quarter and hide each other's load latency): with the SiLU
+// gate, quarter c owns gate columns [32c, 32c+32) and the matching up
+// columns, so silu(g)*u stays in-thread; the E4M3 output (per row per 128
+// columns) exchanges the four quarters' amax through shared memory under an
+// mbarrier.
+constexpr int kThreadsF8 = 576;  // producer, MMA issuer, 16 epilogue warps
 
 template <int EPI, int OUT>  // EPI 1: SiLU gate (OUT 0 bf16 / 2 e4m3); EPI 0: OUT 0 bf16
 __global__ void __launch_bounds__(kThreadsF8, 1)
@@ -698,7 +701,7 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
   int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(smem + L::STAGES * L::STAGE_BYTES + 512);
   int* s_tile = s_off + kMaxGroups + 2;
-  float* s_amax = reinterpret_cast<float*>(s_tile + kMaxGroups + 2);  // [2 parity][2 halves][128 rows]
+  float* s_amax = reinterpret_cast<float*>(s_tile + kMaxGroups + 2);  // [2 parity][4 quarters][128 rows]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G_total;
@@ -745,9 +748,9 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&pfull[a], 1);
-      ptx::mbar_init(&pempty[a], 256);
+      ptx::mbar_init(&pempty[a], 512);
     }
-    ptx::mbar_init(xchg, 256);
+    ptx::mbar_init(xchg, 512);
     ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
@@ -851,14 +854,14 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
       ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
     }
   } else {
-    // -------------------------------------------------------------- epilogue (8 warps)
-    const int q = warp & 3;
-    const int h = (warp - 2) >> 2;  // column half
+    // -------------------------------------------------------------- epilogue (16 warps)
+    const int q = warp & 3;           // TMEM lane quarter this warp may access
+    const int cq = (warp - 2) >> 2;   // column quarter
     const int row_t = q * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
-    // TMEM column offsets of this thread's two 64-column pieces (gate, up) or its 128 columns
-    const int c_lo = EPI ? h * 64 : h * 128;
-    const int c_hi = EPI ? 128 + h * 64 : h * 128 + 64;
+    // TMEM columns of this thread's two 32-column pieces: (gate, up) or one 64-column range
+    const int c_lo = EPI ? 32 * cq : 64 * cq;
+    const int c_hi = EPI ? 128 + 32 * cq : 64 * cq + 32;
     const int nbk = p.K / 128;
     uint32_t pb = 0, puse = 0;
     int it = 0;
@@ -872,24 +875,22 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
       const bool extra = g >= p.G_main;
       const float* bsc = extra ? p.Bx_scales : p.B_scales + static_cast<size_t>(g) * ((EPI ? 2 : 1) * p.N / 128) * nbk;
       // weight-block rows of the two column pieces
-      const int nblk_lo = EPI ? nb : 2 * nb + h;
-      const int nblk_hi = EPI ? p.N / 128 + nb : 2 * nb + h;
+      const int nblk_lo = EPI ? nb : 2 * nb + (cq >> 1);
+      const int nblk_hi = EPI ? p.N / 128 + nb : 2 * nb + (cq >> 1);
       const float* sb_lo = bsc + static_cast<size_t>(nblk_lo) * nbk;
       const float* sb_hi = bsc + static_cast<size_t>(nblk_hi) * nbk;
       const float* sa_row = p.A_scales + grow;
-      float acc[128];
+      float acc[64];
 #pragma unroll
-      for (int i = 0; i < 128; ++i) acc[i] = 0.f;
-      // Scales are fetched well ahead of use so that no K block waits on a
-      // global load: this row's sa[kb] runs through a 4-deep register queue;
-      // the tile's weight-block scales sb[kb] are spread over the lanes in
+      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      // Scales are fetched ahead of use so that no K block waits on a global
+      // load: this row's sa[kb] runs through a 2-deep register queue; the
+      // tile's weight-block scales sb[kb] are spread over the lanes in
       // windows of 32 K blocks (lane j holds block w + j) and broadcast with
       // a shuffle, the next window being loaded halfway through the current.
       const size_t rstride = static_cast<size_t>(p.rows);
       float sa0 = (valid && 0 < nbk) ? __ldg(sa_row) : 0.f;
       float sa1 = (valid && 1 < nbk) ? __ldg(sa_row + rstride) : 0.f;
-      float sa2 = (valid && 2 < nbk) ? __ldg(sa_row + 2 * rstride) : 0.f;
-      float sa3 = (valid && 3 < nbk) ? __ldg(sa_row + 3 * rstride) : 0.f;
       float wl = lane < nbk ? __ldg(sb_lo + lane) : 0.f;
       float wh = lane < nbk ? __ldg(sb_hi + lane) : 0.f;
       float nwl = 0.f, nwh = 0.f;
@@ -905,9 +906,7 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
         }
         const float sa = sa0;
         sa0 = sa1;
-        sa1 = sa2;
-        sa2 = sa3;
-        sa3 = (valid && kb + 4 < nbk) ? __ldg(sa_row + static_cast<size_t>(kb + 4) * rstride) : 0.f;
+        sa1 = (valid && kb + 2 < nbk) ? __ldg(sa_row + static_cast<size_t>(kb + 2) * rstride) : 0.f;
         const float m_lo = sa * __shfl_sync(0xffffffffu, wl, kb & 31);
         const float m_hi = sa * __shfl_sync(0xffffffffu, wh, kb & 31);
         if (!ptx::mbar_wait_warp(&pfull[pb], puse & 1, abort_flag, kWaitLimitNs)) {
@@ -917,11 +916,11 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
         ptx::tc_fence_after();
         const uint32_t t0 = lane_base + pb * MMA_N;
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
+        for (int j = 0; j < 8; ++j) {
           uint32_t v[8];
-          ptx::tmem_ld_32x32b_x8(t0 + (j < 8 ? c_lo : c_hi) + (j & 7) * 8, v);
+          ptx::tmem_ld_32x32b_x8(t0 + (j < 4 ? c_lo : c_hi) + (j & 3) * 8, v);
           ptx::tmem_ld_wait();
-          const float m = j < 8 ? m_lo : m_hi;
+          const float m = j < 4 ? m_lo : m_hi;
 #pragma unroll
           for (int i = 0; i < 8; ++i) acc[8 * j + i] = fmaf(__uint_as_float(v[i]), m, acc[8 * j + i]);
         }
@@ -933,54 +932,55 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
       if (!ok) break;
       if constexpr (EPI == 1) {
 #pragma unroll
-        for (int i = 0; i < 64; ++i) {
+        for (int i = 0; i < 32; ++i) {
           const float gt = acc[i];
-          acc[i] = gt / (1.0f + __expf(-gt)) * acc[64 + i];
+          acc[i] = gt / (1.0f + __expf(-gt)) * acc[32 + i];
         }
         if constexpr (OUT == 2) {
           float amax = 0.f;
 #pragma unroll
-          for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(acc[i]));
-          float* xa = s_amax + (it & 1) * 256;
-          xa[h * 128 + row_t] = amax;
+          for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+          float* xa = s_amax + (it & 1) * 512;
+          xa[cq * 128 + row_t] = amax;
           ptx::mbar_arrive(xchg);
           if (!ptx::mbar_wait_warp(xchg, it & 1, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
           }
-          amax = fmaxf(xa[row_t], xa[128 + row_t]);
+          amax = fmaxf(fmaxf(xa[row_t], xa[128 + row_t]), fmaxf(xa[256 + row_t], xa[384 + row_t]));
           const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
           if (valid) {
-            uint32_t qw[16];
+            uint32_t qw[8];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 8; ++i) {
               const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc));
               const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc));
               qw[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
             }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.C) + grow * p.N + nb * 128 + h * 64);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(qw[4 * v], qw[4 * v + 1], qw[4 * v + 2], qw[4 * v + 3]);
-            if (h == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.C) + grow * p.N + nb * 128 + cq * 32);
+            dst[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+            dst[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
+            if (cq == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
           }
         } else {
           if (valid) {
-            uint32_t pk[32];
+            uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
+            for (int i = 0; i < 16; ++i) {
               const __nv_bfloat162 hb = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
               pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
             }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 128 + h * 64);
+            uint4* dst =
+                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 128 + cq * 32);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
         }
       } else {
         if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 256 + h * 128);
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 256 + cq * 64);
 #pragma unroll
-          for (int v = 0; v < 16; ++v) {
+          for (int v = 0; v < 8; ++v) {
             uint32_t pk[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
