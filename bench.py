@@ -53,6 +53,21 @@ def log(*a):
     print(*a, file=sys.stderr, flush=True)
 
 
+# --------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, world: int, device="cpu") -> float:
+    """The largest value of x over all ranks (the job is as slow as its slowest rank)."""
+    if world <= 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_tokens_per_s(tokens_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput of independent replicas: every rank's tokens over the slowest rank's step."""
+    return world * tokens_per_rank / (ms_per_step_max * 1e-3)
+
+
 def load_peaks():
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
@@ -399,11 +414,7 @@ def run_ours(args, rank, world, dev):
     status = gg.read_device_status(ws)
     if status != 0:
         raise RuntimeError(f"device status {status}")
-    ms = float(np.mean(times))
-    if world > 1:
-        t = torch.tensor([ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(float(np.mean(times)), world, dev)
 
     # --- e2e: host buffers through moe_forward_host, copies inside the timed region
     xh = inp["x"].cpu().pin_memory()
@@ -413,11 +424,7 @@ def run_ours(args, rank, world, dev):
         gg.moe_forward_host(cfg, xh, inp["W_r"], inp["bias"], weights, oh, ws)
 
     e2e_times = time_steps(step_host, max(3, args.steps // 2), 2, flush, stream, hold=False)
-    e2e_ms = float(np.mean(e2e_times))
-    if world > 1:
-        t = torch.tensor([e2e_ms], device=dev)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(float(np.mean(e2e_times)), world, dev)
 
     # --- per-kernel breakdown (staged calls of the same kernels)
     kern = {}
@@ -458,24 +465,29 @@ def main():
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
-    if args.config == "router_micro":
-        return run_router_micro(args, rank, world, local)
-    s = shape_of(args.config, **args.overrides)
-
     if args.impl == "reference":
-        if rank != 0:
+        if rank != 0:  # the CPU reference arm runs on rank 0 only
             return 0
-        return run_reference(args, s, world)
+        if args.config == "router_micro":
+            return run_router_micro(args, rank, world, local)
+        return run_reference(args, shape_of(args.config, **args.overrides), world)
 
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
+    if args.config == "router_micro":
+        rc = run_router_micro(args, rank, world, local)
+        if world > 1:
+            torch.distributed.barrier()
+            torch.distributed.destroy_process_group()
+        return rc
+    s = shape_of(args.config, **args.overrides)
     r = run_ours(args, rank, world, local)
     peaks, peak_kind = load_peaks()
     result = None
     if rank == 0:
         T = s.T
-        value = world * T / (r["ms"] * 1e-3)
+        value = job_tokens_per_s(T, world, r["ms"])
         alg = algorithmic(s, r["counts"])
         up = r["kernels"].get("up_gemm")
         roof = None
@@ -505,7 +517,7 @@ def main():
             "gemm_frac_of_peak": round(gemm_flops / (r["ms"] * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4),
             "roofline": roof,
             "kernels": r["kernels"],
-            "e2e": {"value": round(world * T / (r["e2e_ms"] * 1e-3), 1), "unit": "tokens/s",
+            "e2e": {"value": round(job_tokens_per_s(T, world, r["e2e_ms"]), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * s.d * (4 if s.x_dtype == "f32" else 2),
                     "d2h_bytes_per_step": T * s.d * (4 if r["out_dtype"] == torch.float32 else 2)},
             "gpu_launches": KERNELS_PER_FORWARD * args.steps,
@@ -575,9 +587,11 @@ def run_router_micro(args, rank, world, local):
     def step():
         gg.topk_logits(logits, k, out_idx=idx, out_w=w)
 
+    if world > 1:
+        torch.distributed.barrier()
     with ClockSampler(dev) as clk:
         times = time_steps(step, args.steps, args.warmup, lambda: scrub.fill_(1), stream)
-    ms = float(np.mean(times))
+    ms = max_over_ranks(float(np.mean(times)), world, dev)
     lh = logits.cpu().pin_memory()
     ih = torch.empty((N, k), dtype=torch.int32).pin_memory()
     wh = torch.empty((N, k), dtype=torch.float32).pin_memory()
@@ -588,11 +602,11 @@ def run_router_micro(args, rank, world, local):
         ih.copy_(idx, non_blocking=True)
         wh.copy_(w, non_blocking=True)
 
-    e2e_ms = float(np.mean(time_steps(step_host, max(3, args.steps // 2), 2, lambda: scrub.fill_(1), stream,
-                                      hold=False)))
+    e2e_ms = max_over_ranks(float(np.mean(time_steps(step_host, max(3, args.steps // 2), 2,
+                                                     lambda: scrub.fill_(1), stream, hold=False))), world, dev)
     peaks, kind = load_peaks()
     achieved = bytes_per_step / (ms * 1e-3) / 1e9
-    result = {"metric": METRIC, "value": round(world * N / (ms * 1e-3), 1), "unit": "tokens/s", "n_gpus": world,
+    result = {"metric": METRIC, "value": round(job_tokens_per_s(N, world, ms), 1), "unit": "tokens/s", "n_gpus": world,
               "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
               "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": desc,
               "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": float(peaks["hbm_gbs"]),
@@ -600,7 +614,7 @@ def run_router_micro(args, rank, world, local):
                            "kernel": "finish_kernel (softmax + top-k of stored logits)",
                            "peak_kind": f"{kind} HBM copy bandwidth"},
               "kernel_us": round(ms * 1e3, 2),
-              "e2e": {"value": round(world * N / (e2e_ms * 1e-3), 1), "unit": "tokens/s",
+              "e2e": {"value": round(job_tokens_per_s(N, world, e2e_ms), 1), "unit": "tokens/s",
                       "h2d_bytes_per_step": N * E * 2, "d2h_bytes_per_step": N * k * 8},
               "gpu_launches": args.steps, "clocks": clk.summary()}
     if rank == 0:

@@ -64,6 +64,8 @@ _SIGS = {
     "moe_grouped_gemm_workspace_size": (_sz, []),
     "moe_grouped_gemm": (_i, [_vp, _fp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _vp, _i, _fp, _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _ip, _fp, _i, _i, _i, _i, _vp, _i, _vp]),
+    "moe_selftest_workspace_size": (_sz, []),
+    "moe_selftest_stalled_pipeline": (_i, [_vp, _sz, ctypes.c_ulonglong, _vp]),
     "moe_quantize_weights_fp8": (_i, [_vp, _i, _i, _i, _vp, _fp, _vp]),
     "moe_workspace_size": (_sz, [_CFG]),
     "moe_forward": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _ip, _vp, _sz, _vp]),

@@ -89,6 +89,9 @@ struct GemmArgs {
   int ksplit;               // > 1: fp32 partial products of K slices at C + s * rows * N (no epilogue)
   int mma_n;                // 0 = widest tile that divides N; else 64 / 128 / 256 (no-gate GEMMs)
   int pair_tiles;           // 256-row tiles on CTA pairs: 0 = by average group size, 1 = always, -1 = never
+  uint64_t wait_ns;         // pipeline wait limit (0 = the default of 2 s)
+  int stall;                // failure-detection self-test (see moe_selftest_stalled_pipeline)
+  int grid;                 // CTAs (0 = one per SM)
   int ab_dtype, epilogue, c_dtype;
   void* C;
   float* C_scales;

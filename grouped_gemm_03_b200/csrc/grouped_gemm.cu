@@ -72,6 +72,8 @@ struct Params {
   const float* B_scales;   // [G_main][Nb/128][K/128]
   const float* Bx_scales;  // [Nb/128][K/128] of the extra group
   float* C_scales;         // [N/128][rows] when C is E4M3
+  uint64_t wait_ns;        // limit of every pipeline wait
+  int stall;               // self-test: the epilogue first waits on a barrier no thread arrives at
 };
 
 struct TileCoord {
@@ -122,7 +124,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* tfull = empty + L::STAGES;
   uint64_t* tempty = tfull + 2;
   uint64_t* drain = tempty + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  uint64_t* never = drain + 1;  // self-test only: initialised, never arrived at
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(never + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
   int* s_off = reinterpret_cast<int*>(smem + L::STAGES * L::STAGE_BYTES + 512);
@@ -179,6 +182,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::mbar_init(&tempty[a], 128);
     }
     ptx::mbar_init(drain, 1);
+    ptx::mbar_init(never, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
     ptx::prefetch_tmap(&tmB);
@@ -210,7 +214,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int gb = extra ? 0 : g;
         const int kb0 = tc.ks * nk / p.ksplit, kb1 = (tc.ks + 1) * nk / p.ksplit;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -244,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           } else {
             --s;
           }
-          ptx::mbar_wait(&full[s], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+          ptx::mbar_wait(&full[s], ph, reinterpret_cast<volatile int*>(s_bad), p.wait_ns);
         }
       }
     }
@@ -257,7 +261,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
         const int acc = it & 1;
         const uint32_t use = static_cast<uint32_t>(it >> 1);
-        if (!ptx::mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+        if (!ptx::mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, p.wait_ns)) {
           ok = false;
           break;
         }
@@ -266,7 +270,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int ks = decode_tile(s_tile, s_off, G, nt, tile).ks;
         const int kb0 = ks * nk / p.ksplit, kb1 = (ks + 1) * nk / p.ksplit;
         for (int kb = kb0; kb < kb1; ++kb) {
-          if (!ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag, p.wait_ns)) {
             ok = false;
             break;
           }
@@ -291,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       // every MMA issued must finish before TMEM is released
       ptx::umma_commit(drain);
-      ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+      ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), p.wait_ns);
     }
   } else {
     // -------------------------------------------------------------- epilogue
@@ -307,7 +311,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int r_in = tc.mb * BM + row_t;
       const bool valid = r_in < m_g;
       const size_t grow = static_cast<size_t>(s_off[g] + r_in);
-      if (!ptx::mbar_wait_warp(&tfull[acc], use & 1, abort_flag, kWaitLimitNs)) {
+      if (p.stall && it == 0 && !ptx::mbar_wait_warp(never, 0, abort_flag, p.wait_ns)) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        break;
+      }
+      if (!ptx::mbar_wait_warp(&tfull[acc], use & 1, abort_flag, p.wait_ns)) {
         *abort_flag = 1;
         set_status(p.status, MOE_ERR_TIMEOUT);
         break;
@@ -1078,7 +1087,9 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   p.split_stride = static_cast<size_t>(a.rows) * a.N;
   p.C = a.C;
   p.status = a.status;
-  gg_bf16_kernel<MMA_N, EPI, OUT><<<num_sms(), kThreads, L::SMEM, s>>>(mA, mB, mBx, p);
+  p.wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
+  p.stall = a.stall;
+  gg_bf16_kernel<MMA_N, EPI, OUT><<<a.grid > 0 ? a.grid : num_sms(), kThreads, L::SMEM, s>>>(mA, mB, mBx, p);
   return launch_status(__func__);
 }
 

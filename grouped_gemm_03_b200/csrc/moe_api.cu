@@ -253,6 +253,39 @@ int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const 
   return launch_grouped_gemm(a, s);
 }
 
+// ------------------------------------------------------------------ failure-detection self-test
+size_t moe_selftest_workspace_size(void) { return 1024 + (16 + 128 + 256) * 1024; }
+
+int moe_selftest_stalled_pipeline(void* ws, size_t ws_bytes, unsigned long long wait_limit_ns, void* stream) {
+  if (!ws || !aligned(ws, 256) || ws_bytes < moe_selftest_workspace_size()) return MOE_ERR_WORKSPACE;
+  if (wait_limit_ns < 1000000ull || wait_limit_ns > 2000000000ull) return MOE_ERR_INVALID;
+  cudaStream_t s = as_stream(stream);
+  char* base = static_cast<char*>(ws);
+  void* A = base + 1024;                 // [128, 64] bf16
+  void* B = base + 1024 + 16 * 1024;     // [1024, 64] bf16
+  void* C = base + 1024 + 144 * 1024;    // [128, 1024] bf16
+  MOE_CUDA_CHECK(cudaMemsetAsync(ws, 0, 1024 + 144 * 1024, s));
+  GemmArgs g{};
+  g.A = A;
+  g.B = B;
+  g.offsets = nullptr;  // one group of 128 rows: four 256-column tiles on one CTA
+  g.G = 1;
+  g.rows = 128;
+  g.N = 1024;
+  g.K = 64;
+  g.mma_n = 256;
+  g.pair_tiles = -1;
+  g.ab_dtype = MOE_BF16;
+  g.epilogue = MOE_EPI_NONE;
+  g.c_dtype = MOE_BF16;
+  g.C = C;
+  g.status = static_cast<int*>(ws);
+  g.wait_ns = wait_limit_ns;
+  g.stall = 1;
+  g.grid = 1;
+  return launch_grouped_gemm(g, s);
+}
+
 // ------------------------------------------------------------------ combine
 int moe_combine(const void* Y, const int32_t* token_to_row, const float* topk_w, int has_shared, int T, int d, int k,
                 void* out, int out_dtype, void* stream) {

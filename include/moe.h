@@ -193,6 +193,20 @@ int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const 
                      const int32_t* offsets, int G, int rows, int N, int K, int ab_dtype, int epilogue,
                      void* C, int c_dtype, float* C_scales, void* ws, size_t ws_bytes, void* stream);
 
+/* ---------------------------------------------------------------- failure detection
+ * Self-test of the grouped GEMM's failure path (no counterpart on the source
+ * pages): launches the bf16 grouped-GEMM kernel on one CTA over a small
+ * problem carved from `ws` (four tiles), whose epilogue first waits on a
+ * barrier that no thread ever arrives at.  That wait gives up after
+ * wait_limit_ns (1e6 .. 2e9); the kernel then raises its abort flag, the
+ * producer waits for the copies it has in flight, the MMA issuer drains its
+ * MMAs, TMEM is released and the kernel returns, leaving MOE_ERR_TIMEOUT in
+ * the status word at the start of ws (read it with moe_read_device_status).
+ * No fault, trap or unbounded wait is involved; the context stays usable.
+ * ws: moe_selftest_workspace_size() bytes, 256-byte aligned. */
+size_t moe_selftest_workspace_size(void);
+int moe_selftest_stalled_pipeline(void* ws, size_t ws_bytes, unsigned long long wait_limit_ns, void* stream);
+
 /* ---------------------------------------------------------------- combine
  * Step 6 of "Dense GEMM -> GroupedGEMM -> TP MoE" §2.2 and the sum of
  * "MegaMoE ..." §2.1:

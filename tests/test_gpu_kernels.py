@@ -257,3 +257,30 @@ def test_quantize_weights_bit_exact(G, N, K):
         wq, ws_ = ofp8.quantize_128x128(f64(W[g]).astype(np.float32))
         assert np.array_equal(q[g].cpu().numpy(), wq)
         assert np.array_equal(s[g].cpu().numpy(), ws_)
+
+
+# ---------------------------------------------------------------- failure detection
+def test_stalled_pipeline_times_out_and_context_survives():
+    import time
+    L = gg.lib()
+    ws = torch.zeros(L.moe_selftest_workspace_size(), dtype=torch.uint8, device=DEV)
+    t0 = time.perf_counter()
+    st = L.moe_selftest_stalled_pipeline(gg._ptr(ws), ws.numel(), 50_000_000, gg._stream())
+    assert st == 0
+    assert gg.read_device_status(ws) == -6  # MOE_ERR_TIMEOUT
+    assert time.perf_counter() - t0 < 10.0
+    # the context is intact: a normal grouped GEMM still computes the right thing
+    sizes = [200, 57]
+    A = torch.randn((257, 128), device=DEV).to(torch.bfloat16)
+    B = (torch.randn((2, 256, 128), device=DEV) * 0.05).to(torch.bfloat16)
+    gws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    C = gg.grouped_gemm(A, B, _offsets(sizes), 256, ws=gws)
+    assert gg.read_device_status(gws) == 0
+    assert rel_fro(f64(C), _gemm_ref(A, B, sizes, gg.EPI_NONE, 256)) < 2e-3
+
+
+def test_selftest_rejects_bad_arguments():
+    L = gg.lib()
+    ws = torch.zeros(L.moe_selftest_workspace_size(), dtype=torch.uint8, device=DEV)
+    assert L.moe_selftest_stalled_pipeline(gg._ptr(ws), 100, 50_000_000, gg._stream()) == -3
+    assert L.moe_selftest_stalled_pipeline(gg._ptr(ws), ws.numel(), 10, gg._stream()) == -1
