@@ -92,6 +92,7 @@ struct GemmArgs {
   uint64_t wait_ns;         // pipeline wait limit (0 = the default of 2 s)
   int stall;                // failure-detection self-test (see moe_selftest_stalled_pipeline)
   int grid;                 // CTAs (0 = one per SM)
+  int swap_ab;              // weights on the MMA's 128-row side: 0 = for small groups, 1 = always, -1 = never
   int ab_dtype, epilogue, c_dtype;
   void* C;
   float* C_scales;

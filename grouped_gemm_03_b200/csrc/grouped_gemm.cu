@@ -389,6 +389,263 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 }
 
+// ------------------------------------------------------------------ swap-AB bf16 kernel (small groups)
+// Decode-shaped problems give each expert a handful of tokens.  Here the
+// weights are the 128-row MMA operand and the tokens the narrow one:
+// D[128 weight rows, NT tokens] = W_tile . X_tile^T, so a tile streams 16 KB
+// of weights and only NT x 128 B of activations per k-step (the
+// activation-major kernel would stream a 128-row activation tile, mostly rows
+// of other experts, as many bytes as the weights).  With the SiLU gate the
+// 128 weight rows are four 32-row chunks [16 gate rows; the 16 matching up
+// rows], so lane l < 16 of a warp holds gate(col l) and lane l + 16 holds
+// up(col l): one shuffle pairs them.  Each thread owns one output column and
+// writes it for the tile's tokens.
+constexpr int kSwapNT = 32;     // tokens per tile (MMA N)
+constexpr int kSwapStages = 8;  // (16 KB weights + 4 KB tokens) per stage
+constexpr int kSwapSmem = 1024 + kSwapStages * (16384 + kSwapNT * 128) + 512 + 2 * (kMaxGroups + 2) * 4;
+
+template <int EPI>
+__global__ void __launch_bounds__(kThreads, 1)
+    gg_bf16_swap_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
+                        const __grid_constant__ CUtensorMap tmWx, const Params p) {
+  constexpr int NT = kSwapNT;
+  constexpr int W_BYTES = 128 * 128;
+  constexpr int X_BYTES = NT * 128;
+  constexpr int STAGES = kSwapStages;
+  constexpr int COLS = EPI ? 64 : 128;  // output columns per tile
+  constexpr int TMEM_COLS = 2 * NT;
+  constexpr uint32_t IDESC = ptx::make_idesc(128, NT, 1);
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sW = smem;
+  uint8_t* sX = smem + STAGES * W_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(sX + STAGES * X_BYTES);
+  uint64_t* empty = full + STAGES;
+  uint64_t* tfull = empty + STAGES;
+  uint64_t* tempty = tfull + 2;
+  uint64_t* drain = tempty + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + STAGES * (W_BYTES + X_BYTES) + 512);
+  int* s_tile = s_off + kMaxGroups + 2;
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G_total;
+  const int nt = p.N / COLS;
+
+  if (warp == 0) {
+    for (int g = lane; g <= G; g += 32) s_off[g] = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
+    __syncwarp();
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int bad = 0, mine = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int m = s_off[g + 1] - s_off[g];
+      if (m < 0) bad = 1;
+      mine += (max(m, 0) + NT - 1) / NT * nt;
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - mine;
+    for (int g = g0; g < g1; ++g) {
+      s_tile[g] = run;
+      run += (max(s_off[g + 1] - s_off[g], 0) + NT - 1) / NT * nt;
+    }
+    if (lane == 31) s_tile[G] = incl;
+    if (lane == 0 && (s_off[0] != 0 || s_off[G] > p.rows)) bad = 1;
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      *s_bad = bad;
+      *abort_flag = 0;
+      if (bad && blockIdx.x == 0) set_status(p.status, MOE_ERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  if (*s_bad) return;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      ptx::mbar_init(&full[s], 1);
+      ptx::mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      ptx::mbar_init(&tfull[a], 1);
+      ptx::mbar_init(&tempty[a], 128);
+    }
+    ptx::mbar_init(drain, 1);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmX);
+    ptx::prefetch_tmap(&tmW);
+    ptx::prefetch_tmap(&tmWx);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, TMEM_COLS);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tile[G];
+  const int nk = p.K / 64;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ producer
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const int g = find_group(s_tile, G, tile);
+        const int m_g = s_off[g + 1] - s_off[g];
+        const int mt = (m_g + NT - 1) / NT;
+        const int tl = tile - s_tile[g];
+        const int nb = tl / mt, tb = tl % mt;
+        const int x_row = s_off[g] + tb * NT;
+        const bool extra = g >= p.G_main;
+        const CUtensorMap* mW = extra ? &tmWx : &tmW;
+        const int gb = extra ? 0 : g;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&full[stage], W_BYTES + X_BYTES);
+          uint8_t* w = sW + stage * W_BYTES;
+          if (EPI) {
+            // one 4-D box {64 k, 16 rows, gate/up, 4 chunks}: chunk c lands as
+            // [16 gate rows; the 16 up rows of the same output columns]
+            ptx::tma_load_4d(w, mW, &full[stage], kb * 64, 0, 0, (gb * 2 * p.N + nb * 64) / 16);
+          } else {
+            ptx::tma_load_2d(w, mW, &full[stage], kb * 64, gb * p.N + nb * 128);
+          }
+          ptx::tma_load_2d(sX + stage * X_BYTES, &tmX, &full[stage], kb * 64, x_row);
+          ++issued;
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        const uint32_t pending = issued < static_cast<uint32_t>(STAGES) ? issued : STAGES;
+        uint32_t s = stage, ph = phase;
+        for (uint32_t i = 0; i < pending; ++i) {
+          if (s == 0) {
+            s = STAGES - 1;
+            ph ^= 1;
+          } else {
+            --s;
+          }
+          ptx::mbar_wait(&full[s], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int it = 0;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t use = static_cast<uint32_t>(it >> 1);
+        if (!ptx::mbar_wait(&tempty[acc], (use & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * NT;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint64_t adesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sW + stage * W_BYTES));
+          const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sX + stage * X_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | kk) != 0);
+          ptx::umma_commit(&empty[stage]);
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        ptx::umma_commit(&tfull[acc]);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+      }
+      ptx::umma_commit(drain);
+      ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue
+    const int q = warp & 3;  // TMEM lane quarter = weight rows 32q .. 32q+31
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t use = static_cast<uint32_t>(it >> 1);
+      const int g = find_group(s_tile, G, tile);
+      const int m_g = s_off[g + 1] - s_off[g];
+      const int mt = (m_g + NT - 1) / NT;
+      const int tl = tile - s_tile[g];
+      const int nb = tl / mt, tb = tl % mt;
+      const int ntok = min(NT, m_g - tb * NT);  // valid tokens of this tile
+      const size_t row0 = static_cast<size_t>(s_off[g] + tb * NT);
+      if (!ptx::mbar_wait_warp(&tfull[acc], use & 1, abort_flag, kWaitLimitNs)) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        break;
+      }
+      ptx::tc_fence_after();
+      uint32_t v[32];
+      ptx::tmem_ld_32x32b_x32(lane_base + acc * NT, v);
+      ptx::tmem_ld_wait();
+      ptx::tc_fence_before();
+      ptx::mbar_arrive(&tempty[acc]);  // the values are in registers: release the accumulator early
+      __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C);
+      if constexpr (EPI == 1) {
+        // lanes 0..15: gate of column c; lanes 16..31: up of the same column
+        const int col = nb * 64 + q * 16 + (lane & 15);
+#pragma unroll
+        for (int t = 0; t < NT; ++t) {
+          const float mine = __uint_as_float(v[t]);
+          const float up = __shfl_xor_sync(0xffffffffu, mine, 16);
+          if (lane < 16 && t < ntok) {
+            const float hval = mine / (1.0f + __expf(-mine)) * up;
+            C[(row0 + t) * p.N + col] = __float2bfloat16_rn(hval);
+          }
+        }
+      } else {
+        const int col = nb * 128 + q * 32 + lane;
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+          if (t < ntok) C[(row0 + t) * p.N + col] = __float2bfloat16_rn(__uint_as_float(v[t]));
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, TMEM_COLS);
+  }
+}
+
 // ------------------------------------------------------------------ CTA-pair bf16 kernel
 // For large groups (the compute-bound Mixtral-shaped layer) two SMs of a
 // cluster share one 256-row tile: each CTA stages its own 128 rows of A and
@@ -1055,6 +1312,32 @@ bool make_map(CUtensorMap* m, const void* base, int ebytes, uint64_t rows, uint6
   return true;
 }
 
+// 4-D view of stacked [G][2N][K] bf16 gate/up weights for the swap-AB kernel:
+// (k, row r of a 16-row chunk, half h = gate/up, chunk c) -> row c*16 + r + h*N.
+// Chunks run over all groups' rows; only gate chunks are addressed, the up
+// half adds N rows, so the outermost extent stops N rows short of the end.
+bool make_gateup_map(CUtensorMap* m, const void* base, int G, int N, int K) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) {
+    record_cuda_error(cudaErrorNotSupported, "cuTensorMapEncodeTiled unavailable from the driver");
+    return false;
+  }
+  const uint64_t rowb = static_cast<uint64_t>(K) * 2;
+  const cuuint64_t dims[4] = {static_cast<cuuint64_t>(K), 16, 2,
+                              (static_cast<cuuint64_t>(G) * 2 * N - N) / 16};
+  const cuuint64_t strides[3] = {rowb, rowb * N, rowb * 16};
+  const cuuint32_t box[4] = {64, 16, 2, 4};
+  const cuuint32_t estr[4] = {1, 1, 1, 1};
+  const CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    record_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled rejected the gate/up layout");
+    return false;
+  }
+  return true;
+}
+
 template <int MMA_N, int EPI, int OUT>
 int run_bf16(const GemmArgs& a, cudaStream_t s) {
   using L = Tile<MMA_N>;
@@ -1090,6 +1373,43 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   p.wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
   p.stall = a.stall;
   gg_bf16_kernel<MMA_N, EPI, OUT><<<a.grid > 0 ? a.grid : num_sms(), kThreads, L::SMEM, s>>>(mA, mB, mBx, p);
+  return launch_status(__func__);
+}
+
+template <int EPI>
+int run_bf16_swap(const GemmArgs& a, cudaStream_t s) {
+  static_assert(kSwapSmem <= 227 * 1024, "shared memory budget");
+  const int nb_rows = EPI ? 2 * a.N : a.N;
+  CUtensorMap mX, mW, mWx;
+  if (!make_map(&mX, a.A, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, kSwapNT)) return MOE_ERR_CUDA;
+  const int G = a.G > 0 ? a.G : 1;
+  if (EPI) {
+    if (!make_gateup_map(&mW, a.B, G, a.N, a.K)) return MOE_ERR_CUDA;
+    if (!make_gateup_map(&mWx, a.has_extra ? a.B_extra : a.B, 1, a.N, a.K)) return MOE_ERR_CUDA;
+  } else {
+    if (!make_map(&mW, a.B, 2, static_cast<uint64_t>(G) * nb_rows, a.K, 128)) return MOE_ERR_CUDA;
+    if (!make_map(&mWx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, 128)) return MOE_ERR_CUDA;
+  }
+  static bool attr_set[64] = {};
+  int dev = 0;
+  MOE_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    MOE_CUDA_CHECK(
+        cudaFuncSetAttribute(gg_bf16_swap_kernel<EPI>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSwapSmem));
+    attr_set[dev] = true;
+  }
+  Params p{};
+  p.offsets = a.offsets;
+  p.G_total = a.G + a.has_extra;
+  p.G_main = a.G;
+  p.N = a.N;
+  p.K = a.K;
+  p.rows = a.rows;
+  p.ksplit = 1;
+  p.C = a.C;
+  p.status = a.status;
+  gg_bf16_swap_kernel<EPI><<<num_sms(), kThreads, kSwapSmem, s>>>(mX, mW, mWx, p);
   return launch_status(__func__);
 }
 
@@ -1181,10 +1501,21 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
 int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
   if (a.G + a.has_extra == 0 || a.rows == 0) return MOE_OK;
   if (a.ab_dtype == MOE_BF16) {
-    // CTA pairs pay off when tiles of 256 rows are mostly full: large groups on average
+    // CTA pairs pay off when tiles of 256 rows are mostly full: large groups on average;
+    // groups of a few tokens (decode) put the weights on the 128-row side instead
     const bool pairs = a.pair_tiles > 0 || (a.pair_tiles == 0 && a.rows >= 512 * (a.G + a.has_extra));
+    const bool swap = a.swap_ab > 0 || (a.swap_ab == 0 && a.ksplit <= 1 && a.c_dtype == MOE_BF16 &&
+                                        a.rows < 32 * (a.G + a.has_extra));
+    if (swap && a.ksplit <= 1 && a.c_dtype == MOE_BF16) {
+      if (a.epilogue == MOE_EPI_SILU_GATE && a.N % 64 == 0) return run_bf16_swap<1>(a, s);
+      if (a.epilogue == MOE_EPI_NONE && a.N % 128 == 0) return run_bf16_swap<0>(a, s);
+    }
     if (a.epilogue == MOE_EPI_SILU_GATE) {
-      if (a.c_dtype != MOE_BF16 || a.N % 128 != 0 || a.ksplit > 1) return MOE_ERR_UNSUPPORTED;
+      if (a.c_dtype != MOE_BF16 || a.N % 64 != 0 || a.ksplit > 1) return MOE_ERR_UNSUPPORTED;
+      // few rows (decode): 64-column output tiles (64 gate + 64 up rows of B) give
+      // twice the tiles, so the weight stream spreads over the SMs more evenly
+      const bool narrow = a.mma_n == 128 || a.N % 128 != 0 || (a.mma_n == 0 && a.rows < 64 * num_sms());
+      if (narrow) return run_bf16<128, 1, 0>(a, s);
       return pairs ? run_bf16_pair<1, 0>(a, s) : run_bf16<256, 1, 0>(a, s);
     }
     if (pairs && a.ksplit <= 1 && a.N % 256 == 0 && (a.mma_n == 0 || a.mma_n == 256))

@@ -182,6 +182,12 @@ GEMM_CASES = [
     ([2000, 0, 129], 512, 128, gg.EPI_NONE, torch.float32),
     ([257, 1600, 0, 255], 128, 320, gg.EPI_SILU_GATE, torch.bfloat16),
     ([1536, 1], 256, 512, gg.EPI_SILU_GATE, torch.bfloat16),
+    # a few tokens per group (fewer than 32 rows per group on average): the weights take the
+    # MMA's 128-row side (swap-AB), tokens the 32-wide side
+    ([1, 0, 3, 2, 5, 33, 0, 1, 0, 7, 64, 1], 256, 128, gg.EPI_NONE, torch.bfloat16),
+    ([2, 0, 1, 40, 3, 0, 0, 9], 192, 320, gg.EPI_SILU_GATE, torch.bfloat16),
+    ([31, 32, 33, 0, 1], 128, 64, gg.EPI_NONE, torch.bfloat16),
+    ([65, 0, 2, 0, 0, 0], 64, 256, gg.EPI_SILU_GATE, torch.bfloat16),
 ]
 
 
