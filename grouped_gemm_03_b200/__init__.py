@@ -62,6 +62,7 @@ _SIGS = {
     "moe_permute": (_i, [_vp, _i, _ip, _i, _i, _i, _i, _i, _i, _vp, _fp, _ip, _ip, _ip, _ip, _vp, _sz, _vp]),
     "moe_permute_noalloc": (_i, [_vp, _i, _ip, _i, _i, _i, _i, _i, _i, _vp, _fp, _ip, _ip, _ip, _ip, _vp]),
     "moe_grouped_gemm_workspace_size": (_sz, []),
+    "moe_grouped_gemm_plan": (ctypes.c_char_p, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "moe_grouped_gemm": (_i, [_vp, _fp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _vp, _i, _fp, _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _ip, _fp, _i, _i, _i, _i, _vp, _i, _vp]),
     "moe_selftest_workspace_size": (_sz, []),
@@ -225,6 +226,13 @@ def grouped_gemm(A, B, offsets, N: int, epilogue: int = EPI_NONE, c_dtype=torch.
 
 
 # ---------------------------------------------------------------- combine
+def grouped_gemm_plan(G: int, rows: int, N: int, K: int, ab_dtype: int = MOE_BF16, epilogue: int = EPI_NONE,
+                      c_dtype: int = MOE_BF16, extra_groups: int = 0, num_sms: int = 0) -> str:
+    """Which kernel a grouped GEMM of this shape runs on (host arithmetic only)."""
+    return lib().moe_grouped_gemm_plan(G, extra_groups, rows, N, K, ab_dtype, epilogue, c_dtype,
+                                       num_sms).decode()
+
+
 def combine(Y, token_to_row, topk_w, has_shared: bool, out_dtype=torch.bfloat16, out=None, stream=None):
     _cuda(Y, token_to_row, topk_w)
     T, k = token_to_row.shape

@@ -99,6 +99,8 @@ struct GemmArgs {
   int* status;
 };
 int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s);
+int plan_grouped_gemm(const GemmArgs& a, int sms);  // host-only choice of kernel (see gemm_variant_name)
+const char* gemm_variant_name(int variant);
 
 int launch_combine(const void* Y, const int32_t* t2r, const float* w, int has_shared, int T, int d, int k,
                    void* out, int out_dtype, cudaStream_t s);

@@ -1498,48 +1498,112 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
 
 }  // namespace
 
-int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
-  if (a.G + a.has_extra == 0 || a.rows == 0) return MOE_OK;
+// Which kernel a grouped GEMM runs on: decided on the host from shapes alone
+// (the per-group row counts live on the device).
+enum GemmVariant {
+  kEmpty = 0, kUnsupported, kInvalid,
+  kSwapGate, kSwapNone,                       // weights on the 128-row side (a few tokens per group)
+  kGate64, kGate128, kPairGate,               // SiLU gate: 64 / 128 output columns per tile, CTA pairs
+  kPairNone, kPairNoneF32,                    // no epilogue on CTA pairs (bf16 / fp32 out)
+  kNone256, kNone128, kNone64,                // single-CTA, bf16 out
+  kNone256F32, kNone128F32, kNone64F32,       // single-CTA, fp32 out (router logits, split-K)
+  kFp8GateE4M3, kFp8GateBf16, kFp8None        // E4M3 operands, per-128-K promotion
+};
+
+int plan_grouped_gemm(const GemmArgs& a, int sms) {
+  const int groups = a.G + a.has_extra;
+  if (groups == 0 || a.rows == 0) return kEmpty;
   if (a.ab_dtype == MOE_BF16) {
     // CTA pairs pay off when tiles of 256 rows are mostly full: large groups on average;
     // groups of a few tokens (decode) put the weights on the 128-row side instead
-    const bool pairs = a.pair_tiles > 0 || (a.pair_tiles == 0 && a.rows >= 512 * (a.G + a.has_extra));
-    const bool swap = a.swap_ab > 0 || (a.swap_ab == 0 && a.ksplit <= 1 && a.c_dtype == MOE_BF16 &&
-                                        a.rows < 32 * (a.G + a.has_extra));
+    const bool pairs = a.pair_tiles > 0 || (a.pair_tiles == 0 && a.rows >= 512 * groups);
+    const bool swap = a.swap_ab > 0 || (a.swap_ab == 0 && a.rows < 32 * groups);
     if (swap && a.ksplit <= 1 && a.c_dtype == MOE_BF16) {
-      if (a.epilogue == MOE_EPI_SILU_GATE && a.N % 64 == 0) return run_bf16_swap<1>(a, s);
-      if (a.epilogue == MOE_EPI_NONE && a.N % 128 == 0) return run_bf16_swap<0>(a, s);
+      if (a.epilogue == MOE_EPI_SILU_GATE && a.N % 64 == 0) return kSwapGate;
+      if (a.epilogue == MOE_EPI_NONE && a.N % 128 == 0) return kSwapNone;
     }
     if (a.epilogue == MOE_EPI_SILU_GATE) {
-      if (a.c_dtype != MOE_BF16 || a.N % 64 != 0 || a.ksplit > 1) return MOE_ERR_UNSUPPORTED;
-      // few rows (decode): 64-column output tiles (64 gate + 64 up rows of B) give
-      // twice the tiles, so the weight stream spreads over the SMs more evenly
-      const bool narrow = a.mma_n == 128 || a.N % 128 != 0 || (a.mma_n == 0 && a.rows < 64 * num_sms());
-      if (narrow) return run_bf16<128, 1, 0>(a, s);
-      return pairs ? run_bf16_pair<1, 0>(a, s) : run_bf16<256, 1, 0>(a, s);
+      if (a.c_dtype != MOE_BF16 || a.N % 64 != 0 || a.ksplit > 1) return kUnsupported;
+      // small problems: 64-column output tiles (64 gate + 64 up rows of B) give twice
+      // the tiles when 128-column tiles would not fill two waves of the SMs
+      const long long est_tiles = (static_cast<long long>(a.rows) / 128 + groups) * (a.N / 128);
+      const bool narrow =
+          a.mma_n == 128 || a.N % 128 != 0 || (a.mma_n == 0 && !pairs && est_tiles < 2ll * sms);
+      if (narrow) return kGate64;
+      return pairs ? kPairGate : kGate128;
     }
+    if (a.c_dtype != MOE_F32 && a.c_dtype != MOE_BF16) return kUnsupported;
+    const bool out = a.c_dtype == MOE_F32;
     if (pairs && a.ksplit <= 1 && a.N % 256 == 0 && (a.mma_n == 0 || a.mma_n == 256))
-      return a.c_dtype == MOE_F32 ? run_bf16_pair<0, 1>(a, s) : run_bf16_pair<0, 0>(a, s);
-    const int out = a.c_dtype == MOE_F32 ? 1 : 0;
-    if (a.c_dtype != MOE_F32 && a.c_dtype != MOE_BF16) return MOE_ERR_UNSUPPORTED;
-    if (a.ksplit > 1 && (!out || a.ksplit > a.K / 64)) return MOE_ERR_UNSUPPORTED;
+      return out ? kPairNoneF32 : kPairNone;
+    if (a.ksplit > 1 && (!out || a.ksplit > a.K / 64)) return kUnsupported;
     const int want = a.mma_n;
-    if ((want == 0 || want == 256) && a.N % 256 == 0) return out ? run_bf16<256, 0, 1>(a, s) : run_bf16<256, 0, 0>(a, s);
-    if ((want == 0 || want == 128) && a.N % 128 == 0) return out ? run_bf16<128, 0, 1>(a, s) : run_bf16<128, 0, 0>(a, s);
-    if ((want == 0 || want == 64) && a.N % 64 == 0) return out ? run_bf16<64, 0, 1>(a, s) : run_bf16<64, 0, 0>(a, s);
-    return MOE_ERR_UNSUPPORTED;
+    if ((want == 0 || want == 256) && a.N % 256 == 0) return out ? kNone256F32 : kNone256;
+    if ((want == 0 || want == 128) && a.N % 128 == 0) return out ? kNone128F32 : kNone128;
+    if ((want == 0 || want == 64) && a.N % 64 == 0) return out ? kNone64F32 : kNone64;
+    return kUnsupported;
   }
   if (a.ab_dtype == MOE_E4M3) {
-    if (a.ksplit > 1 || !a.A_scales || !a.B_scales || (a.has_extra && !a.B_extra_scales)) return MOE_ERR_UNSUPPORTED;
+    if (a.ksplit > 1) return kUnsupported;
     if (a.epilogue == MOE_EPI_SILU_GATE && a.N % 128 == 0) {
-      if (a.c_dtype == MOE_E4M3) return a.C_scales ? run_fp8<1, 2>(a, s) : MOE_ERR_INVALID;
-      if (a.c_dtype == MOE_BF16) return run_fp8<1, 0>(a, s);
-      return MOE_ERR_UNSUPPORTED;
+      if (a.c_dtype == MOE_E4M3) return kFp8GateE4M3;
+      if (a.c_dtype == MOE_BF16) return kFp8GateBf16;
+      return kUnsupported;
     }
-    if (a.epilogue == MOE_EPI_NONE && a.N % 256 == 0 && a.c_dtype == MOE_BF16) return run_fp8<0, 0>(a, s);
-    return MOE_ERR_UNSUPPORTED;
+    if (a.epilogue == MOE_EPI_NONE && a.N % 256 == 0 && a.c_dtype == MOE_BF16) return kFp8None;
+    return kUnsupported;
   }
-  return MOE_ERR_UNSUPPORTED;
+  return kUnsupported;
+}
+
+const char* gemm_variant_name(int v) {
+  switch (v) {
+    case kEmpty: return "empty";
+    case kUnsupported: return "unsupported";
+    case kInvalid: return "invalid";
+    case kSwapGate: return "bf16 swap-ab 128x32 silu-gate";
+    case kSwapNone: return "bf16 swap-ab 128x32";
+    case kGate64: return "bf16 128x128 silu-gate (64 out cols)";
+    case kGate128: return "bf16 128x256 silu-gate";
+    case kPairGate: return "bf16 cta-pair 256x256 silu-gate";
+    case kPairNone: return "bf16 cta-pair 256x256";
+    case kPairNoneF32: return "bf16 cta-pair 256x256 fp32-out";
+    case kNone256: return "bf16 128x256";
+    case kNone128: return "bf16 128x128";
+    case kNone64: return "bf16 128x64";
+    case kNone256F32: return "bf16 128x256 fp32-out";
+    case kNone128F32: return "bf16 128x128 fp32-out";
+    case kNone64F32: return "bf16 128x64 fp32-out";
+    case kFp8GateE4M3: return "e4m3 128x256 silu-gate e4m3-out";
+    case kFp8GateBf16: return "e4m3 128x256 silu-gate";
+    case kFp8None: return "e4m3 128x256";
+    default: return "unknown";
+  }
+}
+
+int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
+  if (a.ab_dtype == MOE_E4M3 && (!a.A_scales || !a.B_scales || (a.has_extra && !a.B_extra_scales)))
+    return MOE_ERR_UNSUPPORTED;
+  switch (plan_grouped_gemm(a, num_sms())) {
+    case kEmpty: return MOE_OK;
+    case kSwapGate: return run_bf16_swap<1>(a, s);
+    case kSwapNone: return run_bf16_swap<0>(a, s);
+    case kGate64: return run_bf16<128, 1, 0>(a, s);
+    case kGate128: return run_bf16<256, 1, 0>(a, s);
+    case kPairGate: return run_bf16_pair<1, 0>(a, s);
+    case kPairNone: return run_bf16_pair<0, 0>(a, s);
+    case kPairNoneF32: return run_bf16_pair<0, 1>(a, s);
+    case kNone256: return run_bf16<256, 0, 0>(a, s);
+    case kNone128: return run_bf16<128, 0, 0>(a, s);
+    case kNone64: return run_bf16<64, 0, 0>(a, s);
+    case kNone256F32: return run_bf16<256, 0, 1>(a, s);
+    case kNone128F32: return run_bf16<128, 0, 1>(a, s);
+    case kNone64F32: return run_bf16<64, 0, 1>(a, s);
+    case kFp8GateE4M3: return a.C_scales ? run_fp8<1, 2>(a, s) : MOE_ERR_INVALID;
+    case kFp8GateBf16: return run_fp8<1, 0>(a, s);
+    case kFp8None: return run_fp8<0, 0>(a, s);
+    default: return MOE_ERR_UNSUPPORTED;
+  }
 }
 
 }  // namespace moe

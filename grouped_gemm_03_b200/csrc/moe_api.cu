@@ -286,6 +286,20 @@ int moe_selftest_stalled_pipeline(void* ws, size_t ws_bytes, unsigned long long 
   return launch_grouped_gemm(g, s);
 }
 
+const char* moe_grouped_gemm_plan(int G, int extra_groups, int rows, int N, int K, int ab_dtype, int epilogue,
+                                  int c_dtype, int num_sms) {
+  GemmArgs a{};
+  a.G = G;
+  a.has_extra = extra_groups ? 1 : 0;
+  a.rows = rows;
+  a.N = N;
+  a.K = K;
+  a.ab_dtype = ab_dtype;
+  a.epilogue = epilogue;
+  a.c_dtype = c_dtype;
+  return gemm_variant_name(plan_grouped_gemm(a, num_sms > 0 ? num_sms : 148));
+}
+
 // ------------------------------------------------------------------ combine
 int moe_combine(const void* Y, const int32_t* token_to_row, const float* topk_w, int has_shared, int T, int d, int k,
                 void* out, int out_dtype, void* stream) {

@@ -189,6 +189,11 @@ int moe_permute_noalloc(const void* x, int x_dtype, const int32_t* topk_idx, int
  * (NONE); E4M3: K % 128 == 0, N % 128 == 0 (SILU_GATE, C bf16 or E4M3) or
  * N % 256 == 0 (NONE, C bf16); G <= 1024. */
 size_t moe_grouped_gemm_workspace_size(void);
+/* The kernel a grouped GEMM of this shape runs on, as a short description
+ * (host arithmetic only, no device needed; num_sms <= 0 means 148).
+ * extra_groups = 1 counts the shared expert moe_forward appends as a group. */
+const char* moe_grouped_gemm_plan(int G, int extra_groups, int rows, int N, int K, int ab_dtype, int epilogue,
+                                  int c_dtype, int num_sms);
 int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const float* B_scales,
                      const int32_t* offsets, int G, int rows, int N, int K, int ab_dtype, int epilogue,
                      void* C, int c_dtype, float* C_scales, void* ws, size_t ws_bytes, void* stream);

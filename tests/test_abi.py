@@ -98,3 +98,48 @@ def test_missing_library_fails_loudly(monkeypatch, tmp_path):
     monkeypatch.setattr(gg, "_LIB", None)
     with pytest.raises(RuntimeError, match="missing"):
         gg.lib()
+
+
+def _layer_plans(name):
+    from workload import shape_of
+    s = shape_of(name)
+    extra = 1 if s.shared_inter else 0
+    rows = s.T * s.k + (s.T if extra else 0)
+    ab = gg.MOE_E4M3 if s.fp8 else gg.MOE_BF16
+    up = gg.grouped_gemm_plan(s.E, rows, s.inter, s.d, ab, gg.EPI_SILU_GATE, ab, extra)
+    down = gg.grouped_gemm_plan(s.E, rows, s.d, s.inter, ab, gg.EPI_NONE, gg.MOE_BF16, extra)
+    return up, down
+
+
+# The kernel each benchmarked layer runs on. A heuristic change that moves a
+# workload to another kernel shows up here before it shows up as a slowdown.
+@pytest.mark.parametrize("name,up,down", [
+    ("mixtral", "bf16 cta-pair 256x256 silu-gate", "bf16 cta-pair 256x256"),
+    ("fine", "bf16 128x256 silu-gate", "bf16 128x256"),
+    ("fine_skew", "bf16 128x256 silu-gate", "bf16 128x256"),
+    ("decode", "bf16 swap-ab 128x32 silu-gate", "bf16 swap-ab 128x32"),
+    ("tiny", "bf16 128x128 silu-gate (64 out cols)", "bf16 128x256"),
+    ("fine_fp8", "e4m3 128x256 silu-gate e4m3-out", "e4m3 128x256"),
+])
+def test_grouped_gemm_plan_per_workload(L, name, up, down):
+    assert _layer_plans(name) == (up, down)
+
+
+def test_grouped_gemm_plan_edges(L):
+    P = gg.grouped_gemm_plan
+    assert P(8, 0, 256, 128) == "empty"
+    assert P(0, 1024, 256, 128) == "empty"
+    # widths the kernels do not tile
+    assert P(4, 1024, 96, 128, epilogue=gg.EPI_SILU_GATE) == "unsupported"
+    assert P(4, 4096, 100, 128) == "unsupported"
+    assert P(4, 4096, 384, 256, ab_dtype=gg.MOE_E4M3) == "unsupported"
+    # a gate width that is a multiple of 64 only takes the 64-column tiles
+    assert P(4, 100000, 192, 256, epilogue=gg.EPI_SILU_GATE) == "bf16 128x128 silu-gate (64 out cols)"
+    # few rows per group -> weights on the 128-row side; many -> CTA pairs
+    assert P(64, 64 * 31, 1024, 1024).startswith("bf16 swap-ab")
+    assert P(64, 64 * 32, 1024, 1024) == "bf16 128x256"
+    assert P(8, 8 * 512, 1024, 1024) == "bf16 cta-pair 256x256"
+    # narrow gate tiles only while 128-column tiles fill under two waves of the SMs
+    assert P(8, 8 * 256, 1024, 1024, epilogue=gg.EPI_SILU_GATE, num_sms=148) == \
+        "bf16 128x128 silu-gate (64 out cols)"
+    assert P(8, 8 * 256, 4096, 1024, epilogue=gg.EPI_SILU_GATE, num_sms=148) == "bf16 128x256 silu-gate"
