@@ -175,73 +175,6 @@ def make_cfg(gg, s):
                           gg.MOE_E4M3 if s.fp8 else gg.MOE_BF16, odt, s.renormalize)
 
 
-class Staged:
-    """The forward as its separate C-ABI calls (same kernels as moe_forward), for per-kernel timing."""
-
-    def __init__(self, gg, s, inp, dev):
-        self.gg, self.s, self.inp = gg, s, inp
-        T, k, E, d, I = s.T, s.k, s.E, s.d, s.inter
-        shared = bool(s.shared_inter)
-        R = T * k + (T if shared else 0)
-        self.rows = R
-        self.idx = torch.empty((T, k), dtype=torch.int32, device=dev)
-        self.w = torch.empty((T, k), dtype=torch.float32, device=dev)
-        self.rws = torch.empty(gg.lib().moe_router_workspace_size(T, E), dtype=torch.uint8, device=dev)
-        self.pws = torch.empty(gg.lib().moe_permute_workspace_size(T, E), dtype=torch.uint8, device=dev)
-        self.gws = torch.empty(256, dtype=torch.uint8, device=dev)
-        self.xp = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
-        self.counts = torch.empty(E, dtype=torch.int32, device=dev)
-        self.offsets = torch.empty(E + 2, dtype=torch.int32, device=dev)
-        self.r2t = torch.empty(R, dtype=torch.int32, device=dev)
-        self.t2r = torch.empty((T, k), dtype=torch.int32, device=dev)
-        self.h = torch.empty((R, I), dtype=torch.bfloat16, device=dev)
-        self.y = torch.empty((R, d), dtype=torch.bfloat16, device=dev)
-        self.out = torch.empty((T, d), dtype=torch.bfloat16, device=dev)
-        self.shared = shared
-
-    def stages(self):
-        gg, s, inp = self.gg, self.s, self.inp
-        L = gg.lib()
-        P = gg._ptr
-        st = gg._stream()
-        T, k, E, d, I = s.T, s.k, s.E, s.d, s.inter
-        x = inp["x"]
-        xdt = gg._dt(x)
-
-        def router():
-            gg._check(L.moe_router_topk(P(x), xdt, P(inp["W_r"]), gg._dt(inp["W_r"]), P(inp["bias"]), T, d, E, k,
-                                        int(s.renormalize), None, P(self.idx), P(self.w), P(self.rws),
-                                        self.rws.numel(), st), "router")
-
-        def permute():
-            gg._check(L.moe_permute(P(x), xdt, P(self.idx), T, d, E, k, int(self.shared), gg.MOE_BF16, P(self.xp),
-                                    None, P(self.counts), P(self.offsets), P(self.r2t), P(self.t2r), P(self.pws),
-                                    self.pws.numel(), st), "permute")
-
-        def up():
-            gg._check(self._gemm(L, P(self.xp), inp["W1"], inp["W1s"], I, d, gg.EPI_SILU_GATE, P(self.h), st), "up")
-
-        def down():
-            gg._check(self._gemm(L, P(self.h), inp["W2"], inp["W2s"], d, I, gg.EPI_NONE, P(self.y), st), "down")
-
-        def combine():
-            gg._check(L.moe_combine(P(self.y), P(self.t2r), P(self.w), int(self.shared), T, d, k, P(self.out),
-                                    gg.MOE_BF16, st), "combine")
-
-        return [("router", router), ("permute", permute), ("up_gemm", up), ("down_gemm", down),
-                ("combine", combine)]
-
-    def _gemm(self, L, A, B, Bx, N, K, epi, C, st):
-        # the routed experts and, when present, the shared expert: two launches of the standalone entry
-        # point would differ from moe_forward's single launch, so time the fused one through the forward's
-        # own path when a shared expert exists (the staged breakdown is exact only without one)
-        gg = self.gg
-        P = gg._ptr
-        E = self.s.E
-        return L.moe_grouped_gemm(A, None, P(B), None, P(self.offsets), E, self.rows, N, K, gg.MOE_BF16, epi, C,
-                                  gg.MOE_BF16, None, P(self.gws), self.gws.numel(), st)
-
-
 HOLD_CYCLES = 2_000_000  # ~1 ms spin queued ahead of each timed step
 
 
@@ -264,44 +197,52 @@ def time_steps(fn, steps, warmup, flush, stream, hold=True):
     return [a.elapsed_time(b) for a, b in ev]
 
 
-def time_staged(staged, steps, flush, stream):
-    st = staged.stages()
+STAGES = ("router", "permute", "up_gemm", "down_gemm", "combine")
+
+
+def time_marked(gg, cfg, inp, weights, out, counts, ws, steps, flush, stream):
+    """Per-kernel device time inside whole forwards: moe_forward_marked records an
+    event before each of the layer's five kernels and one after the last."""
+    def run(evs):
+        gg.moe_forward_marked(cfg, inp["x"], inp["W_r"], inp["bias"], weights, evs, out, counts_out=counts, ws=ws)
+
     for _ in range(2):
-        for _, f in st:
-            f()
+        run([torch.cuda.Event(enable_timing=True) for _ in range(6)])
     torch.cuda.synchronize()
-    per = {n: [] for n, _ in st}
+    per = {n: [] for n in STAGES}
     for _ in range(steps):
         flush()
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+        for e in evs:  # create the CUDA events before the hold so the timed launches are not delayed
+            e.record(stream)
         torch.cuda._sleep(HOLD_CYCLES)
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(len(st) + 1)]
-        evs[0].record(stream)
-        for i, (_, f) in enumerate(st):
-            f()
-            evs[i + 1].record(stream)
+        run(evs)
         torch.cuda.synchronize()
-        for i, (n, _) in enumerate(st):
+        for i, n in enumerate(STAGES):
             per[n].append(evs[i].elapsed_time(evs[i + 1]))
     return {n: float(np.mean(v)) for n, v in per.items()}
 
 
-def traffic_from_profile(kernel_src_hash):
-    """DRAM bytes per launch of the up GEMM from the committed ncu summary, if it matches this source."""
-    p = os.path.join(ROOT, "profiles", "up_gemm_traffic.json")
-    if not os.path.exists(p):
-        return None
+def traffic_from_profile(workload, stage, kernel_src_hash):
+    """DRAM bytes per launch of `stage` on `workload` from the committed ncu summary, if it
+    was taken on the kernel sources as they are now."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
     try:
-        d = json.load(open(p))
-    except Exception:
+        d = json.load(open(p)).get(workload, {}).get(stage)
+    except (OSError, ValueError):
         return None
-    if d.get("source_sha256") != kernel_src_hash:
+    if not d or d.get("source_sha256") != kernel_src_hash:
         return None
-    return d.get("bytes_per_launch_full")
+    return d.get("bytes_per_launch")
 
 
-def kernel_source_hash():
+STAGE_SOURCES = {"router": "router.cu", "permute": "permute.cu", "up_gemm": "grouped_gemm.cu",
+                 "down_gemm": "grouped_gemm.cu", "combine": "combine.cu"}
+
+
+def kernel_source_hash(stage):
     h = hashlib.sha256()
-    for f in ("grouped_gemm.cu", "ptx.cuh", "common.cuh"):
+    for f in (STAGE_SOURCES[stage], "ptx.cuh", "common.cuh"):
         h.update(open(os.path.join(ROOT, "grouped_gemm_03_b200", "csrc", f), "rb").read())
     return h.hexdigest()
 
@@ -325,6 +266,33 @@ def algorithmic(s, counts=None):
                       "bytes": (active + sh) * d * I * eb + Rp * I * eb + Rp * d * 2},
         "combine": {"bytes": Rp * d * 2 + T * d * ob + T * k * 8},
     }
+
+
+STAGE_NAMES = {"router": "router GEMM + softmax + top-k", "permute": "histogram / scan / scatter",
+               "up_gemm": "up-projection grouped GEMM (SiLU gate)", "down_gemm": "down-projection grouped GEMM",
+               "combine": "combine (gather, weight, sum + shared)"}
+
+
+def roofline(s, alg, kernels, peaks, peak_kind):
+    """The roofline entry of the kernel with the largest share of the step.  A GEMM
+    whose algorithmic FLOP per byte is below the ridge point (tensor peak / HBM peak)
+    is bound by HBM (the expert weights), otherwise by the tensor pipe."""
+    if not kernels:
+        return None
+    stage = max(kernels, key=lambda n: kernels[n]["us"])
+    t = kernels[stage]["us"] * 1e-6
+    a = alg[stage]
+    hbm = float(peaks["hbm_gbs"])
+    tensor = float(peaks["bf16_tflops"]) * (2.0 if s.fp8 else 1.0)
+    tensor_kind = "bf16 burst (cuBLAS 8192^3)" + (" x 2, the nominal e4m3 / bf16 dense ratio" if s.fp8 else "")
+    if "flops" in a and a["flops"] / a["bytes"] >= tensor * 1e12 / (hbm * 1e9):
+        achieved, peak, unit, bound, kind = a["flops"] / t / 1e12, tensor, "TFLOP/s", "tensor", tensor_kind
+    else:
+        achieved, peak, unit, bound, kind = a["bytes"] / t / 1e9, hbm, "GB/s", "hbm", "HBM copy bandwidth"
+    return {"bound": bound, "achieved": round(achieved, 1), "peak": peak, "unit": unit,
+            "frac": round(achieved / peak, 4),
+            "traffic": traffic_from_profile(s.name, stage, kernel_source_hash(stage)),
+            "kernel": STAGE_NAMES[stage], "algorithmic": a, "peak_kind": f"{peak_kind} {kind}"}
 
 
 class HostExperts:
@@ -426,20 +394,17 @@ def run_ours(args, rank, world, dev):
     e2e_times = time_steps(step_host, max(3, args.steps // 2), 2, flush, stream, hold=False)
     e2e_ms = max_over_ranks(float(np.mean(e2e_times)), world, dev)
 
-    # --- per-kernel breakdown (staged calls of the same kernels)
+    # --- per-kernel breakdown: the same forward with an event between its kernels
+    kt = time_marked(gg, cfg, inp, weights, out, counts, ws, max(3, args.steps // 2), flush, stream)
+    alg = algorithmic(s, counts.cpu().numpy())
     kern = {}
-    if not s.shared_inter and not s.fp8:
-        staged = Staged(gg, s, inp, dev)
-        kt = time_staged(staged, max(3, args.steps // 2), flush, stream)
-        alg = algorithmic(s, counts.cpu().numpy())
-        peaks, _ = load_peaks()
-        for name, t_ms in kt.items():
-            a = alg[name]
-            e = {"us": round(t_ms * 1e3, 2)}
-            if "flops" in a:
-                e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
-            e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
-            kern[name] = e
+    for name, t_ms in kt.items():
+        a = alg[name]
+        e = {"us": round(t_ms * 1e3, 2)}
+        if "flops" in a:
+            e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
+        e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
+        kern[name] = e
     return dict(ms=ms, e2e_ms=e2e_ms, kernels=kern, clocks=clk.summary(), inp=inp, s=s, counts=counts.cpu().numpy(),
                 out_dtype=out.dtype)
 
@@ -489,16 +454,11 @@ def main():
         T = s.T
         value = job_tokens_per_s(T, world, r["ms"])
         alg = algorithmic(s, r["counts"])
-        up = r["kernels"].get("up_gemm")
-        roof = None
-        if up:
-            achieved = alg["up_gemm"]["flops"] / (up["us"] * 1e-6) / 1e12
-            peak = float(peaks["bf16_tflops"])
-            roof = {"bound": "tensor", "achieved": round(achieved, 1), "peak": peak, "unit": "TFLOP/s",
-                    "frac": round(achieved / peak, 4), "traffic": traffic_from_profile(kernel_source_hash()),
-                    "kernel": "up-projection grouped GEMM (SiLU gate)",
-                    "peak_kind": f"{peak_kind} bf16 burst (cuBLAS 8192^3)"}
+        roof = roofline(s, alg, r["kernels"], peaks, peak_kind)
         gemm_flops = s.gemm_flops()
+        gemm_us = r["kernels"]["up_gemm"]["us"] + r["kernels"]["down_gemm"]["us"]
+        gemm_tf = gemm_flops / (gemm_us * 1e-6) / 1e12
+        tensor_peak = float(peaks["bf16_tflops"]) * (2.0 if s.fp8 else 1.0)
         result = {
             "metric": METRIC,
             "value": round(value, 1),
@@ -513,8 +473,9 @@ def main():
             "dtype": "e4m3" if s.fp8 else "bf16",
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
             "config": config_block(s),
-            "gemm_tflops": round(gemm_flops / (r["ms"] * 1e-3) / 1e12, 1),
-            "gemm_frac_of_peak": round(gemm_flops / (r["ms"] * 1e-3) / 1e12 / float(peaks["bf16_tflops"]), 4),
+            # grouped-GEMM FLOP over the two GEMM kernels' own time, against the dense tensor peak
+            "gemm_tflops": round(gemm_tf, 1),
+            "gemm_frac_of_peak": round(gemm_tf / tensor_peak, 4),
             "roofline": roof,
             "kernels": r["kernels"],
             "e2e": {"value": round(job_tokens_per_s(T, world, r["e2e_ms"]), 1), "unit": "tokens/s",

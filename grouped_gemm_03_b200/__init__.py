@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "LIB_PATH", "MoEError", "MoEConfig", "lib", "exported_symbols", "status_string", "device_info",
     "router_topk", "topk_logits", "permute", "grouped_gemm", "combine", "quantize_weights_fp8",
-    "workspace_size", "moe_forward", "moe_forward_host", "host_staging_size", "read_device_status",
+    "workspace_size", "moe_forward", "moe_forward_marked", "moe_forward_host", "host_staging_size", "read_device_status",
     "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "EPI_NONE", "EPI_SILU_GATE",
 ]
 
@@ -70,6 +70,8 @@ _SIGS = {
     "moe_quantize_weights_fp8": (_i, [_vp, _i, _i, _i, _vp, _fp, _vp]),
     "moe_workspace_size": (_sz, [_CFG]),
     "moe_forward": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _ip, _vp, _sz, _vp]),
+    "moe_forward_marked": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _ip, _vp, _sz,
+                                ctypes.POINTER(ctypes.c_void_p), _vp]),
     "moe_host_staging_size": (_sz, [_CFG]),
     "moe_forward_host": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _vp, _sz, _vp]),
 }
@@ -299,6 +301,28 @@ def moe_forward(cfg: MoEConfig, x, W_r, bias, w: ExpertWeights, out=None, counts
                              _ptr(w.W2s_scales), _ptr(o), _ptr(counts_out), _ptr(ws), ws.numel(), _stream(stream)),
            "moe_forward")
     return o
+
+
+def moe_forward_marked(cfg: MoEConfig, x, W_r, bias, w: ExpertWeights, events, out, counts_out=None, ws=None,
+                       stream=None):
+    """moe_forward that records the six torch.cuda.Event objects in `events` around its five kernels
+    (router, permute, up GEMM, down GEMM, combine) for per-kernel timing inside the whole layer."""
+    _cuda(x, W_r, bias, w.W1, w.W2, w.W1s, w.W2s)
+    if len(events) != 6:
+        raise ValueError("six events: before each of the five stages and after the last")
+    st = torch.cuda.current_stream() if stream is None else stream
+    for e in events:
+        if not e.cuda_event:  # torch creates the CUDA event on its first record
+            e.record(st)
+    handles = (ctypes.c_void_p * 6)(*[e.cuda_event for e in events])
+    if ws is None:
+        ws = _scratch(workspace_size(cfg), x.device)
+    _check(lib().moe_forward_marked(ctypes.byref(cfg), _ptr(x), _ptr(W_r), _ptr(bias), _ptr(w.W1),
+                                    _ptr(w.W1_scales), _ptr(w.W2), _ptr(w.W2_scales), _ptr(w.W1s),
+                                    _ptr(w.W1s_scales), _ptr(w.W2s), _ptr(w.W2s_scales), _ptr(out),
+                                    _ptr(counts_out), _ptr(ws), ws.numel(), handles, _stream(st)),
+           "moe_forward_marked")
+    return out
 
 
 def moe_forward_host(cfg: MoEConfig, x_host, W_r, bias, w: ExpertWeights, out_host, ws, stream=None):

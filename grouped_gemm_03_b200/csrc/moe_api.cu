@@ -326,10 +326,14 @@ size_t moe_workspace_size(const moe_config* cfg) {
   return fwd_layout(*cfg).total;
 }
 
-int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const float* router_bias, const void* W1,
-                const float* W1_scales, const void* W2, const float* W2_scales, const void* W1_shared,
-                const float* W1s_scales, const void* W2_shared, const float* W2s_scales, void* out,
-                int32_t* counts_out, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+
+// The layer's five stages; `marks` (or NULL) gets one event recorded before
+// each stage and one after the last.
+int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const float* router_bias, const void* W1,
+                 const float* W1_scales, const void* W2, const float* W2_scales, const void* W1_shared,
+                 const float* W1s_scales, const void* W2_shared, const float* W2s_scales, void* out,
+                 int32_t* counts_out, void* ws, size_t ws_bytes, void* stream, void* const* marks) {
   int st = check_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config c = *cfg;
@@ -359,10 +363,16 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   }
   const int T = c.T, d = c.d, E = c.E, k = c.k, I = c.inter;
   const int Rp = T * k + (shared ? T : 0);
+  auto mark = [&](int i) -> int {
+    if (marks) MOE_CUDA_CHECK(cudaEventRecord(static_cast<cudaEvent_t>(marks[i]), s));
+    return MOE_OK;
+  };
 
+  if ((st = mark(0)) != MOE_OK) return st;
   st = launch_router(x, c.x_dtype, W_r, c.router_dtype, router_bias, T, d, E, k, c.renormalize, nullptr, idx, w,
                      reinterpret_cast<float*>(base + L.logits), status, s);
   if (st != MOE_OK) return st;
+  if ((st = mark(1)) != MOE_OK) return st;
 
   PermuteArgs pa;
   pa.x = x;
@@ -384,6 +394,7 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   pa.status = status;
   st = launch_permute(pa, s);
   if (st != MOE_OK) return st;
+  if ((st = mark(2)) != MOE_OK) return st;
 
   GemmArgs up{};
   up.A = base + L.xp;
@@ -408,6 +419,7 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   }
   st = launch_grouped_gemm(up, s);
   if (st != MOE_OK) return st;
+  if ((st = mark(3)) != MOE_OK) return st;
 
   GemmArgs dn{};
   dn.A = base + L.h;
@@ -431,11 +443,35 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
   }
   st = launch_grouped_gemm(dn, s);
   if (st != MOE_OK) return st;
+  if ((st = mark(4)) != MOE_OK) return st;
 
   st = launch_combine(base + L.y, t2r, w, shared ? 1 : 0, T, d, k, out, c.out_dtype, s);
   if (st != MOE_OK) return st;
+  if ((st = mark(5)) != MOE_OK) return st;
   if (counts_out) MOE_CUDA_CHECK(cudaMemcpyAsync(counts_out, counts, sizeof(int32_t) * E, cudaMemcpyDeviceToDevice, s));
   return MOE_OK;
+}
+
+}  // namespace
+
+int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const float* router_bias, const void* W1,
+                const float* W1_scales, const void* W2, const float* W2_scales, const void* W1_shared,
+                const float* W1s_scales, const void* W2_shared, const float* W2s_scales, void* out,
+                int32_t* counts_out, void* ws, size_t ws_bytes, void* stream) {
+  return forward_impl(cfg, x, W_r, router_bias, W1, W1_scales, W2, W2_scales, W1_shared, W1s_scales, W2_shared,
+                      W2s_scales, out, counts_out, ws, ws_bytes, stream, nullptr);
+}
+
+int moe_forward_marked(const moe_config* cfg, const void* x, const void* W_r, const float* router_bias,
+                       const void* W1, const float* W1_scales, const void* W2, const float* W2_scales,
+                       const void* W1_shared, const float* W1s_scales, const void* W2_shared,
+                       const float* W2s_scales, void* out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                       void* const* stage_events, void* stream) {
+  if (!stage_events) return MOE_ERR_INVALID;
+  for (int i = 0; i < 6; ++i)
+    if (!stage_events[i]) return MOE_ERR_INVALID;
+  return forward_impl(cfg, x, W_r, router_bias, W1, W1_scales, W2, W2_scales, W1_shared, W1s_scales, W2_shared,
+                      W2s_scales, out, counts_out, ws, ws_bytes, stream, stage_events);
 }
 
 size_t moe_host_staging_size(const moe_config* cfg) {

@@ -249,6 +249,18 @@ int moe_forward(const moe_config* cfg, const void* x, const void* W_r, const flo
                 const float* W2s_scales, void* out, int32_t* counts_out, void* ws, size_t ws_bytes,
                 void* stream);
 
+/* As moe_forward, and also records stage_events[0..5] (cudaEvent_t handles
+ * the caller created) on `stream`: [0] before the router, [1] before the
+ * permute, [2] before the up GEMM, [3] before the down GEMM, [4] before the
+ * combine and [5] after it, so that the caller can time each kernel of the
+ * layer as it runs inside the whole forward.  A NULL array or handle is
+ * MOE_ERR_INVALID; with T == 0 no event is recorded. */
+int moe_forward_marked(const moe_config* cfg, const void* x, const void* W_r, const float* router_bias,
+                       const void* W1, const float* W1_scales, const void* W2, const float* W2_scales,
+                       const void* W1_shared, const float* W1s_scales, const void* W2_shared,
+                       const float* W2s_scales, void* out, int32_t* counts_out, void* ws, size_t ws_bytes,
+                       void* const* stage_events, void* stream);
+
 /* As moe_forward, but x_host and out_host are HOST buffers (page-locked for
  * the copies to overlap): x is copied into the workspace, the layer runs,
  * and out is copied back, all on `stream`.  The call returns without

@@ -91,6 +91,10 @@ def test_host_validation_rejects_bad_arguments(L):
     assert L.moe_forward(ctypes.byref(cfg), *args, fake, 1024, null) == -3
     cfg2 = gg.make_config(T=256, d=256, E=8, k=2, inter=512, shared_inter=256)
     assert L.moe_forward(ctypes.byref(cfg2), *args, fake, 1 << 30, null) == -2
+    # marked forward: the six event handles are required
+    assert L.moe_forward_marked(ctypes.byref(cfg), *args, fake, 1 << 30, null, null) == -1
+    events = (ctypes.c_void_p * 6)(*([0x20000] * 5 + [0]))
+    assert L.moe_forward_marked(ctypes.byref(cfg), *args, fake, 1 << 30, events, null) == -1
 
 
 def test_missing_library_fails_loudly(monkeypatch, tmp_path):

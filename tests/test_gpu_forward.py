@@ -148,6 +148,21 @@ def test_host_buffer_entry_matches_device_entry():
     assert torch.equal(oh, dev_out.cpu())
 
 
+def test_marked_entry_matches_and_orders_its_events():
+    s = shape_of("tiny", T=384, shared_inter=512, x_dtype="bf16", router_dtype="bf16")
+    inp = make_inputs(s, seed=9, device=DEV)
+    cfg = _cfg(s)
+    ws = torch.empty(gg.workspace_size(cfg), dtype=torch.uint8, device=DEV)
+    ref = gg.moe_forward(cfg, inp["x"], inp["W_r"], inp["bias"], _weights(inp), ws=ws).clone()
+    out = torch.empty_like(ref)
+    evs = [torch.cuda.Event(enable_timing=True) for _ in range(6)]
+    gg.moe_forward_marked(cfg, inp["x"], inp["W_r"], inp["bias"], _weights(inp), evs, out, ws=ws)
+    torch.cuda.synchronize()
+    assert torch.equal(out, ref)
+    gaps = [evs[i].elapsed_time(evs[i + 1]) for i in range(5)]
+    assert all(g >= 0 for g in gaps) and sum(gaps) > 0
+
+
 def test_empty_batch():
     s = shape_of("tiny", T=0, x_dtype="bf16", router_dtype="bf16")
     cfg = _cfg(s)
