@@ -943,12 +943,34 @@ __global__ void __launch_bounds__(kThreads, 1)
 // mbarrier.
 constexpr int kThreadsF8 = 576;  // producer, MMA issuer, 16 epilogue warps
 
+// Shared memory of the FP8 kernel, as offsets from the 1024-byte aligned base.
+// Without the gate, each epilogue warp stages its 32 output rows (32 x 128 B
+// of bf16) for one bulk tensor store, which takes the room of one operand
+// stage; the gated kernels store their narrower rows directly.
+template <int EPI, int OUT>
+struct F8Smem {
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = 256 * 128;
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static constexpr bool STAGE_OUT = EPI == 0;
+  static constexpr int OUT_WARP = STAGE_OUT ? 4096 : 0;
+  static constexpr int STAGES = STAGE_OUT ? 3 : 4;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int OUTB = STAGES * STAGE_BYTES;              // output staging
+  static constexpr int BARS = OUTB + 16 * OUT_WARP;              // barriers and flags
+  static constexpr int TABLES = BARS + 512;                      // group offsets and tile prefix
+  static constexpr int AMAX = TABLES + 2 * (kMaxGroups + 2) * 4;  // [2 parity][4 quarters][128 rows]
+  static constexpr int SMEM = AMAX + 2 * 4 * 128 * 4 + 1024;     // + alignment slack
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
 template <int EPI, int OUT>  // EPI 1: SiLU gate (OUT 0 bf16 / 2 e4m3); EPI 0: OUT 0 bf16
 __global__ void __launch_bounds__(kThreadsF8, 1)
     gg_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                  const __grid_constant__ CUtensorMap tmBx, const Params p) {
+                  const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC,
+                  const Params p) {
   constexpr int MMA_N = 256;
-  using L = Tile<MMA_N>;
+  using L = F8Smem<EPI, OUT>;
   constexpr int OUT_COLS = EPI ? 128 : 256;
   constexpr uint32_t IDESC = ptx::make_idesc(BM, MMA_N, 0);
 
@@ -956,7 +978,7 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sA = smem;
   uint8_t* sB = smem + L::STAGES * L::A_BYTES;
-  uint64_t* full = reinterpret_cast<uint64_t*>(sB + L::STAGES * L::B_BYTES);
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
   uint64_t* empty = full + L::STAGES;
   uint64_t* pfull = empty + L::STAGES;
   uint64_t* pempty = pfull + 2;
@@ -965,9 +987,9 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
-  int* s_off = reinterpret_cast<int*>(smem + L::STAGES * L::STAGE_BYTES + 512);
+  int* s_off = reinterpret_cast<int*>(smem + L::TABLES);
   int* s_tile = s_off + kMaxGroups + 2;
-  float* s_amax = reinterpret_cast<float*>(s_tile + kMaxGroups + 2);  // [2 parity][4 quarters][128 rows]
+  float* s_amax = reinterpret_cast<float*>(smem + L::AMAX);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = p.G_total;
@@ -1014,9 +1036,9 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
     }
     for (int a = 0; a < 2; ++a) {
       ptx::mbar_init(&pfull[a], 1);
-      ptx::mbar_init(&pempty[a], 512);
+      ptx::mbar_init(&pempty[a], 16);  // one arrival per epilogue warp
     }
-    ptx::mbar_init(xchg, 512);
+    ptx::mbar_init(xchg, 16);
     ptx::mbar_init(drain, 1);
     ptx::fence_mbar_init();
     ptx::prefetch_tmap(&tmA);
@@ -1071,15 +1093,15 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
         *abort_flag = 1;
         set_status(p.status, MOE_ERR_TIMEOUT);
         const uint32_t pending = issued < static_cast<uint32_t>(L::STAGES) ? issued : L::STAGES;
-        uint32_t s = stage, ph = phase;
+        uint32_t s2 = stage, ph = phase;
         for (uint32_t i = 0; i < pending; ++i) {
-          if (s == 0) {
-            s = L::STAGES - 1;
+          if (s2 == 0) {
+            s2 = L::STAGES - 1;
             ph ^= 1;
           } else {
-            --s;
+            --s2;
           }
-          ptx::mbar_wait(&full[s], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+          ptx::mbar_wait(&full[s2], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
         }
       }
     }
@@ -1138,43 +1160,34 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
       const int r_in = tc.mb * BM + row_t;
       const bool valid = r_in < tc.m_g;
       const size_t grow = static_cast<size_t>(s_off[g] + r_in);
-      const bool extra = g >= p.G_main;
-      const float* bsc = extra ? p.Bx_scales : p.B_scales + static_cast<size_t>(g) * ((EPI ? 2 : 1) * p.N / 128) * nbk;
-      // weight-block rows of the two column pieces
-      const int nblk_lo = EPI ? nb : 2 * nb + (cq >> 1);
-      const int nblk_hi = EPI ? p.N / 128 + nb : 2 * nb + (cq >> 1);
-      const float* sb_lo = bsc + static_cast<size_t>(nblk_lo) * nbk;
-      const float* sb_hi = bsc + static_cast<size_t>(nblk_hi) * nbk;
-      const float* sa_row = p.A_scales + grow;
-      float acc[64];
+      // weight-block scales of the thread's two column pieces: (gate, up) blocks, or one block of 128 columns
+      const float* bsc = g >= p.G_main ? p.Bx_scales
+                                       : p.B_scales + static_cast<size_t>(g) * ((EPI ? 2 : 1) * p.N / 128) * nbk;
+      const float* sb_lo_p = bsc + static_cast<size_t>(EPI ? nb : 2 * nb + (cq >> 1)) * nbk;
+      const float* sb_hi_p = bsc + static_cast<size_t>(EPI ? p.N / 128 + nb : 2 * nb + (cq >> 1)) * nbk;
+      // fp32 accumulators as pairs for the packed FMA: acc[i] holds columns 2i, 2i+1 of the thread's 64
+      float2 acc[32];
 #pragma unroll
-      for (int i = 0; i < 64; ++i) acc[i] = 0.f;
+      for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.f, 0.f);
       // Scales are fetched ahead of use so that no K block waits on a global
-      // load: this row's sa[kb] runs through a 2-deep register queue; the
-      // tile's weight-block scales sb[kb] are spread over the lanes in
-      // windows of 32 K blocks (lane j holds block w + j) and broadcast with
-      // a shuffle, the next window being loaded halfway through the current.
+      // load: the row's sa[kb] through a 2-deep register queue, the two
+      // weight-block scales one K block ahead (the same address in every lane).
+      const float* sa_p = p.A_scales + grow;
       const size_t rstride = static_cast<size_t>(p.rows);
-      float sa0 = (valid && 0 < nbk) ? __ldg(sa_row) : 0.f;
-      float sa1 = (valid && 1 < nbk) ? __ldg(sa_row + rstride) : 0.f;
-      float wl = lane < nbk ? __ldg(sb_lo + lane) : 0.f;
-      float wh = lane < nbk ? __ldg(sb_hi + lane) : 0.f;
-      float nwl = 0.f, nwh = 0.f;
+      float sa0 = valid ? __ldg(sa_p) : 0.f;
+      float sa1 = (valid && 1 < nbk) ? __ldg(sa_p + rstride) : 0.f;
+      sa_p += 2 * rstride;
+      float sbl = __ldg(sb_lo_p), sbh = __ldg(sb_hi_p);
       for (int kb = 0; kb < nbk; ++kb) {
-        if ((kb & 31) == 0 && kb > 0) {
-          wl = nwl;
-          wh = nwh;
-        }
-        if ((kb & 31) == 16) {
-          const int kw = (kb & ~31) + 32 + lane;
-          nwl = kw < nbk ? __ldg(sb_lo + kw) : 0.f;
-          nwh = kw < nbk ? __ldg(sb_hi + kw) : 0.f;
-        }
-        const float sa = sa0;
+        const float m_lo = sa0 * sbl;
+        const float m_hi = sa0 * sbh;
         sa0 = sa1;
-        sa1 = (valid && kb + 2 < nbk) ? __ldg(sa_row + static_cast<size_t>(kb + 2) * rstride) : 0.f;
-        const float m_lo = sa * __shfl_sync(0xffffffffu, wl, kb & 31);
-        const float m_hi = sa * __shfl_sync(0xffffffffu, wh, kb & 31);
+        sa1 = (valid && kb + 2 < nbk) ? __ldg(sa_p) : 0.f;
+        sa_p += rstride;
+        if (kb + 1 < nbk) {
+          sbl = __ldg(sb_lo_p + kb + 1);
+          sbh = __ldg(sb_hi_p + kb + 1);
+        }
         if (!ptx::mbar_wait_warp(&pfull[pb], puse & 1, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;
@@ -1187,77 +1200,117 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
           ptx::tmem_ld_32x32b_x8(t0 + (j < 4 ? c_lo : c_hi) + (j & 3) * 8, v);
           ptx::tmem_ld_wait();
           const float m = j < 4 ? m_lo : m_hi;
+          const float2 m2 = make_float2(m, m);
 #pragma unroll
-          for (int i = 0; i < 8; ++i) acc[8 * j + i] = fmaf(__uint_as_float(v[i]), m, acc[8 * j + i]);
+          for (int i = 0; i < 4; ++i)
+            acc[4 * j + i] =
+                __ffma2_rn(make_float2(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1])), m2, acc[4 * j + i]);
         }
         ptx::tc_fence_before();
-        ptx::mbar_arrive(&pempty[pb]);
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&pempty[pb]);
         pb ^= 1;
         if (pb == 0) ++puse;
       }
       if (!ok) break;
+      // Output.  A warp whose 32 rows all belong to the group stages them in
+      // its shared-memory buffer and writes them with one bulk tensor store
+      // (full 128-byte lines); a slice that crosses the group's end stores
+      // its valid rows one by one, so the next group's rows are never touched.
+      const int r0 = tc.mb * BM + q * 32;
+      const bool slice_full = L::STAGE_OUT && r0 + 32 <= tc.m_g;
+      uint8_t* s_out = smem + L::OUTB + (warp - 2) * L::OUT_WARP;
+      if (slice_full) {
+        if (lane == 0) ptx::bulk_wait_read_all();  // the previous tile's store has read the buffer
+        __syncwarp();
+      }
       if constexpr (EPI == 1) {
+        // columns 0..31 of the thread are gate, 32..63 the matching up columns;
+        // h = silu(gate) * up replaces the gate half in place
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-          const float gt = acc[i];
-          acc[i] = gt / (1.0f + __expf(-gt)) * acc[32 + i];
+        for (int i = 0; i < 16; ++i) {
+          const float2 gt = acc[i], up = acc[16 + i];
+          acc[i].x = gt.x / (1.0f + __expf(-gt.x)) * up.x;
+          acc[i].y = gt.y / (1.0f + __expf(-gt.y)) * up.y;
         }
+
         if constexpr (OUT == 2) {
           float amax = 0.f;
 #pragma unroll
-          for (int i = 0; i < 32; ++i) amax = fmaxf(amax, fabsf(acc[i]));
+          for (int i = 0; i < 16; ++i) amax = fmaxf(amax, fmaxf(fabsf(acc[i].x), fabsf(acc[i].y)));
           float* xa = s_amax + (it & 1) * 512;
           xa[cq * 128 + row_t] = amax;
-          ptx::mbar_arrive(xchg);
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(xchg);
           if (!ptx::mbar_wait_warp(xchg, it & 1, abort_flag, kWaitLimitNs)) {
             ok = false;
             break;
           }
           amax = fmaxf(fmaxf(xa[row_t], xa[128 + row_t]), fmaxf(xa[256 + row_t], xa[384 + row_t]));
           const float sc = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
-          if (valid) {
-            uint32_t qw[8];
+          uint32_t qw[8];
 #pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(acc[4 * i], sc), __fdiv_rn(acc[4 * i + 1], sc));
-              const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(acc[4 * i + 2], sc), __fdiv_rn(acc[4 * i + 3], sc));
-              qw[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
-            }
+          for (int i = 0; i < 8; ++i) {
+            const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(acc[2 * i].x, sc), __fdiv_rn(acc[2 * i].y, sc));
+            const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(acc[2 * i + 1].x, sc), __fdiv_rn(acc[2 * i + 1].y, sc));
+            qw[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+          }
+          if (valid && cq == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
+          if (slice_full) {  // 32 rows x 32 B, row-major
+            uint4* d = reinterpret_cast<uint4*>(s_out + lane * 32);
+            d[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
+            d[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
+          } else if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.C) + grow * p.N + nb * 128 + cq * 32);
             dst[0] = make_uint4(qw[0], qw[1], qw[2], qw[3]);
             dst[1] = make_uint4(qw[4], qw[5], qw[6], qw[7]);
-            if (cq == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
           }
         } else {
-          if (valid) {
-            uint32_t pk[16];
+          uint32_t pk[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const __nv_bfloat162 hb = __floats2bfloat162_rn(acc[2 * i], acc[2 * i + 1]);
-              pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
-            }
-            uint4* dst =
-                reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 128 + cq * 32);
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(acc[i].x, acc[i].y);
+            pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
+          }
+          uint4* dst = slice_full ? reinterpret_cast<uint4*>(s_out + lane * 64)  // 32 rows x 64 B, row-major
+                                  : reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N +
+                                                             nb * 128 + cq * 32);
+          if (slice_full || valid) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
           }
         }
       } else {
-        if (valid) {
+        uint32_t pk[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+          const __nv_bfloat162 hb = __floats2bfloat162_rn(acc[i].x, acc[i].y);
+          pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
+        }
+        if (slice_full) {
+          // 32 rows x 128 B in the 128-byte swizzled layout of the store map:
+          // 16-byte chunk c of row r sits at chunk c ^ (r % 8)
+#pragma unroll
+          for (int c = 0; c < 8; ++c)
+            *reinterpret_cast<uint4*>(s_out + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        } else if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 256 + cq * 64);
 #pragma unroll
-          for (int v = 0; v < 8; ++v) {
-            uint32_t pk[4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              const __nv_bfloat162 hb = __floats2bfloat162_rn(acc[8 * v + 2 * i], acc[8 * v + 2 * i + 1]);
-              pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
-            }
-            dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-          }
+          for (int c = 0; c < 8; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        }
+      }
+      if (slice_full) {
+        ptx::fence_proxy_async_smem();
+        __syncwarp();
+        if (lane == 0) {
+          const int x = EPI ? nb * 128 + cq * 32 : nb * 256 + cq * 64;
+          ptx::tma_store_2d(&tmC, s_out, x, s_off[g] + r0);
+          ptx::bulk_commit_group();
         }
       }
     }
+    if (lane == 0) ptx::bulk_wait_all();  // this warp's stores are complete before the CTA exits
     if (!ok) {
       *abort_flag = 1;
       set_status(p.status, MOE_ERR_TIMEOUT);
@@ -1307,6 +1360,30 @@ bool make_map(CUtensorMap* m, const void* base, int ebytes, uint64_t rows, uint6
                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) {
     record_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled rejected the operand layout");
+    return false;
+  }
+  return true;
+}
+
+// 2-D map over a row-major [rows, cols] output for tiled bulk stores of
+// {box_cols, box_rows} boxes (box_cols * ebytes = 128 with 128-byte swizzle).
+bool make_store_map(CUtensorMap* m, void* base, int ebytes, uint64_t rows, uint64_t cols, uint32_t box_cols,
+                    uint32_t box_rows, bool swizzle128) {
+  EncodeTiledFn enc = get_encode_fn();
+  if (!enc) {
+    record_cuda_error(cudaErrorNotSupported, "cuTensorMapEncodeTiled unavailable from the driver");
+    return false;
+  }
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * static_cast<uint64_t>(ebytes)};
+  const cuuint32_t box[2] = {box_cols, box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUtensorMapDataType dt = ebytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  const CUresult r = enc(m, dt, 2, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                         swizzle128 ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
+                         CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) {
+    record_cuda_error(cudaErrorInvalidValue, "cuTensorMapEncodeTiled rejected the output layout");
     return false;
   }
   return true;
@@ -1462,20 +1539,23 @@ int run_bf16_pair(const GemmArgs& a, cudaStream_t s) {
 
 template <int EPI, int OUT>
 int run_fp8(const GemmArgs& a, cudaStream_t s) {
-  using L = Tile<256>;
-  static_assert(L::SMEM <= 227 * 1024, "shared memory budget");
+  constexpr int kF8Smem = F8Smem<EPI, OUT>::SMEM;
   const int nb_rows = EPI ? 2 * a.N : a.N;
   const uint32_t box_b = EPI ? 128 : 256;
   CUtensorMap mA, mB, mBx;
   if (!make_map(&mA, a.A, 1, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
   if (!make_map(&mB, a.B, 1, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 1, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  // output boxes of one warp's 32 rows: 64 bf16 columns (128-byte swizzle), or 32 columns of the gated output
+  CUtensorMap mC;
+  const uint64_t c_rows = static_cast<uint64_t>(a.rows > 0 ? a.rows : 1);
+  if (!make_store_map(&mC, a.C, OUT == 2 ? 1 : 2, c_rows, a.N, EPI ? 32 : 64, 32, !EPI)) return MOE_ERR_CUDA;
   static bool attr_set[64] = {};
   int dev = 0;
   MOE_CUDA_CHECK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
   if (!attr_set[dev]) {
-    MOE_CUDA_CHECK(cudaFuncSetAttribute(gg_fp8_kernel<EPI, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, L::SMEM));
+    MOE_CUDA_CHECK(cudaFuncSetAttribute(gg_fp8_kernel<EPI, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kF8Smem));
     attr_set[dev] = true;
   }
   Params p{};
@@ -1492,7 +1572,7 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
   p.B_scales = a.B_scales;
   p.Bx_scales = a.has_extra ? a.B_extra_scales : a.B_scales;
   p.C_scales = a.C_scales;
-  gg_fp8_kernel<EPI, OUT><<<num_sms(), kThreadsF8, L::SMEM, s>>>(mA, mB, mBx, p);
+  gg_fp8_kernel<EPI, OUT><<<num_sms(), kThreadsF8, kF8Smem, s>>>(mA, mB, mBx, mC, p);
   return launch_status(__func__);
 }
 
