@@ -42,6 +42,8 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat
                                                               const int32_t* __restrict__ t2r,
                                                               const float* __restrict__ w, int has_shared,
                                                               int T, int d, int k, OT* __restrict__ out) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   const int t = blockIdx.x;
   const int c0 = blockIdx.y * kCombCols + threadIdx.x * 8;               // first piece
   const int c1 = c0 + kCombThreads * 8;                                   // second piece
@@ -109,11 +111,10 @@ int launch_combine(const void* Y, const int32_t* t2r, const float* w, int has_sh
   const __nv_bfloat16* y = static_cast<const __nv_bfloat16*>(Y);
   const dim3 grid(T, (d + kCombCols - 1) / kCombCols);
   if (out_dtype == MOE_F32)
-    combine_kernel<float><<<grid, kCombThreads, 0, s>>>(y, t2r, w, has_shared, T, d, k, static_cast<float*>(out));
-  else
-    combine_kernel<__nv_bfloat16>
-        <<<grid, kCombThreads, 0, s>>>(y, t2r, w, has_shared, T, d, k, static_cast<__nv_bfloat16*>(out));
-  return launch_status(__func__);
+    return launch_pdl(__func__, combine_kernel<float>, grid, dim3(kCombThreads), 0, s, y, t2r, w, has_shared, T, d, k,
+                      static_cast<float*>(out));
+  return launch_pdl(__func__, combine_kernel<__nv_bfloat16>, grid, dim3(kCombThreads), 0, s, y, t2r, w, has_shared, T,
+                    d, k, static_cast<__nv_bfloat16*>(out));
 }
 
 }  // namespace moe

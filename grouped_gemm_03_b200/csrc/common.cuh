@@ -8,6 +8,7 @@
 #include <cuda_fp16.h>
 #include <cuda_fp8.h>
 #include <cuda_runtime.h>
+#include <utility>
 
 #include <cstdint>
 
@@ -116,6 +117,34 @@ int record_cuda_error(cudaError_t e, const char* where);
 // Status of the kernel launch just made.
 inline int launch_status(const char* where) {
   const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : record_cuda_error(e, where);
+}
+
+// Programmatic dependent launch.  Every kernel of the library is launched so
+// that it may start while the kernel before it on the stream is finishing,
+// and every kernel begins with pdl_wait(), which returns once the preceding
+// grid has completed and its memory is visible: no kernel touches global
+// memory before that.  pdl_launch_dependents() lets the next kernel's CTAs
+// be scheduled as soon as every CTA of this grid has issued it.  Both are
+// no-ops for a kernel launched without the attribute.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
+// Launch `kernel` on `s` with programmatic stream serialisation allowed.
+template <typename... Params, typename... Args>
+int launch_pdl(const char* where, void (*kernel)(Params...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
+               Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
   return e == cudaSuccess ? MOE_OK : record_cuda_error(e, where);
 }
 }  // namespace moe

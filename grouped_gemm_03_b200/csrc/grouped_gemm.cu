@@ -111,6 +111,8 @@ template <int MMA_N, int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gg_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                    const __grid_constant__ CUtensorMap tmBx, const Params p) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   using L = Tile<MMA_N>;
   constexpr int OUT_COLS = EPI ? MMA_N / 2 : MMA_N;
   constexpr uint32_t IDESC = ptx::make_idesc(BM, MMA_N, 1);
@@ -408,6 +410,8 @@ template <int EPI>
 __global__ void __launch_bounds__(kThreads, 1)
     gg_bf16_swap_kernel(const __grid_constant__ CUtensorMap tmX, const __grid_constant__ CUtensorMap tmW,
                         const __grid_constant__ CUtensorMap tmWx, const Params p) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   constexpr int NT = kSwapNT;
   constexpr int W_BYTES = 128 * 128;
   constexpr int X_BYTES = NT * 128;
@@ -664,6 +668,8 @@ template <int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gg_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBx, const Params p) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   constexpr int MMA_N = 256;
   constexpr int BM2 = 256;
   constexpr int A_BYTES = 128 * 128;
@@ -969,6 +975,8 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
     gg_fp8_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                   const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC,
                   const Params p) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   constexpr int MMA_N = 256;
   using L = F8Smem<EPI, OUT>;
   constexpr int OUT_COLS = EPI ? 128 : 256;
@@ -1449,8 +1457,8 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   p.status = a.status;
   p.wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
   p.stall = a.stall;
-  gg_bf16_kernel<MMA_N, EPI, OUT><<<a.grid > 0 ? a.grid : num_sms(), kThreads, L::SMEM, s>>>(mA, mB, mBx, p);
-  return launch_status(__func__);
+  return launch_pdl(__func__, gg_bf16_kernel<MMA_N, EPI, OUT>, dim3(a.grid > 0 ? a.grid : num_sms()), dim3(kThreads),
+                    L::SMEM, s, mA, mB, mBx, p);
 }
 
 template <int EPI>
@@ -1486,8 +1494,7 @@ int run_bf16_swap(const GemmArgs& a, cudaStream_t s) {
   p.ksplit = 1;
   p.C = a.C;
   p.status = a.status;
-  gg_bf16_swap_kernel<EPI><<<num_sms(), kThreads, kSwapSmem, s>>>(mX, mW, mWx, p);
-  return launch_status(__func__);
+  return launch_pdl(__func__, gg_bf16_swap_kernel<EPI>, dim3(num_sms()), dim3(kThreads), kSwapSmem, s, mX, mW, mWx, p);
 }
 
 template <int EPI, int OUT>
@@ -1523,6 +1530,11 @@ int run_bf16_pair(const GemmArgs& a, cudaStream_t s) {
     clusters[dev] = n > 0 ? n : 1;
   }
   cfg.gridDim = dim3(2 * clusters[dev]);
+  cudaLaunchAttribute attrs[2] = {cfg.attrs[0], {}};
+  attrs[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;  // see launch_pdl
+  attrs[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attrs;
+  cfg.numAttrs = 2;
   Params p{};
   p.offsets = a.offsets;
   p.G_total = a.G + a.has_extra;
@@ -1572,8 +1584,8 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
   p.B_scales = a.B_scales;
   p.Bx_scales = a.has_extra ? a.B_extra_scales : a.B_scales;
   p.C_scales = a.C_scales;
-  gg_fp8_kernel<EPI, OUT><<<num_sms(), kThreadsF8, kF8Smem, s>>>(mA, mB, mBx, mC, p);
-  return launch_status(__func__);
+  return launch_pdl(__func__, gg_fp8_kernel<EPI, OUT>, dim3(num_sms()), dim3(kThreadsF8), kF8Smem, s, mA, mB, mBx, mC,
+                    p);
 }
 
 }  // namespace

@@ -25,6 +25,8 @@ constexpr int kPermThreads = 256;
 
 __global__ void __launch_bounds__(kPermThreads) hist_kernel(const int32_t* __restrict__ idx, int T, int E, int k,
                                                             int32_t* __restrict__ cnt, int* status) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   extern __shared__ int s_cnt[];
   const int b = blockIdx.x;
   const int t0 = b * kTokPerBlock;
@@ -51,6 +53,8 @@ __global__ void __launch_bounds__(kPermThreads) hist_kernel(const int32_t* __res
 __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, int nblk, int E, int R, int T,
                                                     int shared, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   __shared__ int s_part[1024];
   __shared__ int s_tot[1024];
   __shared__ int s_warp[32];
@@ -135,6 +139,8 @@ constexpr int kScatterCols = 512;
 
 template <typename XT, bool kFp8>
 __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   __shared__ int s_idx[kTokPerBlock * kMaxTopK];
   __shared__ int s_row[kTokPerBlock * (kMaxTopK + 1)];
   const int b = blockIdx.x;
@@ -277,25 +283,20 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
     MOE_CUDA_CHECK(cudaMemsetAsync(a.offsets, 0, sizeof(int32_t) * (a.E + 1 + (a.shared ? 1 : 0)), s));
     return MOE_OK;
   }
-  hist_kernel<<<nblk, kPermThreads, sizeof(int) * a.E, s>>>(a.idx, a.T, a.E, a.k, a.block_base, a.status);
-  MOE_CUDA_CHECK(cudaGetLastError());
-  scan_kernel<<<1, 1024, 0, s>>>(a.block_base, nblk, a.E, a.T * a.k, a.T, a.shared, a.counts, a.offsets);
-  MOE_CUDA_CHECK(cudaGetLastError());
+  int st = launch_pdl("hist_kernel", hist_kernel, dim3(nblk), dim3(kPermThreads), sizeof(int) * a.E, s, a.idx, a.T,
+                      a.E, a.k, a.block_base, a.status);
+  if (st != MOE_OK) return st;
+  st = launch_pdl("scan_kernel", scan_kernel, dim3(1), dim3(1024), 0, s, a.block_base, nblk, a.E, a.T * a.k, a.T,
+                  a.shared, a.counts, a.offsets);
+  if (st != MOE_OK) return st;
   const bool fp8 = a.xp_dtype == MOE_E4M3;
   const dim3 grid(nblk, (a.d + kScatterCols - 1) / kScatterCols);
-  if (a.x_dtype == MOE_BF16) {
-    if (fp8)
-      scatter_kernel<__nv_bfloat16, true><<<grid, kPermThreads, 0, s>>>(a);
-    else
-      scatter_kernel<__nv_bfloat16, false><<<grid, kPermThreads, 0, s>>>(a);
-  } else {
-    if (fp8)
-      scatter_kernel<float, true><<<grid, kPermThreads, 0, s>>>(a);
-    else
-      scatter_kernel<float, false><<<grid, kPermThreads, 0, s>>>(a);
-  }
-  MOE_CUDA_CHECK(cudaGetLastError());
-  return MOE_OK;
+  const dim3 block(kPermThreads);
+  if (a.x_dtype == MOE_BF16)
+    return fp8 ? launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true>, grid, block, 0, s, a)
+               : launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, false>, grid, block, 0, s, a);
+  return fp8 ? launch_pdl("scatter_kernel", scatter_kernel<float, true>, grid, block, 0, s, a)
+             : launch_pdl("scatter_kernel", scatter_kernel<float, false>, grid, block, 0, s, a);
 }
 
 }  // namespace moe

@@ -9,6 +9,8 @@ namespace {
 
 __global__ void __launch_bounds__(256) quant_block_kernel(const __nv_bfloat16* __restrict__ W, int N, int K,
                                                           uint8_t* __restrict__ Wq, float* __restrict__ scales) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   __shared__ float s_max[8];
   const int kb = blockIdx.x, nb = blockIdx.y, g = blockIdx.z;
   const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
@@ -59,8 +61,8 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const __nv_bfloat16* _
 int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, cudaStream_t s) {
   if (G == 0) return MOE_OK;
   dim3 grid(K / 128, N / 128, G);
-  quant_block_kernel<<<grid, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(W), N, K, Wq, scales);
-  return launch_status(__func__);
+  return launch_pdl(__func__, quant_block_kernel, grid, dim3(256), 0, s, static_cast<const __nv_bfloat16*>(W), N, K, Wq,
+                    scales);
 }
 
 }  // namespace moe

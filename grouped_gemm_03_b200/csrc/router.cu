@@ -87,6 +87,8 @@ __device__ __forceinline__ void smem8(const __nv_bfloat16* p, float (&f)[8]) {
 template <typename XT, typename WT>
 __global__ void __launch_bounds__(kRWarps * 32) logits_simt_kernel(const XT* __restrict__ x, const WT* __restrict__ Wr,
                                                           int T, int d, int E, float* __restrict__ logits) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   constexpr int DC = 32768 / (kREC * static_cast<int>(sizeof(WT)));  // columns per staged chunk
   constexpr int VPE = 16 / static_cast<int>(sizeof(WT));            // elements per 16-byte copy
   __shared__ __align__(16) WT s_w[kREC][DC];
@@ -199,6 +201,8 @@ __global__ void __launch_bounds__(256) finish_kernel(const LT* __restrict__ part
                                                      int pstride, const float* __restrict__ bias, int N, int E,
                                                      int k, int renorm, float* __restrict__ logits_out,
                                                      int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
   constexpr int TPW = 32 / G;
   constexpr int kBytes = V * static_cast<int>(sizeof(LT));
   constexpr float kLog2e = 1.4426950408889634f;
@@ -327,12 +331,10 @@ int finish_launch(const void* parts, int nsplit, size_t stride, int pstride, con
   const int blocks = max(1, min((N + TPB - 1) / TPB, num_sms() * 32));
   const LT* pp = static_cast<const LT*>(parts);
   if (sizeof(LT) == 2 && nsplit == 1 && bias == nullptr && E <= 65535)
-    finish_kernel<LT, V, G, sizeof(LT) == 2><<<blocks, 256, 0, s>>>(pp, nsplit, stride, pstride, bias, N, E, k, renorm,
-                                                                     lo, idx, w);
-  else
-    finish_kernel<LT, V, G, false><<<blocks, 256, 0, s>>>(pp, nsplit, stride, pstride, bias, N, E, k, renorm, lo,
-                                                          idx, w);
-  return launch_status(__func__);
+    return launch_pdl(__func__, finish_kernel<LT, V, G, sizeof(LT) == 2>, dim3(blocks), dim3(256), 0, s, pp, nsplit,
+                      stride, pstride, bias, N, E, k, renorm, lo, idx, w);
+  return launch_pdl(__func__, finish_kernel<LT, V, G, false>, dim3(blocks), dim3(256), 0, s, pp, nsplit, stride,
+                    pstride, bias, N, E, k, renorm, lo, idx, w);
 }
 
 template <typename LT>
@@ -353,9 +355,8 @@ int finish_dispatch(const void* parts, int nsplit, size_t stride, int pstride, c
 template <typename XT, typename WT>
 int simt_logits(const void* x, const void* Wr, int T, int d, int E, float* logits, cudaStream_t s) {
   dim3 grid((T + kRTok - 1) / kRTok, (E + kREC - 1) / kREC);
-  logits_simt_kernel<XT, WT><<<grid, kRWarps * 32, 0, s>>>(static_cast<const XT*>(x), static_cast<const WT*>(Wr), T, d, E,
-                                                  logits);
-  return launch_status(__func__);
+  return launch_pdl(__func__, logits_simt_kernel<XT, WT>, grid, dim3(kRWarps * 32), 0, s, static_cast<const XT*>(x),
+                    static_cast<const WT*>(Wr), T, d, E, logits);
 }
 
 }  // namespace
