@@ -341,6 +341,13 @@ template <typename LT>
 int finish_dispatch(const void* parts, int nsplit, size_t stride, int pstride, const float* bias, int N, int E, int k,
                     int renorm, float* lo, int32_t* idx, float* w, cudaStream_t s) {
 #define MOE_FINISH(VV, GG) finish_launch<LT, VV, GG>(parts, nsplit, stride, pstride, bias, N, E, k, renorm, lo, idx, w, s)
+  // Few experts: more lanes per token (one or two experts each), so that a
+  // batch of a few thousand tokens still spreads over every SM.
+  if (N >= 1024) {
+    if (E <= 8) return MOE_FINISH(1, 8);
+    if (E <= 16) return MOE_FINISH(1, 16);
+    if (E <= 32) return MOE_FINISH(2, 16);
+  }
   if (E <= 16) return MOE_FINISH(16, 1);
   if (E <= 32) return MOE_FINISH(16, 2);
   if (E <= 64) return MOE_FINISH(16, 4);

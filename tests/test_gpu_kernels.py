@@ -35,7 +35,11 @@ def _rng(seed):
 # ---------------------------------------------------------------- top-k of logits
 @pytest.mark.parametrize("N,E,k,dtype", [(4096, 128, 4, torch.float16), (65536, 128, 4, torch.float16),
                                          (777, 64, 2, torch.float32), (300, 256, 8, torch.bfloat16),
-                                         (129, 8, 2, torch.float16), (64, 40, 3, torch.float32)])
+                                         (129, 8, 2, torch.float16), (64, 40, 3, torch.float32),
+                                         # few experts and many tokens: one or two experts per lane
+                                         (2048, 8, 2, torch.float16), (3001, 16, 4, torch.bfloat16),
+                                         (1500, 32, 8, torch.float32), (1024, 24, 3, torch.float32),
+                                         (4096, 7, 1, torch.float16)])
 @pytest.mark.parametrize("renorm", [False, True])
 def test_topk_logits(N, E, k, dtype, renorm):
     l = make_router_logits(N, E, seed=5, device=DEV, dtype=dtype)
@@ -182,6 +186,8 @@ GEMM_CASES = [
     ([2000, 0, 129], 512, 128, gg.EPI_NONE, torch.float32),
     ([257, 1600, 0, 255], 128, 320, gg.EPI_SILU_GATE, torch.bfloat16),
     ([1536, 1], 256, 512, gg.EPI_SILU_GATE, torch.bfloat16),
+    # gated pair launches leave tails of <= 128 rows (here 128, 128, 1) to a single-CTA launch
+    ([640, 641, 384, 0, 1000, 257], 384, 256, gg.EPI_SILU_GATE, torch.bfloat16),
     # a few tokens per group (fewer than 32 rows per group on average): the weights take the
     # MMA's 128-row side (swap-AB), tokens the 32-wide side
     ([1, 0, 3, 2, 5, 33, 0, 1, 0, 7, 64, 1], 256, 128, gg.EPI_NONE, torch.bfloat16),
