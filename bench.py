@@ -46,7 +46,7 @@ from workload.gen import ROUTER_MICRO  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200; grouped-GEMM TFLOP/s as % of dense tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_FORWARD = 7  # router, hist, scan, scatter, up GEMM, down GEMM, combine
+KERNELS_PER_FORWARD = 8  # router logits, top-k, hist, scan, scatter, up GEMM, down GEMM, combine
 
 
 def log(*a):
