@@ -51,11 +51,10 @@ struct Tile {
   static constexpr int B_BYTES = MMA_N * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TABLE_BYTES = 2 * (kMaxGroups + 2) * 4;
-  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512 - 4096) / STAGE_BYTES;
+  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = 2 * MMA_N;
-  static constexpr int EXTRA_BYTES = 4096;  // amax exchange of the E4M3 epilogue
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES + EXTRA_BYTES;
+  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES;
 };
 
 struct Params {
@@ -667,7 +666,8 @@ constexpr int kPairSmem = 1024 + kPairStages * 32768 + 512 + 2 * (kMaxGroups + 2
 template <int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gg_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                        const __grid_constant__ CUtensorMap tmBx, const Params p) {
+                        const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmB64,
+                        const __grid_constant__ CUtensorMap tmBx64, const Params p) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
   constexpr int MMA_N = 256;
@@ -679,6 +679,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int TMEM_COLS = 512;
   constexpr int OUT_COLS = EPI ? 128 : 256;
   constexpr uint32_t IDESC = ptx::make_idesc(BM2, MMA_N, 1);
+  constexpr uint32_t IDESC_HALF = ptx::make_idesc(128, MMA_N, 1);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -773,12 +774,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int mt = (m_g + BM2 - 1) / BM2;
         const int tl = tile - s_tile[g];
         const int nb = tl / mt, mb = tl % mt;
-        const int a_row = s_off[g] + mb * BM2 + static_cast<int>(rank) * 128;
+        // a group's last tile with at most 128 rows runs as a 128-row pair MMA (64 rows per CTA)
+        const bool half = m_g - mb * BM2 <= 128;
+        const int a_row = s_off[g] + mb * BM2 + static_cast<int>(rank) * (half ? 64 : 128);
         const bool extra = g >= p.G_main;
         const CUtensorMap* mB = extra ? &tmBx : &tmB;
+        const CUtensorMap* mB64 = extra ? &tmBx64 : &tmB64;
         const int gb = extra ? 0 : g;
         const int brow = EPI ? gb * 2 * p.N + static_cast<int>(rank) * p.N + nb * 128
                              : gb * p.N + nb * 256 + static_cast<int>(rank) * 128;
+        // gated half tile: this CTA's 128 B rows are 64 gate rows and the 64 matching up rows, so
+        // that each accumulator lane holds a row's gate and up columns side by side
+        const int hrow = gb * 2 * p.N + nb * 128 + static_cast<int>(rank) * 64;
         for (int kb = 0; kb < nk; ++kb) {
           if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
             ok = false;
@@ -787,7 +794,12 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t fb = ptx::map_to_rank(ptx::smem_u32(&full[stage]), 0);
           if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
           ptx::tma_load_2d_pair(sA + stage * A_BYTES, &tmA, fb, kb * 64, a_row);
-          ptx::tma_load_2d_pair(sB + stage * B_BYTES, mB, fb, kb * 64, brow);
+          if (EPI && half) {
+            ptx::tma_load_2d_pair(sB + stage * B_BYTES, mB64, fb, kb * 64, hrow);
+            ptx::tma_load_2d_pair(sB + stage * B_BYTES + 64 * 128, mB64, fb, kb * 64, hrow + p.N);
+          } else {
+            ptx::tma_load_2d_pair(sB + stage * B_BYTES, mB, fb, kb * 64, brow);
+          }
           if (++stage == STAGES) {
             stage = 0;
             phase ^= 1;
@@ -815,6 +827,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MMA_N;
+        const int g = find_group(s_tile, G, tile);
+        const int m_g = s_off[g + 1] - s_off[g];
+        const int mt = (m_g + BM2 - 1) / BM2;
+        const uint32_t idesc = m_g - ((tile - s_tile[g]) % mt) * BM2 <= 128 ? IDESC_HALF : IDESC;
         for (int kb = 0; kb < nk; ++kb) {
           if (!ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
             ok = false;
@@ -825,7 +841,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sB + stage * B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_f16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb | kk) != 0);
+            ptx::umma_f16_pair(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb | kk) != 0);
           ptx::umma_commit_pair_both(&empty[stage]);
           if (++stage == STAGES) {
             stage = 0;
@@ -856,7 +872,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       const int mt = (m_g + BM2 - 1) / BM2;
       const int tl = tile - s_tile[g];
       const int nb = tl / mt, mb = tl % mt;
-      const int r_in = mb * BM2 + static_cast<int>(rank) * 128 + row_t;
+      // Half tile (128-row pair MMA): each CTA holds 64 rows; lanes 0-63 carry the first 128
+      // columns of the MMA's 256 and lanes 64-127 the last 128, both at accumulator columns 0-127.
+      const bool half = m_g - mb * BM2 <= 128;
+      const int lrow = half ? (row_t & 63) : row_t;
+      const int hsel = half ? (row_t >> 6) : 0;
+      const int r_in = mb * BM2 + static_cast<int>(rank) * (half ? 64 : 128) + lrow;
       const bool valid = r_in < m_g;
       const size_t grow = static_cast<size_t>(s_off[g] + r_in);
       if (!ptx::mbar_wait_warp(&tfull[acc], use & 1, abort_flag, kWaitLimitNs)) {
@@ -866,13 +887,17 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_fence_after();
       const uint32_t tacc = lane_base + acc * MMA_N;
+      // output columns of this lane: in a half tile each lane has half of them (with the gate:
+      // gate at accumulator columns [0, 64), up at [64, 128)), in a full tile all
+      const int ncols = half ? OUT_COLS / 2 : OUT_COLS;
+      const int col0 = nb * OUT_COLS + hsel * ncols;
       if constexpr (EPI == 1) {
-        __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS;
+        __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + grow * p.N + col0;
 #pragma unroll 1
-        for (int c = 0; c < OUT_COLS; c += 32) {
+        for (int c = 0; c < ncols; c += 32) {
           uint32_t gv[32], uv[32];
           ptx::tmem_ld_32x32b_x32(tacc + c, gv);
-          ptx::tmem_ld_32x32b_x32(tacc + OUT_COLS + c, uv);
+          ptx::tmem_ld_32x32b_x32(tacc + ncols + c, uv);
           ptx::tmem_ld_wait();
           if (valid) {
             uint32_t packed[16];
@@ -892,13 +917,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       } else {
 #pragma unroll 1
-        for (int c = 0; c < OUT_COLS; c += 32) {
+        for (int c = 0; c < ncols; c += 32) {
           uint32_t v[32];
           ptx::tmem_ld_32x32b_x32(tacc + c, v);
           ptx::tmem_ld_wait();
           if (valid) {
             if constexpr (OUT == 1) {
-              uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.C) + grow * p.N + nb * OUT_COLS + c);
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<float*>(p.C) + grow * p.N + col0 + c);
 #pragma unroll
               for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
             } else {
@@ -909,8 +934,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
                 packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
               }
-              uint4* dst =
-                  reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS + c);
+              uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + col0 + c);
 #pragma unroll
               for (int i = 0; i < 4; ++i)
                 dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
@@ -1505,6 +1529,10 @@ int run_bf16_pair(const GemmArgs& a, cudaStream_t s) {
   if (!make_map(&mA, a.A, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, 128)) return MOE_ERR_CUDA;
   if (!make_map(&mB, a.B, 2, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, 128)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, 128)) return MOE_ERR_CUDA;
+  // 64-row boxes for the gated half tiles (64 gate rows, then the 64 matching up rows)
+  CUtensorMap mB64, mBx64;
+  if (!make_map(&mB64, a.B, 2, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, 64)) return MOE_ERR_CUDA;
+  if (!make_map(&mBx64, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, 64)) return MOE_ERR_CUDA;
   static int clusters[64] = {};
   int dev = 0;
   MOE_CUDA_CHECK(cudaGetDevice(&dev));
@@ -1545,7 +1573,7 @@ int run_bf16_pair(const GemmArgs& a, cudaStream_t s) {
   p.ksplit = 1;
   p.C = a.C;
   p.status = a.status;
-  MOE_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gg_bf16_pair_kernel<EPI, OUT>, mA, mB, mBx, p));
+  MOE_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gg_bf16_pair_kernel<EPI, OUT>, mA, mB, mBx, mB64, mBx64, p));
   return MOE_OK;
 }
 

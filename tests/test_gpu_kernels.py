@@ -186,8 +186,10 @@ GEMM_CASES = [
     ([2000, 0, 129], 512, 128, gg.EPI_NONE, torch.float32),
     ([257, 1600, 0, 255], 128, 320, gg.EPI_SILU_GATE, torch.bfloat16),
     ([1536, 1], 256, 512, gg.EPI_SILU_GATE, torch.bfloat16),
-    # gated pair launches leave tails of <= 128 rows (here 128, 128, 1) to a single-CTA launch
-    ([640, 641, 384, 0, 1000, 257], 384, 256, gg.EPI_SILU_GATE, torch.bfloat16),
+    # last tiles of 128, 129, 128, 232, 129 and 1 rows: those of at most 128 rows run as 128-row pair MMAs
+    ([640, 641, 384, 0, 1000, 1153, 257], 384, 256, gg.EPI_SILU_GATE, torch.bfloat16),
+    # fp32 output on CTA pairs, last tiles of 76 and 30 rows (128-row pair MMAs)
+    ([1100, 30], 256, 128, gg.EPI_NONE, torch.float32),
     # a few tokens per group (fewer than 32 rows per group on average): the weights take the
     # MMA's 128-row side (swap-AB), tokens the 32-wide side
     ([1, 0, 3, 2, 5, 33, 0, 1, 0, 7, 64, 1], 256, 128, gg.EPI_NONE, torch.bfloat16),
