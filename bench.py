@@ -384,6 +384,20 @@ def run_ours(args, rank, world, dev):
         raise RuntimeError(f"device status {status}")
     ms = max_over_ranks(float(np.mean(times)), world, dev)
 
+    # --- the same forward replayed from a CUDA graph (one launch of the whole layer)
+    gstream = torch.cuda.Stream()
+    gstream.wait_stream(stream)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.stream(gstream):
+        step()  # warm the capture stream
+        with torch.cuda.graph(graph, stream=gstream):
+            step()
+    stream.wait_stream(gstream)
+    torch.cuda.synchronize()
+    graph_times = time_steps(graph.replay, max(3, args.steps // 2), 3, flush, stream)
+    graph_ms = max_over_ranks(float(np.mean(graph_times)), world, dev)
+    del graph
+
     # --- e2e: host buffers through moe_forward_host, copies inside the timed region
     xh = inp["x"].cpu().pin_memory()
     oh = torch.empty((s.T, s.d), dtype=out.dtype).pin_memory()
@@ -405,7 +419,7 @@ def run_ours(args, rank, world, dev):
             e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
         e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
         kern[name] = e
-    return dict(ms=ms, e2e_ms=e2e_ms, kernels=kern, clocks=clk.summary(), inp=inp, s=s, counts=counts.cpu().numpy(),
+    return dict(ms=ms, e2e_ms=e2e_ms, graph_ms=graph_ms, kernels=kern, clocks=clk.summary(), inp=inp, s=s, counts=counts.cpu().numpy(),
                 out_dtype=out.dtype)
 
 
@@ -481,6 +495,9 @@ def main():
             "e2e": {"value": round(job_tokens_per_s(T, world, r["e2e_ms"]), 1), "unit": "tokens/s",
                     "h2d_bytes_per_step": T * s.d * (4 if s.x_dtype == "f32" else 2),
                     "d2h_bytes_per_step": T * s.d * (4 if r["out_dtype"] == torch.float32 else 2)},
+            "graph": {"ms_per_step": round(r["graph_ms"], 4),
+                      "value": round(job_tokens_per_s(T, world, r["graph_ms"]), 1), "unit": "tokens/s",
+                      "note": "the same forward captured once in a CUDA graph and replayed"},
             "gpu_launches": KERNELS_PER_FORWARD * args.steps,
             "clocks": r["clocks"],
             "expert_counts": {"min": int(r["counts"].min()), "max": int(r["counts"].max()),
