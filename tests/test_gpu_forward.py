@@ -80,7 +80,9 @@ def test_tiny_layer_every_element(renorm):
 
 
 @pytest.mark.parametrize("T,E,k,I,shared", [(1, 8, 2, 128, True), (37, 4, 4, 256, False), (500, 16, 1, 384, True),
-                                             (64, 64, 2, 128, False)])
+                                             (64, 64, 2, 128, False),
+                                             # the largest layer shape the library takes: 1023 experts + shared, top-32
+                                             (40, 1023, 32, 128, True)])
 def test_small_ragged_layers(T, E, k, I, shared):
     s = shape_of("tiny", T=T, E=E, k=k, inter=I, shared_inter=I if shared else 0, x_dtype="bf16",
                  router_dtype="bf16")

@@ -39,7 +39,9 @@ def _rng(seed):
                                          # few experts and many tokens: one or two experts per lane
                                          (2048, 8, 2, torch.float16), (3001, 16, 4, torch.bfloat16),
                                          (1500, 32, 8, torch.float32), (1024, 24, 3, torch.float32),
-                                         (4096, 7, 1, torch.float16)])
+                                         (4096, 7, 1, torch.float16),
+                                         # the largest supported: 1024 experts, top-32
+                                         (300, 1024, 32, torch.float32), (129, 1000, 17, torch.bfloat16)])
 @pytest.mark.parametrize("renorm", [False, True])
 def test_topk_logits(N, E, k, dtype, renorm):
     l = make_router_logits(N, E, seed=5, device=DEV, dtype=dtype)
@@ -108,7 +110,9 @@ def _random_routing(T, E, k, seed, skew=0.0):
 @pytest.mark.parametrize("T,E,k,shared,xdt", [(256, 8, 2, True, torch.float32), (77, 8, 2, False, torch.bfloat16),
                                               (1000, 256, 8, True, torch.bfloat16), (33, 64, 2, False, torch.float32),
                                               (4096, 8, 2, False, torch.bfloat16), (5, 4, 4, True, torch.bfloat16),
-                                              (1, 16, 3, False, torch.bfloat16)])
+                                              (1, 16, 3, False, torch.bfloat16),
+                                              # the largest supported: 1024 experts (1023 with the shared group), top-32
+                                              (100, 1024, 32, False, torch.bfloat16), (70, 1023, 32, True, torch.float32)])
 def test_permute_bf16(T, E, k, shared, xdt):
     d = 256
     x = torch.randn((T, d), device=DEV).to(xdt)
@@ -196,6 +200,9 @@ GEMM_CASES = [
     ([2, 0, 1, 40, 3, 0, 0, 9], 192, 320, gg.EPI_SILU_GATE, torch.bfloat16),
     ([31, 32, 33, 0, 1], 128, 64, gg.EPI_NONE, torch.bfloat16),
     ([65, 0, 2, 0, 0, 0], 64, 256, gg.EPI_SILU_GATE, torch.bfloat16),
+    # the largest group count one launch takes (1024): a few rows each (swap-AB), and up to 300 rows each
+    ([int(v) for v in np.random.default_rng(1).integers(0, 4, 1024)], 128, 64, gg.EPI_NONE, torch.bfloat16),
+    ([int(v) for v in np.random.default_rng(2).integers(0, 300, 1024)], 128, 64, gg.EPI_SILU_GATE, torch.bfloat16),
 ]
 
 
