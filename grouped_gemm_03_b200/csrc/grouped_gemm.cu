@@ -32,6 +32,14 @@
 // SiLU-gate epilogue: per k-step the B tile is [gate rows n0..n0+127 ; up rows
 // N+n0..N+n0+127], so one 128 x 256 MMA produces gate and up side by side in
 // TMEM and the epilogue writes h = silu(g) * u for 128 output columns.
+//
+// Variants, chosen on the host from the shapes alone (plan_grouped_gemm):
+//   gg_bf16_kernel       the structure above (128-row tiles, N_mma 64..256);
+//   gg_bf16_pair_kernel  CTA pairs sharing 256-row tiles (large groups);
+//   gg_bf16_swap_kernel  weights on the MMA's 128-row side, tokens on the
+//                        32-wide side (groups of a few tokens);
+//   gg_fp8_kernel        E4M3 operands, scales applied per 128-wide K block.
+// Every kernel begins with the programmatic-dependent-launch wait (common.cuh).
 #include <cstdio>
 #include <mutex>
 
