@@ -120,6 +120,11 @@ inline int launch_status(const char* where) {
   return e == cudaSuccess ? MOE_OK : record_cuda_error(e, where);
 }
 
+// silu(g) = g / (1 + e^-g) with the fast reciprocal-based division (a few ulp;
+// for g below about -87 the denominator overflows and the result is -0, the
+// limit of the function).
+__device__ __forceinline__ float silu(float g) { return __fdividef(g, 1.0f + __expf(-g)); }
+
 // Programmatic dependent launch.  Every kernel of the library is launched so
 // that it may start while the kernel before it on the stream is finishing,
 // and every kernel begins with pdl_wait(), which returns once the preceding

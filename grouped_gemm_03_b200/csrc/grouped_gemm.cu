@@ -345,8 +345,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
-              const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(uv[2 * i]);
-              const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(uv[2 * i + 1]);
+              const float h0 = silu(g0) * __uint_as_float(uv[2 * i]);
+              const float h1 = silu(g1) * __uint_as_float(uv[2 * i + 1]);
               const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
               packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
             }
@@ -636,7 +636,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const float mine = __uint_as_float(v[t]);
           const float up = __shfl_xor_sync(0xffffffffu, mine, 16);
           if (lane < 16 && t < ntok) {
-            const float hval = mine / (1.0f + __expf(-mine)) * up;
+            const float hval = silu(mine) * up;
             C[(row0 + t) * p.N + col] = __float2bfloat16_rn(hval);
           }
         }
@@ -912,8 +912,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
               const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
-              const float h0 = g0 / (1.0f + __expf(-g0)) * __uint_as_float(uv[2 * i]);
-              const float h1 = g1 / (1.0f + __expf(-g1)) * __uint_as_float(uv[2 * i + 1]);
+              const float h0 = silu(g0) * __uint_as_float(uv[2 * i]);
+              const float h1 = silu(g1) * __uint_as_float(uv[2 * i + 1]);
               const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
               packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
             }
@@ -1270,8 +1270,8 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float2 gt = acc[i], up = acc[16 + i];
-          acc[i].x = gt.x / (1.0f + __expf(-gt.x)) * up.x;
-          acc[i].y = gt.y / (1.0f + __expf(-gt.y)) * up.y;
+          acc[i].x = silu(gt.x) * up.x;
+          acc[i].y = silu(gt.y) * up.y;
         }
 
         if constexpr (OUT == 2) {

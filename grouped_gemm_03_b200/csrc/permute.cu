@@ -49,37 +49,44 @@ __global__ void __launch_bounds__(kPermThreads) hist_kernel(const int32_t* __res
 }
 
 // Single CTA of 1024 threads: thread (e, c) owns expert e and a contiguous
-// chunk c of the token blocks.
+// chunk c of the token blocks; the tpe (<= 32) threads of one expert are
+// consecutive lanes of one warp, so the chunk prefix is a segmented shuffle
+// scan.  Counts are read and rewritten 8 blocks at a time so that the loads
+// of a batch are in flight together.
+constexpr int kScanBatch = 8;
+
 __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, int nblk, int E, int R, int T,
                                                     int shared, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
-  __shared__ int s_part[1024];
   __shared__ int s_tot[1024];
+  __shared__ int s_off[1024];
   __shared__ int s_warp[32];
-  int tpe = 1;  // threads per expert (power of two, tpe * E <= 1024)
-  while (tpe * 2 * E <= 1024 && tpe * 2 <= nblk) tpe *= 2;
+  int tpe = 1;  // threads per expert (power of two <= 32, tpe * E <= 1024)
+  while (tpe < 32 && tpe * 2 * E <= 1024 && tpe * 2 <= nblk) tpe *= 2;
   const int chunk = (nblk + tpe - 1) / tpe;
   const int e = threadIdx.x / tpe, c = threadIdx.x % tpe;
   const bool active = e < E;
   const int b0 = c * chunk, b1 = min(nblk, b0 + chunk);
   int local = 0;
-  if (active)
-    for (int b = b0; b < b1; ++b) local += base[static_cast<size_t>(b) * E + e];
-  s_part[threadIdx.x] = local;
-  __syncthreads();
-  // per-expert total and exclusive chunk prefix (tpe is small)
-  int chunk_pre = 0;
   if (active) {
-    int tot = 0;
-    for (int cc = 0; cc < tpe; ++cc) {
-      const int v = s_part[e * tpe + cc];
-      if (cc < c) chunk_pre += v;
-      tot += v;
+    for (int b = b0; b < b1; b += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int u = 0; u < kScanBatch; ++u) v[u] = b + u < b1 ? base[static_cast<size_t>(b + u) * E + e] : 0;
+#pragma unroll
+      for (int u = 0; u < kScanBatch; ++u) local += v[u];
     }
-    if (c == 0) s_tot[e] = tot;
   }
+  // inclusive scan of the chunk sums over the expert's tpe lanes (every lane takes part)
+  int incl_c = local;
+  for (int o = 1; o < tpe; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, incl_c, o);
+    if (c >= o) incl_c += y;
+  }
+  const int chunk_pre = incl_c - local;
+  if (active && c == tpe - 1) s_tot[e] = incl_c;  // the expert's total
   __syncthreads();
   // exclusive scan of s_tot[0..E) by the whole block (one value per thread)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -104,9 +111,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, 
   }
   __syncthreads();
   const int excl = incl - mine + s_warp[warp];
-  __syncthreads();
   if (threadIdx.x < E) {
-    s_part[threadIdx.x] = excl;  // reuse: offsets
+    s_off[threadIdx.x] = excl;
     counts[threadIdx.x] = mine;
     offsets[threadIdx.x] = excl;
   }
@@ -116,12 +122,16 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, 
   }
   __syncthreads();
   if (active) {
-    int run = s_part[e] + chunk_pre;
-    for (int b = b0; b < b1; ++b) {
-      const size_t i = static_cast<size_t>(b) * E + e;
-      const int v = base[i];
-      base[i] = run;
-      run += v;
+    int run = s_off[e] + chunk_pre;
+    for (int b = b0; b < b1; b += kScanBatch) {
+      int v[kScanBatch];
+#pragma unroll
+      for (int u = 0; u < kScanBatch; ++u) v[u] = b + u < b1 ? base[static_cast<size_t>(b + u) * E + e] : 0;
+#pragma unroll
+      for (int u = 0; u < kScanBatch; ++u) {
+        if (b + u < b1) base[static_cast<size_t>(b + u) * E + e] = run;
+        run += v[u];
+      }
     }
   }
 }
