@@ -347,6 +347,10 @@ int finish_dispatch(const void* parts, int nsplit, size_t stride, int pstride, c
     if (E <= 8) return MOE_FINISH(1, 8);
     if (E <= 16) return MOE_FINISH(1, 16);
     if (E <= 32) return MOE_FINISH(2, 16);
+  } else if (E > 16 && E <= 128) {
+    // few tokens: 16 lanes per token, so that a decode batch spreads over more CTAs
+    if (E <= 64) return MOE_FINISH(4, 16);
+    return MOE_FINISH(8, 16);
   }
   if (E <= 16) return MOE_FINISH(16, 1);
   if (E <= 32) return MOE_FINISH(16, 2);

@@ -41,7 +41,9 @@ def _rng(seed):
                                          (1500, 32, 8, torch.float32), (1024, 24, 3, torch.float32),
                                          (4096, 7, 1, torch.float16),
                                          # the largest supported: 1024 experts, top-32
-                                         (300, 1024, 32, torch.float32), (129, 1000, 17, torch.bfloat16)])
+                                         (300, 1024, 32, torch.float32), (129, 1000, 17, torch.bfloat16),
+                                         # few tokens, 65..128 experts: 16 lanes of 8 experts per token
+                                         (500, 100, 4, torch.float16), (200, 128, 6, torch.bfloat16)])
 @pytest.mark.parametrize("renorm", [False, True])
 def test_topk_logits(N, E, k, dtype, renorm):
     l = make_router_logits(N, E, seed=5, device=DEV, dtype=dtype)
