@@ -31,6 +31,17 @@ def test_header_declares_the_binding_surface():
     assert header_functions() == gg.exported_symbols()
 
 
+def test_binding_signatures_match_the_header():
+    # parameter count of every declaration against the ctypes argument list of the binding
+    text = re.sub(r"/\*.*?\*/", "", open(HEADER).read(), flags=re.S)
+    decls = re.findall(r"\b(moe_[a-z0-9_]+)\s*\(([^;{]*?)\)\s*;", text, flags=re.S)
+    assert len(decls) == len(gg.exported_symbols())
+    for name, params in decls:
+        p = params.strip()
+        n = 0 if p in ("", "void") else len(p.split(","))
+        assert len(gg._SIGS[name][1]) == n, name
+
+
 def test_library_exports_every_declared_symbol(L):
     out = subprocess.run(["nm", "-D", "--defined-only", gg.LIB_PATH], capture_output=True, text=True).stdout
     exported = set(re.findall(r"\bT (moe_[a-z0-9_]+)$", out, flags=re.M))
