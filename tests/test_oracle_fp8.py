@@ -11,7 +11,12 @@
     (a different association of the same sum), which catches a wrong scale
     index or a transposed block;
   * the FP8 forward with identical experts follows the same closed form as
-    the bf16 one within quantisation error.
+    the bf16 one within quantisation error;
+  * the FFN's intermediate h: its value is silu(g) * u of the dequantised
+    products (scipy's logistic function), its codes and scales follow one
+    scale per row per 128 columns group by group (a one-scale-per-row
+    variant is shown to fail that check), and y is a plain matmul of the
+    dequantised codes.
 (MegaMoE walk-through §2.3 and §5.1: per-token / per-block scales, E4M3 forward.)
 """
 import numpy as np
@@ -148,3 +153,88 @@ def test_fp8_forward_identical_experts_closed_form():
 def test_quantiser_rejects_ragged_blocks(shape):
     with pytest.raises(ValueError):
         fp8.quantize_128x128(np.zeros(shape, np.float32))
+
+
+# ---------------------------------------------------------------- the re-quantisation of h
+# swiglu_ffn_fp8 quantises the intermediate h = silu(g) * u once more, per row
+# per 128 columns, before the down projection (MegaMoE walk-through §2.3 and
+# §5.1: activations carry one scale per token per 128-element group).  The
+# pins below check its three outputs against what the definition fixes,
+# computed here by other means: h against scipy's logistic function on the
+# dequantised operands, hq / sh group by group against the quantisation rule,
+# y against a plain matmul of the dequantised codes.
+
+def _ffn_case(I=384, d=256, T=8, seed=11):
+    """Quantised operands whose h has 128-column groups of very different size."""
+    rng = np.random.default_rng(seed)
+    x = oracle.bf16_round(rng.normal(size=(T, d))).astype(np.float32)
+    W1 = rng.normal(size=(2 * I, d)) * 0.05
+    mag = np.array([1.0, 40.0, 0.02])[: I // 128]       # per 128-column group of h
+    for gi, m in enumerate(mag):
+        W1[128 * gi:128 * gi + 128] *= np.sqrt(m)            # gate rows of the group
+        W1[I + 128 * gi:I + 128 * gi + 128] *= np.sqrt(m)    # the matching up rows
+    W2 = rng.normal(size=(d, I)) * 0.05
+    xq, sx = fp8.quantize_1x128(x)
+    W1q, s1 = fp8.quantize_128x128(W1.astype(np.float32))
+    W2q, s2 = fp8.quantize_128x128(W2.astype(np.float32))
+    return xq, sx, W1q, s1, W2q, s2
+
+
+def test_fp8_ffn_h_is_silu_gate_of_the_dequantised_products():
+    from scipy.special import expit
+    xq, sx, W1q, s1, W2q, s2 = _ffn_case()
+    r = fp8.swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)
+    I = W1q.shape[0] // 2
+    X = fp8.dequantize_1x128(xq, sx)
+    W1 = fp8.dequantize_128x128(W1q, s1)
+    g = X @ W1[:I].T
+    u = X @ W1[I:].T
+    want = g * expit(g) * u
+    assert np.allclose(r["h"], want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def _check_groupwise_quantisation(h32, hq, sh):
+    """Every row's every 128-column group: amax -> +-448*s with s = fp32(amax)/448,
+    the rest within half an E4M3 step at that group's scale.  Returns the
+    number of groups that break the rule (0 when hq / sh are right)."""
+    M, N = h32.shape
+    deq = fp8.e4m3_decode(hq)
+    broken = 0
+    for m in range(M):
+        for gi in range(N // 128):
+            blk = h32[m, 128 * gi:128 * gi + 128].astype(np.float64)
+            amax = np.float32(np.abs(blk).max())
+            s = np.float32(amax / np.float32(448.0)) if amax > 0 else np.float32(1.0)
+            got = deq[m, 128 * gi:128 * gi + 128]
+            j = int(np.argmax(np.abs(blk)))
+            ok = sh[m, gi] == s and abs(got[j]) == 448.0 and np.sign(got[j]) == np.sign(blk[j])
+            v = blk / float(s)
+            half_step = np.maximum(np.abs(v) * 2.0 ** -4, 2.0 ** -10) * (1 + 1e-9)
+            ok = ok and np.all(np.abs(got - v) <= half_step)
+            broken += 0 if ok else 1
+    return broken
+
+
+def test_fp8_ffn_h_codes_follow_one_scale_per_row_per_128_columns():
+    xq, sx, W1q, s1, W2q, s2 = _ffn_case()
+    r = fp8.swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)
+    h32 = r["h"].astype(np.float32)
+    assert r["sh"].shape == (h32.shape[0], h32.shape[1] // 128) and r["sh"].dtype == np.float32
+    # the three groups of a row really do have very different scales
+    assert np.all(r["sh"][:, 1] > 100 * r["sh"][:, 2])
+    assert _check_groupwise_quantisation(h32, r["hq"], r["sh"]) == 0
+    # the check is sharp: one scale per row (over all I columns) breaks it
+    row_amax = np.abs(h32).max(axis=1).astype(np.float32)
+    s_row = (row_amax / np.float32(448.0)).astype(np.float32)
+    hq_row = fp8.e4m3_encode((h32 / s_row[:, None]).astype(np.float32))
+    sh_row = np.repeat(s_row[:, None], h32.shape[1] // 128, axis=1)
+    assert _check_groupwise_quantisation(h32, hq_row, sh_row) >= h32.shape[0]
+
+
+def test_fp8_ffn_y_is_the_product_of_the_dequantised_codes():
+    xq, sx, W1q, s1, W2q, s2 = _ffn_case()
+    r = fp8.swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)
+    H = fp8.dequantize_1x128(r["hq"], r["sh"])
+    W2 = fp8.dequantize_128x128(W2q, s2)
+    want = H @ W2.T
+    assert np.allclose(r["y"], want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
