@@ -19,6 +19,8 @@ namespace moe {
 constexpr int kMaxGroups = 1024;     // experts (+ shared) one grouped GEMM launch handles
 constexpr int kMaxTopK = 32;
 constexpr int kMaxExperts = 1024;
+// Rows of a permuted buffer (T*k + T) are int32 indices in the kernels.
+constexpr long long kMaxPermuteRows = 1ll << 30;
 constexpr uint64_t kWaitLimitNs = 2000000000ull;  // 2 s per pipeline wait
 
 // Record the first device-side error in the status word (0 = OK).

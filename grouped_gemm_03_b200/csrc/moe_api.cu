@@ -92,7 +92,7 @@ int check_config(const moe_config* c) {
   if (c->d % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->expert_dtype == MOE_E4M3 && c->d % 256 != 0) return MOE_ERR_UNSUPPORTED;
   const long long rows = static_cast<long long>(c->T) * (c->k + 1);
-  if (rows * c->d > (1ll << 40) || rows > (1ll << 30)) return MOE_ERR_UNSUPPORTED;
+  if (rows * c->d > (1ll << 40) || rows > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
 }
 
@@ -181,6 +181,7 @@ int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int 
                 int xp_dtype, void* xp, float* xp_scales, int32_t* counts, int32_t* offsets, int32_t* row_to_token,
                 int32_t* token_to_row, void* ws, size_t ws_bytes, void* stream) {
   if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || k > kMaxTopK || E > kMaxExperts) return MOE_ERR_INVALID;
+  if (static_cast<long long>(T) * (k + 1) > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
   if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID;
   if (xp_dtype != MOE_BF16 && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID;
   if (d % 8 != 0 || (xp_dtype == MOE_E4M3 && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;

@@ -315,16 +315,15 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
 // Allocation-free permute (moe_permute_noalloc).
 //
 // Some callers cannot hand this library a workspace: a plugin whose host
-// runtime owns all device memory and offers none, code that must not call
-// cudaMalloc while a stream capture is in progress, or a serving loop whose
-// memory plan is frozen at start-up.  For them the permute's scratch (the
-// status word and the per-block expert counts) lives in this file-scope
-// device array instead of a caller workspace.  Every GPU that loads the
-// library keeps the array (1 MiB + 256 bytes) until the process exits; all
-// calls on a device share it, so calls whose kernels overlap on the GPU (two
-// streams, say) race on it and must be ordered by the caller.  A call
-// rewrites every count it reads and clears the status word first, so what
-// a previous call left there does not matter.
+// runtime owns all device memory and offers none, or a serving loop whose
+// memory plan is frozen at start-up and allows no allocation afterwards.
+// For them the permute's scratch (the status word and the per-block expert
+// counts) lives in this file-scope device array instead of a caller
+// workspace.  Every GPU that loads the library keeps the array (1 MiB + 256
+// bytes) until the process exits; all calls on a device share it, so calls
+// whose kernels overlap on the GPU (two streams, say) race on it and must be
+// ordered by the caller.  A call rewrites every count it reads and clears
+// the status word first, so what a previous call left there does not matter.
 namespace moe {
 namespace {
 
@@ -333,25 +332,76 @@ constexpr size_t kNoAllocCountWords = 262144;    // per-block expert counts (1 M
 
 static __device__ __align__(256) int32_t g_permute_scratch[kNoAllocStatusWords + kNoAllocCountWords];
 
-std::mutex g_scratch_mu;
-int32_t* g_scratch_dev[64] = {};
+// The device address of a __device__ array belongs to the CUDA context the
+// module is loaded in, not to a device ordinal: a caller may drive the
+// library from a context of its own, and a context destroyed by
+// cudaDeviceReset is replaced by a new one with the module loaded afresh.
+// So the address is cached per context, keyed by the context's unique id
+// (cuCtxGetId: never reused within the process, unlike a CUcontext handle).
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
 
-// Device address of g_permute_scratch on the current device.  In host code
+struct ScratchEntry {
+  unsigned long long ctx_id;
+  int32_t* ptr;
+};
+std::mutex g_scratch_mu;
+ScratchEntry g_scratch_cache[64] = {};
+int g_scratch_used = 0;
+int g_scratch_next = 0;  // next entry to replace once the table is full
+
+template <typename Fn>
+Fn driver_entry(const char* name) {
+  void* f = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &f, cudaEnableDefault, &q) != cudaSuccess || q != cudaDriverEntryPointSuccess)
+    return nullptr;
+  return reinterpret_cast<Fn>(f);
+}
+
+// Device address of g_permute_scratch in the current context.  In host code
 // the array's name is only a host-side stand-in, so it must never be passed
-// to a kernel; the address is looked up once per device (with that device
-// current) and cached.
+// to a kernel; the address is looked up once per context, with that context
+// current, and cached.
 int noalloc_scratch(int32_t** out) {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess) return MOE_ERR_CUDA;
-  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
-  std::lock_guard<std::mutex> lock(g_scratch_mu);
-  if (!g_scratch_dev[dev]) {
-    void* p = nullptr;
-    const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
-    if (e != cudaSuccess || p == nullptr) return MOE_ERR_CUDA;
-    g_scratch_dev[dev] = static_cast<int32_t*>(p);
+  static const CtxGetCurrentFn get_ctx = driver_entry<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_entry<CtxGetIdFn>("cuCtxGetId");
+  if (!get_ctx || !get_id) return record_cuda_error(cudaErrorNotSupported, "cuCtxGetCurrent / cuCtxGetId");
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS) return record_cuda_error(cudaErrorDeviceUninitialized, "cuCtxGetCurrent");
+  void* fresh = nullptr;
+  if (ctx == nullptr) {
+    // no context is current on this thread yet: the runtime binds the
+    // current device's primary context on its first call, this lookup
+    const cudaError_t e = cudaGetSymbolAddress(&fresh, g_permute_scratch);
+    if (e != cudaSuccess) return record_cuda_error(e, "cudaGetSymbolAddress(g_permute_scratch)");
+    if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr)
+      return record_cuda_error(cudaErrorDeviceUninitialized, "no current CUDA context for moe_permute_noalloc");
   }
-  *out = g_scratch_dev[dev];
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return record_cuda_error(cudaErrorDeviceUninitialized, "cuCtxGetId");
+  std::lock_guard<std::mutex> lock(g_scratch_mu);
+  for (int i = 0; i < g_scratch_used; ++i)
+    if (g_scratch_cache[i].ctx_id == id) {
+      *out = g_scratch_cache[i].ptr;
+      return MOE_OK;
+    }
+  void* p = fresh;
+  if (p == nullptr) {
+    const cudaError_t e = cudaGetSymbolAddress(&p, g_permute_scratch);
+    if (e != cudaSuccess) return record_cuda_error(e, "cudaGetSymbolAddress(g_permute_scratch)");
+  }
+  if (p == nullptr) return record_cuda_error(cudaErrorInvalidSymbol, "cudaGetSymbolAddress(g_permute_scratch)");
+  // a bounded table: once full, the oldest entry is replaced
+  int slot;
+  if (g_scratch_used < 64) {
+    slot = g_scratch_used++;
+  } else {
+    slot = g_scratch_next;
+    g_scratch_next = (g_scratch_next + 1) % 64;
+  }
+  g_scratch_cache[slot] = {id, static_cast<int32_t*>(p)};
+  *out = static_cast<int32_t*>(p);
   return MOE_OK;
 }
 
@@ -363,6 +413,7 @@ extern "C" int moe_permute_noalloc(const void* x, int x_dtype, const int32_t* to
                                    int32_t* offsets, int32_t* row_to_token, int32_t* token_to_row, void* stream) {
   using namespace moe;
   if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || k > kMaxTopK || E > kMaxExperts) return MOE_ERR_INVALID;
+  if (static_cast<long long>(T) * (k + 1) > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
   if (static_cast<size_t>(permute_blocks(T)) * static_cast<size_t>(E) > kNoAllocCountWords)
     return MOE_ERR_UNSUPPORTED;  // beyond the built-in scratch: use moe_permute with a workspace
   if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID;

@@ -127,6 +127,7 @@ int moe_topk_logits(const void* logits, int dtype, int N, int E, int k, int reno
  *                = sum of counts before e, offsets[E] = R, offsets[E+1] = R+T
  *   row_to_token [R'] int32;  token_to_row [T, k] int32
  *   ws           moe_permute_workspace_size(T, E) bytes (status + per-block counts)
+ * T * (k + 1) <= 2^30 (rows are int32 indices), else MOE_ERR_UNSUPPORTED.
  * Out-of-range or repeated expert ids set MOE_ERR_INVALID in the status word
  * and leave the outputs unspecified. */
 size_t moe_permute_workspace_size(int T, int E);
@@ -137,18 +138,21 @@ int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int 
 
 /* Allocation-free variant of moe_permute, for callers that cannot give the
  * library any device memory of its own: a plugin whose host runtime owns all
- * allocations and offers no workspace, code that runs while a stream capture
- * is in progress (where cudaMalloc is not allowed), or a serving loop whose
- * memory plan is fixed at start-up.  The source pages have no counterpart;
- * the operation and the arguments are those of moe_permute, minus `ws`.
+ * allocations and offers no workspace, or a serving loop whose memory plan
+ * is fixed at start-up and allows no allocation afterwards.  The source
+ * pages have no counterpart; the operation and the arguments are those of
+ * moe_permute, minus `ws`.
  *   Scratch (status word + per-block expert counts) lives in a 1 MiB + 256 B
  *   array of static device memory inside the library, which every GPU that
  *   loads the library keeps until the process exits.  Limit:
  *   ceil(T / 32) * E <= 262144 (e.g. T <= 32768 at E = 256, T <= 65536 at
- *   E = 128); larger calls return MOE_ERR_UNSUPPORTED before launching.
- *   The first call on a device looks up the array's device address (once per
- *   device, with that device current); make that first call before any
- *   stream capture begins.
+ *   E = 128) and T * (k + 1) <= 2^30; larger calls return
+ *   MOE_ERR_UNSUPPORTED before launching.
+ *   The first call in each CUDA context looks up the array's device address
+ *   in that context (with it current) and caches it under the context's
+ *   unique id, so a caller's own context, or the new primary context after
+ *   cudaDeviceReset, gets its own lookup.  Make the first call of a context
+ *   before any stream capture begins.
  *   All calls on a device share the one array and leave their contents
  *   there; each call clears the status word and rewrites every count it
  *   reads.  Calls whose kernels overlap on the GPU (e.g. on two streams)

@@ -89,6 +89,11 @@ def test_host_validation_rejects_bad_arguments(L):
     # E4M3 permute needs d % 128 == 0
     assert L.moe_permute(fake, 2, fake, 16, 200, 4, 2, 0, 3, fake, fake, fake, fake, fake, fake,
                          fake, 1 << 20, null) == -2
+    # permuted rows are int32 indices: T * (k + 1) > 2^30 is refused before any launch
+    assert L.moe_permute(fake, 2, fake, 1 << 27, 256, 16, 8, 0, 2, fake, null, fake, fake, fake, fake,
+                         fake, 1 << 40, null) == -2
+    assert L.moe_permute(fake, 2, fake, (1 << 29) - 1, 256, 16, 1, 0, 2, fake, null, fake, fake, fake, fake,
+                         fake, 8, null) == -3   # within the bound: the short workspace is what fails
     # grouped GEMM: K not a multiple of 64 / null offsets
     assert L.moe_grouped_gemm(fake, null, fake, null, fake, 4, 64, 256, 100, 2, 0, fake, 2, null,
                               fake, 256, null) == -2

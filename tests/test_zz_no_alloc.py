@@ -1,12 +1,12 @@
 """The allocation-free permute entry point (moe_permute_noalloc).
 
 It exists for callers that cannot give the library device memory of its own
--- a plugin whose host runtime owns every allocation, code running inside a
-stream capture where cudaMalloc is not allowed, a serving loop with a memory
-plan fixed at start-up -- so its scratch lives in static device memory of
-the library instead of a caller workspace.  These tests call it through the
-C ABI and check that two calls in a row (different shapes, so the second
-runs over scratch the first left behind) give exactly what moe_permute gives;
+-- a plugin whose host runtime owns every allocation, a serving loop with a
+memory plan fixed at start-up -- so its scratch lives in static device memory
+of the library instead of a caller workspace.  These tests call it through
+the C ABI and check that calls in a row (different shapes: the second covers
+more scratch than the first, the third runs inside what the second left
+behind) give exactly what moe_permute gives;
 the permutation plan and the permuted bytes are compared bit for bit, the
 tolerance every permute test uses.  This file is collected last so a run
 that stops at the first failure has run everything else already.
@@ -60,12 +60,13 @@ def _noalloc(x, idx, E, shared, fp8):
 
 
 CALLS = [  # T, E, k, d, x dtype, shared, fp8
-    (1000, 256, 8, 512, torch.bfloat16, True, True),
-    (300, 8, 2, 256, torch.float32, False, False),
+    (300, 8, 2, 256, torch.float32, False, False),     # 10 blocks x 8 experts of count words
+    (1000, 256, 8, 512, torch.bfloat16, True, True),   # 32 x 256: beyond what the first call wrote
+    (200, 64, 4, 384, torch.bfloat16, True, False),    # 7 x 64: over the second call's leftovers
 ]
 
 
-def test_two_calls_in_a_row_match_moe_permute():
+def test_calls_in_a_row_match_moe_permute():
     results = []
     for n, (T, E, k, d, xdt, shared, fp8) in enumerate(CALLS):
         x, idx = _inputs(T, E, k, d, xdt, seed=17 + n)
@@ -84,5 +85,9 @@ def test_rejects_sizes_beyond_the_static_scratch():
     fake = ctypes.c_void_p(0x10000)
     # ceil(65537 / 32) * 256 > 262144 count words
     st = gg.lib().moe_permute_noalloc(fake, gg.MOE_BF16, fake, 65537, 256, 256, 8, 0, gg.MOE_BF16, fake, None,
+                                      fake, fake, fake, fake, None)
+    assert st == -2
+    # permuted rows are int32 indices: T * (k + 1) > 2^30 is refused before anything runs
+    st = gg.lib().moe_permute_noalloc(fake, gg.MOE_BF16, fake, 1 << 27, 256, 1, 1, 0, gg.MOE_BF16, fake, None,
                                       fake, fake, fake, fake, None)
     assert st == -2
