@@ -7,8 +7,10 @@ One step = one whole layer forward (router, permute, up grouped GEMM with the
 SiLU gate, down grouped GEMM, combine) over the workload's T tokens.  The
 default workload is the Mixtral-shaped layer (T=4096, d=4096, E=8 top-2,
 I=14336, Zipf s=1.0 routing skew).  Inputs are seeded synthetic tensors
-resident in HBM; the L2 cache is flushed (a 2x-L2 buffer is rewritten)
-between timed steps, outside the timed events.  Each step is timed with CUDA
+resident in HBM; the L2 cache is flushed between timed steps, outside the
+timed events: a 2x-L2 buffer is rewritten and then read back, so the step
+starts with L2 holding only clean lines (no write-back of the flush's own
+dirty lines is charged to the step).  Each step is timed with CUDA
 events on the launching stream; with N > 1 (torchrun) every rank runs an
 independent replica of the layer on its own tokens (the layer has no
 exchange step on one node's data-parallel path), and the reported time is the
@@ -21,7 +23,12 @@ Printed: ONE JSON line (rank 0) with the contract keys plus
                and D2H of the output inside the timed region)
   cpu_baseline the fp64 oracle on a bounded token sample, on this host's cores
   clocks       SM clock / throttle reasons sampled during the timed region
-`--impl reference` times the oracle alone (the slow CPU reference arm).
+  workloads    (default run at N=1) the same measurement -- ms_per_step,
+               kernels, roofline, clocks, graph, e2e -- for the other layers
+               of the pages' workloads (fine-grained balanced / skewed, their
+               FP8 versions, decode) and the router microbenchmark
+`--impl reference` times the oracle alone (the slow CPU reference arm), on
+the same token batches the cpu_baseline leg uses.
 """
 from __future__ import annotations
 
@@ -85,16 +92,53 @@ def workload_desc(s) -> str:
     return ", ".join(parts)
 
 
+L2_NOTE = "flushed between timed steps (2x L2 buffer rewritten then read back, outside the events)"
+
+
 def config_block(s):
-    return {"workload": workload_desc(s), "tokens_per_step": s.T, "seed": 1234,
-            "l2": "flushed between timed steps (2x L2 buffer rewrite, outside the events)",
+    return {"workload": workload_desc(s), "tokens_per_step": s.T, "seed": 1234, "l2": L2_NOTE,
             "parallelism": "replicas (one independent layer per GPU)"}
+
+
+def host_cpu():
+    """The host's CPU model and core count (reported beside the CPU baseline)."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    try:
+        usable = len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        usable = os.cpu_count()
+    return {"cpu_model": model, "host_cores": os.cpu_count(), "usable_cores": usable}
+
+
+class Flusher:
+    """Evicts L2 between timed steps: a buffer of twice the L2 size is
+    rewritten and then summed, so what L2 holds afterwards is clean lines of
+    this buffer (the dirty ones were written back during the flush)."""
+
+    def __init__(self, dev):
+        l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+        n = max(2 * l2, 256 << 20) // 4
+        self.buf = torch.empty(n, dtype=torch.float32, device=dev)
+        self.sink = torch.empty((), dtype=torch.float32, device=dev)
+
+    def __call__(self):
+        self.buf.fill_(1.0)
+        torch.sum(self.buf, dim=0, out=self.sink)
 
 
 # --------------------------------------------------------------------------- clocks
 class ClockSampler:
     """SM clock and clock-event (throttle) reasons sampled every 10 ms through NVML
-    on a background thread while the timed region runs (nvidia-smi as fallback)."""
+    on a background thread while the timed region runs; without NVML the
+    summary says so instead of giving a number."""
 
     REASONS = {0x4: "sw_power_cap", 0x8: "hw_slowdown", 0x20: "sw_thermal_slowdown",
                0x40: "hw_thermal_slowdown", 0x80: "hw_power_brake_slowdown"}
@@ -296,58 +340,97 @@ def roofline(s, alg, kernels, peaks, peak_kind):
 
 
 class HostExperts:
-    """[e] -> host fp64 copy of expert e of a stacked device weight tensor (input staging, not timed)."""
+    """[e] -> host fp64 copy of expert e of a stacked device weight tensor.
 
-    def __init__(self, t):
-        self.t, self.cache = t, {}
+    With cache=True the copies are kept (staged once, outside the timed
+    oracle calls); with cache=False every access converts afresh, so host
+    memory holds one expert at a time (the fine-grained layers' 257 experts
+    would take ~90 GB as fp64) and the conversion counts as oracle time."""
+
+    def __init__(self, t, cache=True):
+        self.t, self.cache, self.keep = t, {}, cache
 
     def __getitem__(self, e):
         import oracle
         e = int(e)
+        if not self.keep:
+            return oracle.as_f64(self.t[e])
         if e not in self.cache:
             self.cache[e] = oracle.as_f64(self.t[e])
         return self.cache[e]
 
     def stage(self, experts):
-        for e in experts:
-            self[e]
+        if self.keep:
+            for e in experts:
+                self[e]
+
+
+HOST_CACHE_BYTES = 24 << 30  # fp64 expert copies the oracle legs may keep on the host
+
+
+def oracle_batch_tokens(s) -> int:
+    """Tokens per oracle batch: the CPU-baseline leg and the reference arm use the same batches."""
+    return min(s.T, 512)
+
+
+class OracleRunner:
+    """The fp64 oracle forward (routing, the selected experts, shared expert) on
+    seeded random token batches of the workload, timed on the host's cores."""
+
+    def __init__(self, s, inp, seed=7):
+        import oracle
+        self.oracle, self.s, self.inp = oracle, s, inp
+        expert_bytes = s.E * 3 * s.inter * s.d * 8
+        self.cached = expert_bytes <= HOST_CACHE_BYTES
+        self.W1 = HostExperts(inp["W1"], cache=self.cached)
+        self.W2 = HostExperts(inp["W2"], cache=self.cached)
+        self.W1s = oracle.as_f64(inp["W1s"]) if inp["W1s"] is not None else None
+        self.W2s = oracle.as_f64(inp["W2s"]) if inp["W2s"] is not None else None
+        self.rng = np.random.default_rng(seed)
+        self.batch = oracle_batch_tokens(s)
+
+    def step(self) -> float:
+        """One batch; returns the seconds spent in the oracle call itself."""
+        s, o = self.s, self.oracle
+        toks = np.sort(self.rng.choice(s.T, size=self.batch, replace=False))
+        xs = self.inp["x"][toks]
+        if self.cached:  # staging the weights is input preparation, not oracle work
+            need = np.unique(o.route(xs, self.inp["W_r"], self.inp["bias"], s.k)["idx"])
+            self.W1.stage(need)
+            self.W2.stage(need)
+        fwd = o.moe_forward_fp8 if s.fp8 else o.moe_forward
+        t0 = time.perf_counter()
+        fwd(xs, self.inp["W_r"], self.inp["bias"], self.W1, self.W2, self.W1s, self.W2s, k=s.k,
+            renormalize=s.renormalize)
+        return time.perf_counter() - t0
+
+    def describe(self, batches, spent) -> str:
+        how = ("expert weights staged to host fp64 outside the timed calls" if self.cached else
+               "expert weights converted to fp64 inside the timed calls, one expert at a time")
+        return (f"fp64 numpy oracle forward (routing, selected experts, shared) on {batches} batch(es) of "
+                f"{self.batch} random tokens of {self.s.T}, {spent:.1f} s; {how}")
+
+
+def blas_threads() -> int:
+    from threadpoolctl import threadpool_info
+    return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
 
 
 def cpu_baseline(s, inp, budget_s=12.0):
-    """The oracle forward on doubling token samples until ~budget_s of CPU time; tokens/s."""
-    import oracle
-    from threadpoolctl import threadpool_info
-
-    rng = np.random.default_rng(7)
-    W1, W2 = HostExperts(inp["W1"]), HostExperts(inp["W2"])
-    W1s = oracle.as_f64(inp["W1s"]) if inp["W1s"] is not None else None
-    W2s = oracle.as_f64(inp["W2s"]) if inp["W2s"] is not None else None
-    n, done_tokens, spent = 16, 0, 0.0
-    while spent < budget_s and n <= s.T:
-        toks = np.sort(rng.choice(s.T, size=n, replace=False))
-        xs = inp["x"][toks]
-        need = np.unique(oracle.route(xs, inp["W_r"], inp["bias"], s.k)["idx"])
-        W1.stage(need)
-        W2.stage(need)
-        t0 = time.perf_counter()
-        fwd = oracle.moe_forward_fp8 if s.fp8 else oracle.moe_forward
-        fwd(xs, inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k, renormalize=s.renormalize)
-        spent += time.perf_counter() - t0
-        done_tokens += n
-        n *= 2
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-    return {"value": round(done_tokens / spent, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-            "sample": f"fp64 numpy oracle forward (routing, selected experts, shared) of {done_tokens} of {s.T} "
-                      f"tokens in doubling batches from 16, {spent:.1f} s; expert weights staged to host "
-                      f"fp64 before each timed batch"}
+    """The oracle on the reference arm's token batches until ~budget_s of CPU time; tokens/s."""
+    r = OracleRunner(s, inp)
+    batches, spent = 0, 0.0
+    while spent < budget_s and batches < 64:
+        spent += r.step()
+        batches += 1
+    return {"value": round(batches * r.batch / spent, 3), "unit": "tokens/s", "cores": blas_threads(),
+            "kind": "oracle", "sample": r.describe(batches, spent), **host_cpu()}
 
 
-def run_ours(args, rank, world, dev):
-    gg = build_lib()
-    s = shape_of(args.config, **args.overrides)
-    torch.cuda.set_device(dev)
-    stream = torch.cuda.current_stream()
-    inp = make_inputs(s, seed=1234 + rank, device=dev)
+# --------------------------------------------------------------------------- one workload
+def prepare(gg, s, dev, seed):
+    """Device inputs, weights (quantised for FP8 layers, outside any timing), outputs, workspace."""
+    inp = make_inputs(s, seed=seed, device=dev)
     cfg = make_cfg(gg, s)
     ws = torch.empty(gg.workspace_size(cfg) + gg.host_staging_size(cfg), dtype=torch.uint8, device=dev)
     if s.fp8:  # weights quantised once per 128x128 block (offline, outside the timed region)
@@ -361,56 +444,60 @@ def run_ours(args, rank, world, dev):
         weights = gg.ExpertWeights(W1=inp["W1"], W2=inp["W2"], W1s=inp["W1s"], W2s=inp["W2s"])
     out = torch.empty((s.T, s.d), dtype=torch.bfloat16 if s.x_dtype != "f32" else torch.float32, device=dev)
     counts = torch.empty(s.E, dtype=torch.int32, device=dev)
-    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
-    scrub = torch.empty(max(2 * l2, 256 << 20), dtype=torch.uint8, device=dev)
+    return inp, cfg, ws, weights, out, counts
 
-    def flush():
-        scrub.fill_(1)
+
+def measure_layer(gg, s, steps, warmup, world, dev, flush, seed, graph=True, e2e=True):
+    """Times one workload's forward: the headline steps, the CUDA-graph replay,
+    the host-buffer entry point and the per-kernel breakdown."""
+    stream = torch.cuda.current_stream()
+    inp, cfg, ws, weights, out, counts = prepare(gg, s, dev, seed)
 
     def step():
         gg.moe_forward(cfg, inp["x"], inp["W_r"], inp["bias"], weights, out=out, counts_out=counts, ws=ws)
 
-    # --- headline: K timed forwards
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize()
     with ClockSampler(dev) as clk:
-        times = time_steps(step, args.steps, args.warmup, flush, stream)
+        times = time_steps(step, steps, warmup, flush, stream)
         torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     status = gg.read_device_status(ws)
     if status != 0:
-        raise RuntimeError(f"device status {status}")
-    ms = max_over_ranks(float(np.mean(times)), world, dev)
+        raise RuntimeError(f"{s.name}: device status {status}")
+    r = dict(ms=max_over_ranks(float(np.mean(times)), world, dev), clocks=clk.summary())
 
-    # --- the same forward replayed from a CUDA graph (one launch of the whole layer)
-    gstream = torch.cuda.Stream()
-    gstream.wait_stream(stream)
-    graph = torch.cuda.CUDAGraph()
-    with torch.cuda.stream(gstream):
-        step()  # warm the capture stream
-        with torch.cuda.graph(graph, stream=gstream):
-            step()
-    stream.wait_stream(gstream)
-    torch.cuda.synchronize()
-    graph_times = time_steps(graph.replay, max(3, args.steps // 2), 3, flush, stream)
-    graph_ms = max_over_ranks(float(np.mean(graph_times)), world, dev)
-    del graph
+    if graph:  # the same forward replayed from a CUDA graph (one launch of the whole layer)
+        gstream = torch.cuda.Stream()
+        gstream.wait_stream(stream)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.stream(gstream):
+            step()  # warm the capture stream
+            with torch.cuda.graph(g, stream=gstream):
+                step()
+        stream.wait_stream(gstream)
+        torch.cuda.synchronize()
+        gt = time_steps(g.replay, max(3, steps // 2), 3, flush, stream)
+        r["graph_ms"] = max_over_ranks(float(np.mean(gt)), world, dev)
+        del g
 
-    # --- e2e: host buffers through moe_forward_host, copies inside the timed region
-    xh = inp["x"].cpu().pin_memory()
-    oh = torch.empty((s.T, s.d), dtype=out.dtype).pin_memory()
+    if e2e:  # host buffers through moe_forward_host, copies inside the timed region
+        xh = inp["x"].cpu().pin_memory()
+        oh = torch.empty((s.T, s.d), dtype=out.dtype).pin_memory()
 
-    def step_host():
-        gg.moe_forward_host(cfg, xh, inp["W_r"], inp["bias"], weights, oh, ws)
+        def step_host():
+            gg.moe_forward_host(cfg, xh, inp["W_r"], inp["bias"], weights, oh, ws)
 
-    e2e_times = time_steps(step_host, max(3, args.steps // 2), 2, flush, stream, hold=False)
-    e2e_ms = max_over_ranks(float(np.mean(e2e_times)), world, dev)
+        et = time_steps(step_host, max(3, steps // 2), 2, flush, stream, hold=False)
+        r["e2e_ms"] = max_over_ranks(float(np.mean(et)), world, dev)
+        r["h2d"] = xh.numel() * xh.element_size()
+        r["d2h"] = oh.numel() * oh.element_size()
 
-    # --- per-kernel breakdown: the same forward with an event between its kernels
-    kt = time_marked(gg, cfg, inp, weights, out, counts, ws, max(3, args.steps // 2), flush, stream)
-    alg = algorithmic(s, counts.cpu().numpy())
+    kt = time_marked(gg, cfg, inp, weights, out, counts, ws, max(3, steps // 2), flush, stream)
+    c = counts.cpu().numpy()
+    alg = algorithmic(s, c)
     kern = {}
     for name, t_ms in kt.items():
         a = alg[name]
@@ -419,8 +506,37 @@ def run_ours(args, rank, world, dev):
             e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
         e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
         kern[name] = e
-    return dict(ms=ms, e2e_ms=e2e_ms, graph_ms=graph_ms, kernels=kern, clocks=clk.summary(), inp=inp, s=s, counts=counts.cpu().numpy(),
-                out_dtype=out.dtype)
+    r.update(kernels=kern, counts=c, alg=alg, inp=inp)
+    return r
+
+
+def layer_report(s, r, peaks, peak_kind, world):
+    """The per-workload part of the JSON line."""
+    T = s.T
+    roof = roofline(s, r["alg"], r["kernels"], peaks, peak_kind)
+    gemm_us = r["kernels"]["up_gemm"]["us"] + r["kernels"]["down_gemm"]["us"]
+    gemm_tf = s.gemm_flops() / (gemm_us * 1e-6) / 1e12
+    tensor_peak = float(peaks["bf16_tflops"]) * (2.0 if s.fp8 else 1.0)
+    c = r["counts"]
+    rep = {"workload": workload_desc(s), "tokens_per_step": T, "dtype": "e4m3" if s.fp8 else "bf16",
+           "ms_per_step": round(r["ms"], 4), "value": round(job_tokens_per_s(T, world, r["ms"]), 1),
+           "unit": "tokens/s",
+           # grouped-GEMM FLOP over the two GEMM kernels' own time, against the dense tensor peak
+           "gemm_tflops": round(gemm_tf, 1), "gemm_frac_of_peak": round(gemm_tf / tensor_peak, 4),
+           "roofline": roof, "kernels": r["kernels"], "clocks": r["clocks"],
+           "expert_counts": {"min": int(c.min()), "max": int(c.max()), "mean": float(c.mean()),
+                             "zeros": int((c == 0).sum())}}
+    if "graph_ms" in r:
+        rep["graph"] = {"ms_per_step": round(r["graph_ms"], 4),
+                        "value": round(job_tokens_per_s(T, world, r["graph_ms"]), 1), "unit": "tokens/s",
+                        "note": "the same forward captured once in a CUDA graph and replayed"}
+    if "e2e_ms" in r:
+        rep["e2e"] = {"value": round(job_tokens_per_s(T, world, r["e2e_ms"]), 1), "unit": "tokens/s",
+                      "h2d_bytes_per_step": r["h2d"], "d2h_bytes_per_step": r["d2h"]}
+    return rep
+
+
+SIDE_WORKLOADS = ("fine", "fine_skew", "fine_fp8", "fine_fp8_skew", "decode", "tiny")
 
 
 def main():
@@ -431,6 +547,9 @@ def main():
     ap.add_argument("--config", default="mixtral", choices=sorted(CONFIGS) + ["router_micro"])
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--workloads", default="auto",
+                    help="'auto' (the other layers and the router microbenchmark, with the default "
+                         "config at N=1), 'none', or a comma list of workload names")
     ap.add_argument("--set", default="", help="shape overrides for profiling runs, e.g. E=32,T=512")
     args = ap.parse_args()
     args.overrides = {}
@@ -448,63 +567,55 @@ def main():
         if rank != 0:  # the CPU reference arm runs on rank 0 only
             return 0
         if args.config == "router_micro":
-            return run_router_micro(args, rank, world, local)
+            return run_router_micro_reference(args, world)
         return run_reference(args, shape_of(args.config, **args.overrides), world)
 
     if world > 1:
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                              device_id=torch.device("cuda", local))
-    if args.config == "router_micro":
-        rc = run_router_micro(args, rank, world, local)
-        if world > 1:
-            torch.distributed.barrier()
-            torch.distributed.destroy_process_group()
-        return rc
-    s = shape_of(args.config, **args.overrides)
-    r = run_ours(args, rank, world, local)
+    gg = build_lib()
+    torch.cuda.set_device(local)
+    flush = Flusher(local)
     peaks, peak_kind = load_peaks()
-    result = None
-    if rank == 0:
-        T = s.T
-        value = job_tokens_per_s(T, world, r["ms"])
-        alg = algorithmic(s, r["counts"])
-        roof = roofline(s, alg, r["kernels"], peaks, peak_kind)
-        gemm_flops = s.gemm_flops()
-        gemm_us = r["kernels"]["up_gemm"]["us"] + r["kernels"]["down_gemm"]["us"]
-        gemm_tf = gemm_flops / (gemm_us * 1e-6) / 1e12
-        tensor_peak = float(peaks["bf16_tflops"]) * (2.0 if s.fp8 else 1.0)
+    if args.config == "router_micro":
+        m = measure_router_micro(gg, args.steps, args.warmup, world, rank, local, flush, args.overrides)
+        result = router_micro_line(m, args, world, peaks, peak_kind)
+    else:
+        s = shape_of(args.config, **args.overrides)
+        r = measure_layer(gg, s, args.steps, args.warmup, world, local, flush, seed=1234 + rank)
+        rep = layer_report(s, r, peaks, peak_kind, world)
         result = {
-            "metric": METRIC,
-            "value": round(value, 1),
-            "unit": "tokens/s",
-            "n_gpus": world,
-            "steps": args.steps,
-            "warmup": args.warmup,
-            "ms_per_step": round(r["ms"], 4),
-            "higher_is_better": True,
-            "scaling": "weak",
-            "vs_baseline": None,
-            "dtype": "e4m3" if s.fp8 else "bf16",
-            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)",
-            "config": config_block(s),
-            # grouped-GEMM FLOP over the two GEMM kernels' own time, against the dense tensor peak
-            "gemm_tflops": round(gemm_tf, 1),
-            "gemm_frac_of_peak": round(gemm_tf / tensor_peak, 4),
-            "roofline": roof,
-            "kernels": r["kernels"],
-            "e2e": {"value": round(job_tokens_per_s(T, world, r["e2e_ms"]), 1), "unit": "tokens/s",
-                    "h2d_bytes_per_step": T * s.d * (4 if s.x_dtype == "f32" else 2),
-                    "d2h_bytes_per_step": T * s.d * (4 if r["out_dtype"] == torch.float32 else 2)},
-            "graph": {"ms_per_step": round(r["graph_ms"], 4),
-                      "value": round(job_tokens_per_s(T, world, r["graph_ms"]), 1), "unit": "tokens/s",
-                      "note": "the same forward captured once in a CUDA graph and replayed"},
-            "gpu_launches": KERNELS_PER_FORWARD * args.steps,
-            "clocks": r["clocks"],
-            "expert_counts": {"min": int(r["counts"].min()), "max": int(r["counts"].max()),
-                              "mean": float(r["counts"].mean()), "zeros": int((r["counts"] == 0).sum())},
-        }
-        if world == 1 and not args.no_cpu_baseline:
+            "metric": METRIC, "value": rep["value"], "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": rep["ms_per_step"],
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rep["dtype"],
+            "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)", "config": config_block(s),
+            "gemm_tflops": rep["gemm_tflops"], "gemm_frac_of_peak": rep["gemm_frac_of_peak"],
+            "roofline": rep["roofline"], "kernels": rep["kernels"], "e2e": rep["e2e"], "graph": rep["graph"],
+            "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": rep["clocks"],
+            "expert_counts": rep["expert_counts"]}
+        if rank == 0 and world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(s, r["inp"])
+        del r
+        torch.cuda.empty_cache()
+        names = []
+        if args.workloads == "auto":
+            if world == 1 and args.config == "mixtral" and not args.overrides:
+                names = list(SIDE_WORKLOADS) + ["router_micro"]
+        elif args.workloads != "none":
+            names = [n for n in args.workloads.split(",") if n]
+        side = {}
+        for name in names:  # the other workloads, one after the other, each measured the same way
+            if name == "router_micro":
+                m = measure_router_micro(gg, args.steps, args.warmup, world, rank, local, flush, {})
+                side[name] = router_micro_line(m, args, world, peaks, peak_kind, compact=True)
+                continue
+            ws_ = shape_of(name)
+            rr = measure_layer(gg, ws_, args.steps, args.warmup, world, local, flush, seed=1234 + rank)
+            side[name] = layer_report(ws_, rr, peaks, peak_kind, world)
+            del rr
+            torch.cuda.empty_cache()
+        if side:
+            result["workloads"] = side
     if world > 1:
         torch.distributed.barrier()
         torch.distributed.destroy_process_group()
@@ -513,54 +624,23 @@ def main():
     return 0
 
 
-def run_router_micro(args, rank, world, local):
-    """Router-only microbenchmark: softmax + top-k of N fp16 logits rows (moe_topk_logits)."""
-    N, E, k = (args.overrides.get(key, ROUTER_MICRO[key]) for key in ("N", "E", "k"))
-    desc = {"workload": f"router_micro: N={N} tokens, E={E} experts, top-{k}, fp16 logits ~ N(0,1)",
-            "tokens_per_step": N, "seed": 1234,
-            "l2": "flushed between timed steps (2x L2 buffer rewrite, outside the events)"}
-    bytes_per_step = N * E * 2 + N * k * 8
-    if args.impl == "reference":
-        if rank != 0:
-            return 0
-        import oracle
-        from threadpoolctl import threadpool_info
-        logits = make_router_logits(N, E, seed=1234, device="cpu")
-        lf = oracle.as_f64(logits)
-        per_step = min(N, 4096)
-        rng = np.random.default_rng(3)
+# --------------------------------------------------------------------------- router microbenchmark
+def router_micro_shape(overrides):
+    return tuple(overrides.get(key, ROUTER_MICRO[key]) for key in ("N", "E", "k"))
 
-        def step():
-            rows = rng.choice(N, size=per_step, replace=False)
-            oracle.gate_weights(oracle.softmax(lf[rows]), oracle.topk_select(lf[rows], k))
 
-        for _ in range(args.warmup):
-            step()
-        t0 = time.perf_counter()
-        for _ in range(args.steps):
-            step()
-        dt = time.perf_counter() - t0
-        value = args.steps * per_step / dt
-        threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
-        print(json.dumps({"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
-                          "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                          "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
-                          "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-                          "config": desc,
-                          "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": threads,
-                                           "kind": "oracle", "sample": f"{per_step} random rows of {N} per step"},
-                          "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
-                                  "d2h_bytes_per_step": 0}}), flush=True)
-        return 0
-    gg = build_lib()
-    dev = local
-    torch.cuda.set_device(dev)
+def router_micro_desc(N, E, k):
+    return {"workload": f"router_micro: N={N} tokens, E={E} experts, top-{k}, fp16 logits ~ N(0,1)",
+            "tokens_per_step": N, "seed": 1234, "l2": L2_NOTE}
+
+
+def measure_router_micro(gg, steps, warmup, world, rank, dev, flush, overrides):
+    """Softmax + top-k of N fp16 logits rows (moe_topk_logits), device-resident and host-buffered."""
+    N, E, k = router_micro_shape(overrides)
     stream = torch.cuda.current_stream()
     logits = make_router_logits(N, E, seed=1234 + rank, device=dev)
     idx = torch.empty((N, k), dtype=torch.int32, device=dev)
     w = torch.empty((N, k), dtype=torch.float32, device=dev)
-    scrub = torch.empty(max(2 * torch.cuda.get_device_properties(dev).L2_cache_size, 256 << 20), dtype=torch.uint8,
-                        device=dev)
 
     def step():
         gg.topk_logits(logits, k, out_idx=idx, out_w=w)
@@ -568,7 +648,7 @@ def run_router_micro(args, rank, world, local):
     if world > 1:
         torch.distributed.barrier()
     with ClockSampler(dev) as clk:
-        times = time_steps(step, args.steps, args.warmup, lambda: scrub.fill_(1), stream)
+        times = time_steps(step, steps, warmup, flush, stream)
     ms = max_over_ranks(float(np.mean(times)), world, dev)
     lh = logits.cpu().pin_memory()
     ih = torch.empty((N, k), dtype=torch.int32).pin_memory()
@@ -580,42 +660,46 @@ def run_router_micro(args, rank, world, local):
         ih.copy_(idx, non_blocking=True)
         wh.copy_(w, non_blocking=True)
 
-    e2e_ms = max_over_ranks(float(np.mean(time_steps(step_host, max(3, args.steps // 2), 2,
-                                                     lambda: scrub.fill_(1), stream, hold=False))), world, dev)
-    peaks, kind = load_peaks()
+    e2e_ms = max_over_ranks(float(np.mean(time_steps(step_host, max(3, steps // 2), 2, flush, stream,
+                                                     hold=False))), world, dev)
+    return dict(N=N, E=E, k=k, ms=ms, e2e_ms=e2e_ms, clocks=clk.summary())
+
+
+def router_micro_line(m, args, world, peaks, peak_kind, compact=False):
+    N, E, k, ms = m["N"], m["E"], m["k"], m["ms"]
+    bytes_per_step = N * E * 2 + N * k * 8
     achieved = bytes_per_step / (ms * 1e-3) / 1e9
-    result = {"metric": METRIC, "value": round(job_tokens_per_s(N, world, ms), 1), "unit": "tokens/s", "n_gpus": world,
-              "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5), "higher_is_better": True,
-              "scaling": "weak", "vs_baseline": None, "dtype": "f16", "data": "synthetic", "config": desc,
-              "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": float(peaks["hbm_gbs"]),
-                           "unit": "GB/s", "frac": round(achieved / float(peaks["hbm_gbs"]), 4), "traffic": None,
-                           "kernel": "finish_kernel (softmax + top-k of stored logits)",
-                           "peak_kind": f"{kind} HBM copy bandwidth"},
-              "kernel_us": round(ms * 1e3, 2),
-              "e2e": {"value": round(job_tokens_per_s(N, world, e2e_ms), 1), "unit": "tokens/s",
-                      "h2d_bytes_per_step": N * E * 2, "d2h_bytes_per_step": N * k * 8},
-              "gpu_launches": args.steps, "clocks": clk.summary()}
-    if rank == 0:
-        print(json.dumps(result), flush=True)
-    return 0
+    hbm = float(peaks["hbm_gbs"])
+    roof = {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+            "frac": round(achieved / hbm, 4), "traffic": None,
+            "kernel": "softmax + top-k of stored logits", "peak_kind": f"{peak_kind} HBM copy bandwidth",
+            "algorithmic": {"bytes": bytes_per_step}}
+    e2e = {"value": round(job_tokens_per_s(N, world, m["e2e_ms"]), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": N * E * 2, "d2h_bytes_per_step": N * k * 8}
+    if compact:
+        return {"workload": router_micro_desc(N, E, k)["workload"], "tokens_per_step": N, "dtype": "f16",
+                "ms_per_step": round(ms, 5), "value": round(job_tokens_per_s(N, world, ms), 1),
+                "unit": "tokens/s", "kernel_us": round(ms * 1e3, 2), "roofline": roof, "e2e": e2e,
+                "clocks": m["clocks"]}
+    return {"metric": METRIC, "value": round(job_tokens_per_s(N, world, ms), 1), "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms, 5),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f16",
+            "data": "synthetic", "config": router_micro_desc(N, E, k), "roofline": roof,
+            "kernel_us": round(ms * 1e3, 2), "e2e": e2e, "gpu_launches": args.steps, "clocks": m["clocks"]}
 
 
-def run_reference(args, s, world):
-    """The oracle (fp64, host cores) on a bounded token sample per step, as the slow reference arm."""
+def run_router_micro_reference(args, world):
+    """The oracle's softmax + top-k on bounded row samples of the microbenchmark's logits."""
     import oracle
-    from threadpoolctl import threadpool_info
-
-    inp = make_inputs(s, seed=1234, device="cuda" if torch.cuda.is_available() else "cpu")
-    W1, W2 = HostExperts(inp["W1"]), HostExperts(inp["W2"])
-    W1s = oracle.as_f64(inp["W1s"]) if inp["W1s"] is not None else None
-    W2s = oracle.as_f64(inp["W2s"]) if inp["W2s"] is not None else None
+    N, E, k = router_micro_shape(args.overrides)
+    logits = make_router_logits(N, E, seed=1234, device="cpu")
+    lf = oracle.as_f64(logits)
+    per_step = min(N, 4096)
     rng = np.random.default_rng(3)
-    per_step = 8
 
     def step():
-        toks = np.sort(rng.choice(s.T, size=per_step, replace=False))
-        fwd = oracle.moe_forward_fp8 if s.fp8 else oracle.moe_forward
-        fwd(inp["x"][toks], inp["W_r"], inp["bias"], W1, W2, W1s, W2s, k=s.k, renormalize=s.renormalize)
+        rows = rng.choice(N, size=per_step, replace=False)
+        oracle.gate_weights(oracle.softmax(lf[rows]), oracle.topk_select(lf[rows], k))
 
     for _ in range(args.warmup):
         step()
@@ -624,13 +708,34 @@ def run_reference(args, s, world):
         step()
     dt = time.perf_counter() - t0
     value = args.steps * per_step / dt
-    threads = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    print(json.dumps({"impl": "reference", "metric": METRIC, "value": round(value, 1), "unit": "tokens/s",
+                      "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                      "ms_per_step": round(dt / args.steps * 1e3, 3), "higher_is_better": True,
+                      "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+                      "config": router_micro_desc(N, E, k),
+                      "cpu_baseline": {"value": round(value, 1), "unit": "tokens/s", "cores": blas_threads(),
+                                       "kind": "oracle", "sample": f"{per_step} random rows of {N} per step",
+                                       **host_cpu()},
+                      "e2e": {"value": round(value, 1), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                              "d2h_bytes_per_step": 0}}), flush=True)
+    return 0
+
+
+def run_reference(args, s, world):
+    """The oracle (fp64, host cores) as the slow reference arm: each step is one
+    of the cpu_baseline leg's token batches of the same workload."""
+    inp = make_inputs(s, seed=1234, device="cuda" if torch.cuda.is_available() else "cpu")
+    r = OracleRunner(s, inp)
+    for _ in range(args.warmup):
+        r.step()
+    spent = sum(r.step() for _ in range(args.steps))
+    value = args.steps * r.batch / spent
     line = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
             "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-            "ms_per_step": round(dt / args.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
+            "ms_per_step": round(spent / args.steps * 1e3, 2), "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": config_block(s),
-            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": threads, "kind": "oracle",
-                             "sample": f"{per_step} random tokens of {s.T} per step (fp64 oracle forward)"},
+            "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": blas_threads(),
+                             "kind": "oracle", "sample": r.describe(args.steps, spent), **host_cpu()},
             "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0

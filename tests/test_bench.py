@@ -101,3 +101,25 @@ def test_committed_traffic_figures_are_consistent():
         assert stage in bench.STAGE_SOURCES
         assert e["bytes_per_launch"] == e["dram_bytes_read"] + e["dram_bytes_write"]
         assert len(e["source_sha256"]) == 64 and e["command"].startswith("ncu ")
+
+
+def test_reference_arm_times_the_oracle_on_the_cpu_baseline_batches():
+    import subprocess
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "tiny",
+                        "--steps", "2", "--warmup", "3"], capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-2000:]
+    line = json.loads(r.stdout.strip().splitlines()[-1])
+    assert line["impl"] == "reference" and line["unit"] == "tokens/s" and line["value"] > 0
+    cb = line["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["host_cores"] >= 1 and cb["cpu_model"]
+    # the same batches as the cpu_baseline leg: oracle_batch_tokens of the workload
+    assert f"batch(es) of {bench.oracle_batch_tokens(shape_of('tiny'))} random tokens" in cb["sample"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["value"] == line["value"]
+
+
+def test_oracle_batches_are_bounded():
+    assert bench.oracle_batch_tokens(shape_of("mixtral")) == 512
+    assert bench.oracle_batch_tokens(shape_of("decode")) == 128
+    # fine-grained experts do not fit the host cache as fp64: converted one at a time
+    assert 256 * 3 * 2048 * 7168 * 8 > bench.HOST_CACHE_BYTES
+    assert 8 * 3 * 14336 * 4096 * 8 <= bench.HOST_CACHE_BYTES
