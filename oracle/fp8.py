@@ -28,7 +28,7 @@ from .moe_oracle import as_f64, bf16_round, route
 __all__ = [
     "E4M3_MAX", "e4m3_magnitudes", "e4m3_decode", "e4m3_encode", "quantize_1x128",
     "quantize_128x128", "dequantize_1x128", "dequantize_128x128", "fp8_gemm",
-    "swiglu_ffn_fp8", "moe_forward_fp8",
+    "swiglu_ffn_fp8", "quantize_expert", "moe_forward_fp8",
 ]
 
 E4M3_MAX = 448.0
@@ -137,12 +137,25 @@ def swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2) -> dict:
     return dict(h=h, hq=hq, sh=sh, y=fp8_gemm(hq, sh, W2q, s2))
 
 
+def quantize_expert(W1e, W2e) -> tuple:
+    """One expert's weights (bf16 values) quantised per 128x128 block: (W1q, s1, W2q, s2)."""
+    W1q, s1 = quantize_128x128(as_f64(W1e))
+    W2q, s2 = quantize_128x128(as_f64(W2e))
+    return W1q, s1, W2q, s2
+
+
 def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
-                    renormalize: bool = False, tokens=None, idx=None, w=None) -> dict:
+                    renormalize: bool = False, tokens=None, idx=None, w=None,
+                    quantized=None, workers: int = 1) -> dict:
     """FP8 variant of oracle.moe_forward: same routing, quantised expert GEMMs.
 
     Each expert's W1[e] / W2[e] (bf16 values) is quantised per 128x128 block;
-    x (as bf16) per token per 128 columns.
+    x (as bf16) per token per 128 columns.  `quantized`, when given, maps an
+    expert id to its quantize_expert() result (computed once, e.g. for two
+    workloads with the same weights).  With workers > 1 the experts are
+    evaluated on that many threads; each expert's rows are computed exactly as
+    with one thread and the weighted outputs are still added in ascending
+    expert order, so the result does not depend on `workers`.
     """
     xs = x if tokens is None else x[tokens]
     r = route(xs, W_r, bias, k, renormalize)
@@ -155,14 +168,23 @@ def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
     xq, sx = quantize_1x128(xe)
     out = np.zeros(xe.shape, dtype=np.float64)
     if W1s is not None:
-        W1q, s1 = quantize_128x128(as_f64(W1s))
-        W2q, s2 = quantize_128x128(as_f64(W2s))
+        W1q, s1, W2q, s2 = quantize_expert(W1s, W2s)
         out += swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)["y"]
-    for e in np.unique(sel):
+
+    def expert_rows(e):
         t_rows, slots = np.nonzero(sel == e)
-        W1q, s1 = quantize_128x128(as_f64(W1[int(e)]))
-        W2q, s2 = quantize_128x128(as_f64(W2[int(e)]))
-        y = swiglu_ffn_fp8(xq[t_rows], sx[t_rows], W1q, s1, W2q, s2)["y"]
-        out[t_rows] += wts[t_rows, slots][:, None] * y
+        q = quantized[int(e)] if quantized is not None else quantize_expert(W1[int(e)], W2[int(e)])
+        y = swiglu_ffn_fp8(xq[t_rows], sx[t_rows], *q)["y"]
+        return t_rows, wts[t_rows, slots][:, None] * y
+
+    experts = np.unique(sel)
+    if workers > 1:
+        from concurrent.futures import ThreadPoolExecutor
+        with ThreadPoolExecutor(workers) as ex:
+            parts = list(ex.map(expert_rows, experts))
+    else:
+        parts = [expert_rows(e) for e in experts]
+    for t_rows, contrib in parts:   # ascending expert order
+        out[t_rows] += contrib
     r.update(out=out, xq=xq, sx=sx)
     return r

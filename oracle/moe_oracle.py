@@ -38,7 +38,7 @@ import numpy as np
 __all__ = [
     "as_f64", "bf16_round", "router_logits", "softmax", "topk_select", "gate_weights",
     "route", "expert_counts", "expert_offsets", "permutation", "swiglu_ffn",
-    "moe_forward", "imbalance",
+    "moe_forward", "imbalance", "capacity_from_factor", "kept_mask",
 ]
 
 
@@ -156,32 +156,71 @@ def expert_offsets(counts, shared_rows: int = 0) -> np.ndarray:
     return offsets
 
 
-def permutation(idx, E: int, shared: bool = False) -> dict:
+def capacity_from_factor(factor: float, T: int, k: int, E: int) -> int:
+    """Rows one expert may take: ceil(factor * T * k / E), the factor times an
+    even share of the T*k routed rows ([GroupedTP] §5.1 caps each expert's
+    tokens at inference by a capacity factor; [DSMoE] §3.2 bounds the share
+    of a forward's tokens one expert may take)."""
+    import math
+    return max(1, math.ceil(factor * T * k / E))
+
+
+def kept_mask(idx, capacity: int = 0) -> np.ndarray:
+    """kept[t, j]: whether pair (t, j) is within its expert's capacity.
+
+    An expert keeps its first `capacity` pairs in ascending token order (the
+    order of its segment); the rest overflow.  capacity <= 0 keeps all.
+    """
+    idx = np.asarray(idx)
+    T, k = idx.shape
+    kept = np.ones((T, k), dtype=bool)
+    if capacity <= 0:
+        return kept
+    seen = {}
+    for t in range(T):
+        for j in range(k):
+            e = int(idx[t, j])
+            seen[e] = seen.get(e, 0) + 1
+            kept[t, j] = seen[e] <= capacity
+    return kept
+
+
+def permutation(idx, E: int, shared: bool = False, capacity: int = 0) -> dict:
     """Scatter plan of the expert-contiguous buffer.
 
     Within expert e's segment rows follow ascending token id, so the rank of
     token t in expert e is #{t' < t : e in sel(t')}.  Returns counts, offsets,
     row_to_token [R(+T)] and token_to_row [T, k].
+
+    With capacity > 0 an expert keeps only its first `capacity` rows (pairs
+    of rank >= capacity overflow: token_to_row = -1, no row); counts are the
+    kept rows, offsets their exclusive scan, and the shared expert's rows
+    follow the kept rows (offsets[E] .. offsets[E] + T - 1).  Rows past the
+    last used one are unused (row_to_token = -1).
     """
     idx = np.asarray(idx)
     T, k = idx.shape
-    counts = expert_counts(idx, E)
+    kept = kept_mask(idx, capacity)
+    counts = expert_counts(idx[kept], E)
     offsets = expert_offsets(counts, T if shared else 0)
     R = T * k
+    used = int(offsets[E])
     row_to_token = np.full(R + (T if shared else 0), -1, dtype=np.int64)
-    token_to_row = np.empty((T, k), dtype=np.int64)
+    token_to_row = np.full((T, k), -1, dtype=np.int64)
     filled = np.zeros(E, dtype=np.int64)
     for t in range(T):
         for j in range(k):
+            if not kept[t, j]:
+                continue
             e = idx[t, j]
             row = offsets[e] + filled[e]
             filled[e] += 1
             token_to_row[t, j] = row
             row_to_token[row] = t
     if shared:
-        row_to_token[R:] = np.arange(T)
+        row_to_token[used:used + T] = np.arange(T)
     return dict(counts=counts, offsets=offsets, row_to_token=row_to_token,
-                token_to_row=token_to_row)
+                token_to_row=token_to_row, kept=kept)
 
 
 def imbalance(counts) -> float:
@@ -206,28 +245,38 @@ def swiglu_ffn(xrows, W1e, W2e) -> np.ndarray:
 
 
 def moe_forward(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
-                renormalize: bool = False, tokens=None, idx=None, w=None) -> dict:
-    """out[t] = E_shared(x_t) + sum_{j<k} w[t, j] * E_{idx[t, j]}(x_t).
+                renormalize: bool = False, tokens=None, idx=None, w=None, capacity: int = 0) -> dict:
+    """out[t] = E_shared(x_t) + sum_{j<k, kept} w[t, j] * E_{idx[t, j]}(x_t).
 
     W1 / W2 may be any object indexable by expert id (W1[e] -> [2I, d],
     W2[e] -> [d, I]); only the experts some token selects are touched.
     `tokens` restricts the computation to those token ids (routing included).
     `idx` / `w`, when given (shape [len(tokens), k]), replace this oracle's
     own routing (used where the caller adopts another router's choice at a
-    near tie).
+    near tie).  With capacity > 0 each expert takes only its first
+    `capacity` pairs in token order (kept_mask); an overflowing pair adds
+    nothing: its token keeps the shared expert and its other experts, with
+    their gate weights unchanged (the pages' "fallback path" for tokens over
+    capacity is the shared expert / residual the layer already has).
+    Capacity applies to the whole batch, so it must not be combined with
+    `tokens` (a subset would see other ranks).
     """
+    if capacity > 0 and tokens is not None:
+        raise ValueError("capacity is a whole-batch limit: pass the batch itself, not a token subset")
     xs = x if tokens is None else x[tokens]
     r = route(xs, W_r, bias, k, renormalize)
     if idx is not None:
         r["idx"] = np.asarray(idx)
         r["w"] = as_f64(w) if w is not None else gate_weights(r["p"], r["idx"], renormalize)
     sel, wts = r["idx"], r["w"]
+    kept = kept_mask(sel, capacity)
+    r["kept"] = kept
     xe = bf16_round(as_f64(xs))
     out = np.zeros((xe.shape[0], xe.shape[1]), dtype=np.float64)
     if W1s is not None:
         out += swiglu_ffn(xe, W1s, W2s)
-    for e in np.unique(sel):
-        t_rows, slots = np.nonzero(sel == e)
+    for e in np.unique(sel[kept]):
+        t_rows, slots = np.nonzero((sel == e) & kept)
         y = swiglu_ffn(xe[t_rows], W1[int(e)], W2[int(e)])
         out[t_rows] += wts[t_rows, slots][:, None] * y
     r["out"] = out

@@ -238,3 +238,16 @@ def test_fp8_ffn_y_is_the_product_of_the_dequantised_codes():
     W2 = fp8.dequantize_128x128(W2q, s2)
     want = H @ W2.T
     assert np.allclose(r["y"], want, rtol=1e-12, atol=1e-12 * np.abs(want).max())
+
+
+def test_fp8_forward_does_not_depend_on_threads_or_prequantisation():
+    rng = np.random.default_rng(6)
+    T, d, E, I = 24, 256, 6, 128
+    x = oracle.bf16_round(rng.normal(size=(T, d)))
+    Wr = rng.normal(size=(E, d)) * 0.05
+    W1 = rng.normal(size=(E, 2 * I, d)) * 0.05
+    W2 = rng.normal(size=(E, d, I)) * 0.05
+    a = fp8.moe_forward_fp8(x, Wr, None, W1, W2, k=3)["out"]
+    q = {e: fp8.quantize_expert(W1[e], W2[e]) for e in range(E)}
+    b = fp8.moe_forward_fp8(x, Wr, None, W1, W2, k=3, quantized=q, workers=4)["out"]
+    assert np.array_equal(a, b)
