@@ -146,7 +146,7 @@ def quantize_expert(W1e, W2e) -> tuple:
 
 def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
                     renormalize: bool = False, tokens=None, idx=None, w=None,
-                    quantized=None, workers: int = 1) -> dict:
+                    quantized=None, workers: int = 1, capacity: int = 0) -> dict:
     """FP8 variant of oracle.moe_forward: same routing, quantised expert GEMMs.
 
     Each expert's W1[e] / W2[e] (bf16 values) is quantised per 128x128 block;
@@ -155,8 +155,13 @@ def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
     workloads with the same weights).  With workers > 1 the experts are
     evaluated on that many threads; each expert's rows are computed exactly as
     with one thread and the weighted outputs are still added in ascending
-    expert order, so the result does not depend on `workers`.
+    expert order, so the result does not depend on `workers`.  `capacity`
+    drops the pairs over an expert's capacity exactly as oracle.moe_forward
+    does (kept_mask).
     """
+    from .moe_oracle import kept_mask
+    if capacity > 0 and tokens is not None:
+        raise ValueError("capacity is a whole-batch limit: pass the batch itself, not a token subset")
     xs = x if tokens is None else x[tokens]
     r = route(xs, W_r, bias, k, renormalize)
     if idx is not None:
@@ -164,6 +169,8 @@ def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
         r["idx"] = np.asarray(idx)
         r["w"] = as_f64(w) if w is not None else gate_weights(r["p"], r["idx"], renormalize)
     sel, wts = r["idx"], r["w"]
+    kept = kept_mask(sel, capacity)
+    r["kept"] = kept
     xe = bf16_round(as_f64(xs)).astype(np.float32)
     xq, sx = quantize_1x128(xe)
     out = np.zeros(xe.shape, dtype=np.float64)
@@ -172,12 +179,12 @@ def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
         out += swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)["y"]
 
     def expert_rows(e):
-        t_rows, slots = np.nonzero(sel == e)
+        t_rows, slots = np.nonzero((sel == e) & kept)
         q = quantized[int(e)] if quantized is not None else quantize_expert(W1[int(e)], W2[int(e)])
         y = swiglu_ffn_fp8(xq[t_rows], sx[t_rows], *q)["y"]
         return t_rows, wts[t_rows, slots][:, None] * y
 
-    experts = np.unique(sel)
+    experts = np.unique(sel[kept])
     if workers > 1:
         from concurrent.futures import ThreadPoolExecutor
         with ThreadPoolExecutor(workers) as ex:

@@ -121,3 +121,22 @@ def test_capacity_rejects_token_subsets():
     with pytest.raises(ValueError):
         oracle.moe_forward(np.zeros((4, 8)), np.zeros((2, 8)), None, np.zeros((2, 4, 8)), np.zeros((2, 8, 2)),
                            k=1, tokens=[0, 1], capacity=1)
+
+
+def test_fp8_forward_drops_the_same_pairs():
+    from oracle import fp8
+    rng = np.random.default_rng(8)
+    T, d, E, k, I, C = 40, 256, 4, 2, 128, 9
+    x = oracle.bf16_round(rng.normal(size=(T, d)))
+    Wr = rng.normal(size=(E, d)) * 0.3
+    W1 = rng.normal(size=(E, 2 * I, d)) * 0.05
+    W2 = rng.normal(size=(E, d, I)) * 0.05
+    full = fp8.moe_forward_fp8(x, Wr, None, W1, W2, k=k)
+    cap = fp8.moe_forward_fp8(x, Wr, None, W1, W2, k=k, capacity=C)
+    kept = oracle.kept_mask(full["idx"], C)
+    assert np.array_equal(cap["kept"], kept) and not kept.all()
+    # the kept pairs' contributions are those of the full forward: with every pair over capacity
+    # given weight 0 instead, the same output results
+    zeroed = fp8.moe_forward_fp8(x, Wr, None, W1, W2, k=k, idx=full["idx"], w=full["w"] * kept)
+    assert np.allclose(cap["out"], zeroed["out"], rtol=1e-12, atol=1e-12)
+    assert np.array_equal(fp8.moe_forward_fp8(x, Wr, None, W1, W2, k=k, capacity=T)["out"], full["out"])
