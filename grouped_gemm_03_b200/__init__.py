@@ -19,6 +19,7 @@ import torch
 __all__ = [
     "LIB_PATH", "MoEError", "MoEConfig", "lib", "exported_symbols", "status_string", "device_info",
     "router_topk", "topk_logits", "permute", "grouped_gemm", "combine", "quantize_weights_fp8",
+    "capacity_from_factor",
     "workspace_size", "moe_forward", "moe_forward_marked", "moe_forward_host", "host_staging_size", "read_device_status",
     "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "EPI_NONE", "EPI_SILU_GATE",
 ]
@@ -43,7 +44,8 @@ class MoEError(RuntimeError):
 class MoEConfig(ctypes.Structure):
     """Mirror of `moe_config` in include/moe.h."""
     _fields_ = [(n, ctypes.c_int) for n in ("T", "d", "E", "k", "inter", "shared_inter", "x_dtype",
-                                            "router_dtype", "expert_dtype", "out_dtype", "renormalize")]
+                                            "router_dtype", "expert_dtype", "out_dtype", "renormalize",
+                                            "capacity")]
 
 
 _vp, _i, _sz, _fp, _ip = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
@@ -60,11 +62,14 @@ _SIGS = {
     "moe_topk_logits": (_i, [_vp, _i, _i, _i, _i, _i, _ip, _fp, _vp]),
     "moe_permute_workspace_size": (_sz, [_i, _i]),
     "moe_permute": (_i, [_vp, _i, _ip, _i, _i, _i, _i, _i, _i, _vp, _fp, _ip, _ip, _ip, _ip, _vp, _sz, _vp]),
+    "moe_permute_capacity": (_i, [_vp, _i, _ip, _i, _i, _i, _i, _i, _i, _i, _vp, _fp, _ip, _ip, _ip, _ip, _vp, _sz,
+                                  _vp]),
     "moe_permute_noalloc": (_i, [_vp, _i, _ip, _i, _i, _i, _i, _i, _i, _vp, _fp, _ip, _ip, _ip, _ip, _vp]),
     "moe_grouped_gemm_workspace_size": (_sz, []),
     "moe_grouped_gemm_plan": (ctypes.c_char_p, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "moe_grouped_gemm": (_i, [_vp, _fp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _vp, _i, _fp, _vp, _sz, _vp]),
     "moe_combine": (_i, [_vp, _ip, _fp, _i, _i, _i, _i, _vp, _i, _vp]),
+    "moe_combine_plan": (_i, [_vp, _ip, _fp, _ip, _i, _i, _i, _i, _i, _vp, _i, _vp]),
     "moe_selftest_workspace_size": (_sz, []),
     "moe_selftest_stalled_pipeline": (_i, [_vp, _sz, ctypes.c_ulonglong, _vp]),
     "moe_quantize_weights_fp8": (_i, [_vp, _i, _i, _i, _vp, _fp, _vp]),
@@ -184,7 +189,9 @@ def topk_logits(logits, k: int, renormalize: bool = False, out_idx=None, out_w=N
 
 
 # ---------------------------------------------------------------- permute
-def permute(x, topk_idx, E: int, append_shared: bool = False, fp8: bool = False, ws=None, stream=None) -> dict:
+def permute(x, topk_idx, E: int, append_shared: bool = False, fp8: bool = False, ws=None, stream=None,
+            capacity: int = 0) -> dict:
+    """Histogram, scan and scatter (moe_permute; moe_permute_capacity when capacity > 0)."""
     _cuda(x, topk_idx)
     T, d = x.shape
     k = topk_idx.shape[1]
@@ -199,9 +206,15 @@ def permute(x, topk_idx, E: int, append_shared: bool = False, fp8: bool = False,
     L = lib()
     if ws is None:
         ws = _scratch(L.moe_permute_workspace_size(T, E), dev)
-    _check(L.moe_permute(_ptr(x), _dt(x), _ptr(topk_idx), T, d, E, k, int(append_shared),
-                         MOE_E4M3 if fp8 else MOE_BF16, _ptr(xp), _ptr(xps), _ptr(counts), _ptr(offsets),
-                         _ptr(r2t), _ptr(t2r), _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
+    if capacity:
+        _check(L.moe_permute_capacity(_ptr(x), _dt(x), _ptr(topk_idx), T, d, E, k, int(append_shared), int(capacity),
+                                      MOE_E4M3 if fp8 else MOE_BF16, _ptr(xp), _ptr(xps), _ptr(counts),
+                                      _ptr(offsets), _ptr(r2t), _ptr(t2r), _ptr(ws), ws.numel(), _stream(stream)),
+               "moe_permute_capacity")
+    else:
+        _check(L.moe_permute(_ptr(x), _dt(x), _ptr(topk_idx), T, d, E, k, int(append_shared),
+                             MOE_E4M3 if fp8 else MOE_BF16, _ptr(xp), _ptr(xps), _ptr(counts), _ptr(offsets),
+                             _ptr(r2t), _ptr(t2r), _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
     return dict(xp=xp, xp_scales=xps, counts=counts, offsets=offsets, row_to_token=r2t, token_to_row=t2r, ws=ws)
 
 
@@ -235,11 +248,19 @@ def grouped_gemm_plan(G: int, rows: int, N: int, K: int, ab_dtype: int = MOE_BF1
                                        num_sms).decode()
 
 
-def combine(Y, token_to_row, topk_w, has_shared: bool, out_dtype=torch.bfloat16, out=None, stream=None):
-    _cuda(Y, token_to_row, topk_w)
+def combine(Y, token_to_row, topk_w, has_shared: bool, out_dtype=torch.bfloat16, out=None, stream=None,
+            offsets=None):
+    """Gather, weight and sum (moe_combine; with the permute's `offsets`, moe_combine_plan:
+    shared rows from offsets[E], overflowed slots skipped)."""
+    _cuda(Y, token_to_row, topk_w, offsets)
     T, k = token_to_row.shape
     d = Y.shape[1]
     o = out if out is not None else torch.empty((T, d), dtype=out_dtype, device=Y.device)
+    if offsets is not None:
+        E = offsets.numel() - 1 - (1 if has_shared else 0)
+        _check(lib().moe_combine_plan(_ptr(Y), _ptr(token_to_row), _ptr(topk_w), _ptr(offsets), E, int(has_shared),
+                                      T, d, k, _ptr(o), _dt(o), _stream(stream)), "moe_combine_plan")
+        return o
     _check(lib().moe_combine(_ptr(Y), _ptr(token_to_row), _ptr(topk_w), int(has_shared), T, d, k, _ptr(o),
                              _dt(o), _stream(stream)), "moe_combine")
     return o
@@ -261,9 +282,15 @@ def quantize_weights_fp8(W, stream=None):
 
 # ---------------------------------------------------------------- whole layer
 def make_config(T, d, E, k, inter, shared_inter=0, x_dtype=MOE_BF16, router_dtype=MOE_BF16,
-                expert_dtype=MOE_BF16, out_dtype=MOE_BF16, renormalize=False) -> MoEConfig:
+                expert_dtype=MOE_BF16, out_dtype=MOE_BF16, renormalize=False, capacity=0) -> MoEConfig:
     return MoEConfig(T, d, E, k, inter, shared_inter, x_dtype, router_dtype, expert_dtype, out_dtype,
-                     int(renormalize))
+                     int(renormalize), int(capacity))
+
+
+def capacity_from_factor(factor: float, T: int, k: int, E: int) -> int:
+    """Per-expert row limit for a capacity factor: ceil(factor * T * k / E), at least 1."""
+    import math
+    return max(1, math.ceil(factor * T * k / E))
 
 
 def workspace_size(cfg: MoEConfig) -> int:

@@ -2,7 +2,9 @@
 // them by their gate values and sum, adding the shared expert's row
 // ("Dense GEMM -> GroupedGEMM -> TP MoE" §2.2 step 6; "MegaMoE ..." §2.1).
 //   out[t] = Y[R + t] + sum_{j<k} w[t, j] * Y[token_to_row[t, j]]
-// fp32 accumulation in that fixed order, 16-byte loads.
+// fp32 accumulation in that fixed order, 16-byte loads.  R is T*k, or the
+// first shared row the permute recorded (offsets[E]) when experts have a
+// capacity; a slot whose pair overflowed (token_to_row < 0) adds nothing.
 #include "common.cuh"
 
 namespace moe {
@@ -41,7 +43,8 @@ template <typename OT>
 __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat16* __restrict__ Y,
                                                               const int32_t* __restrict__ t2r,
                                                               const float* __restrict__ w, int has_shared,
-                                                              int T, int d, int k, OT* __restrict__ out) {
+                                                              int T, int d, int k, OT* __restrict__ out,
+                                                              const int32_t* __restrict__ shared_base) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
   const int t = blockIdx.x;
@@ -49,7 +52,7 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat
   const int c1 = c0 + kCombThreads * 8;                                   // second piece
   const bool p0 = c0 < d, p1 = c1 < d;
   if (!p0) return;
-  const size_t R = static_cast<size_t>(T) * k;
+  const size_t R = shared_base ? static_cast<size_t>(__ldg(shared_base)) : static_cast<size_t>(T) * k;
   float a0[8], a1[8];
   if (has_shared) {
     const __nv_bfloat16* ys = Y + (R + t) * d;
@@ -67,10 +70,15 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat
     float wj[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
-      const __nv_bfloat16* yr = Y + static_cast<size_t>(__ldg(rows + j + u)) * d;
-      wj[u] = __ldg(ws + j + u);
-      r0[u] = __ldg(reinterpret_cast<const uint4*>(yr + c0));
-      if (p1) r1[u] = __ldg(reinterpret_cast<const uint4*>(yr + c1));
+      const int row = __ldg(rows + j + u);
+      // an overflowed slot (row < 0) contributes +0 * 0: the sum is unchanged
+      const __nv_bfloat16* yr = Y + static_cast<size_t>(row < 0 ? 0 : row) * d;
+      wj[u] = row < 0 ? 0.f : __ldg(ws + j + u);
+      r0[u] = r1[u] = make_uint4(0, 0, 0, 0);
+      if (row >= 0) {
+        r0[u] = __ldg(reinterpret_cast<const uint4*>(yr + c0));
+        if (p1) r1[u] = __ldg(reinterpret_cast<const uint4*>(yr + c1));
+      }
     }
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
@@ -86,7 +94,9 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat
     }
   }
   for (; j < k; ++j) {
-    const __nv_bfloat16* yr = Y + static_cast<size_t>(__ldg(rows + j)) * d;
+    const int row = __ldg(rows + j);
+    if (row < 0) continue;  // overflowed its expert's capacity
+    const __nv_bfloat16* yr = Y + static_cast<size_t>(row) * d;
     const float wj = __ldg(ws + j);
     float f[8];
     unpack8(__ldg(reinterpret_cast<const uint4*>(yr + c0)), f);
@@ -106,15 +116,15 @@ __global__ void __launch_bounds__(kCombThreads) combine_kernel(const __nv_bfloat
 }  // namespace
 
 int launch_combine(const void* Y, const int32_t* t2r, const float* w, int has_shared, int T, int d, int k,
-                   void* out, int out_dtype, cudaStream_t s) {
+                   void* out, int out_dtype, cudaStream_t s, const int32_t* shared_base) {
   if (T == 0) return MOE_OK;
   const __nv_bfloat16* y = static_cast<const __nv_bfloat16*>(Y);
   const dim3 grid(T, (d + kCombCols - 1) / kCombCols);
   if (out_dtype == MOE_F32)
     return launch_pdl(__func__, combine_kernel<float>, grid, dim3(kCombThreads), 0, s, y, t2r, w, has_shared, T, d, k,
-                      static_cast<float*>(out));
+                      static_cast<float*>(out), shared_base);
   return launch_pdl(__func__, combine_kernel<__nv_bfloat16>, grid, dim3(kCombThreads), 0, s, y, t2r, w, has_shared, T,
-                    d, k, static_cast<__nv_bfloat16*>(out));
+                    d, k, static_cast<__nv_bfloat16*>(out), shared_base);
 }
 
 }  // namespace moe

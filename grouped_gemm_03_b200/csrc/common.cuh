@@ -75,6 +75,7 @@ struct PermuteArgs {
   int32_t* token_to_row;
   int32_t* block_base;  // scratch [nblocks * E]
   int* status;
+  int capacity = 0;     // > 0: an expert keeps only its first `capacity` pairs in token order
 };
 int permute_blocks(int T);  // number of token blocks the permute kernels use
 int launch_permute(const PermuteArgs& a, cudaStream_t s);
@@ -105,8 +106,11 @@ int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s);
 int plan_grouped_gemm(const GemmArgs& a, int sms);  // host-only choice of kernel (see gemm_variant_name)
 const char* gemm_variant_name(int variant);
 
+// shared_base: device int32 holding the first shared row (offsets[E] of the
+// permute), or nullptr for the fixed T*k.  token_to_row entries < 0 are
+// slots that overflowed an expert's capacity and are skipped.
 int launch_combine(const void* Y, const int32_t* t2r, const float* w, int has_shared, int T, int d, int k,
-                   void* out, int out_dtype, cudaStream_t s);
+                   void* out, int out_dtype, cudaStream_t s, const int32_t* shared_base = nullptr);
 int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, cudaStream_t s);
 
 int num_sms();

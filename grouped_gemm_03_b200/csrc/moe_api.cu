@@ -91,6 +91,7 @@ int check_config(const moe_config* c) {
   if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID;
   if (c->d % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->expert_dtype == MOE_E4M3 && c->d % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (c->capacity < 0) return MOE_ERR_INVALID;
   const long long rows = static_cast<long long>(c->T) * (c->k + 1);
   if (rows * c->d > (1ll << 40) || rows > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -177,11 +178,13 @@ size_t moe_permute_workspace_size(int T, int E) {
   return 256 + align_up(static_cast<size_t>(permute_blocks(T)) * E * 4, 256);
 }
 
-int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k, int append_shared,
-                int xp_dtype, void* xp, float* xp_scales, int32_t* counts, int32_t* offsets, int32_t* row_to_token,
-                int32_t* token_to_row, void* ws, size_t ws_bytes, void* stream) {
+namespace {
+int permute_impl(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k, int append_shared,
+                 int capacity, int xp_dtype, void* xp, float* xp_scales, int32_t* counts, int32_t* offsets,
+                 int32_t* row_to_token, int32_t* token_to_row, void* ws, size_t ws_bytes, void* stream) {
   if (T < 0 || d <= 0 || E <= 0 || k <= 0 || k > E || k > kMaxTopK || E > kMaxExperts) return MOE_ERR_INVALID;
   if (static_cast<long long>(T) * (k + 1) > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
+  if (capacity < 0) return MOE_ERR_INVALID;
   if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID;
   if (xp_dtype != MOE_BF16 && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID;
   if (d % 8 != 0 || (xp_dtype == MOE_E4M3 && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;
@@ -211,7 +214,24 @@ int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int 
   a.token_to_row = token_to_row;
   a.block_base = reinterpret_cast<int32_t*>(static_cast<char*>(ws) + 256);
   a.status = static_cast<int*>(ws);
+  a.capacity = capacity;
   return launch_permute(a, s);
+}
+}  // namespace
+
+int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k, int append_shared,
+                int xp_dtype, void* xp, float* xp_scales, int32_t* counts, int32_t* offsets, int32_t* row_to_token,
+                int32_t* token_to_row, void* ws, size_t ws_bytes, void* stream) {
+  return permute_impl(x, x_dtype, topk_idx, T, d, E, k, append_shared, 0, xp_dtype, xp, xp_scales, counts, offsets,
+                      row_to_token, token_to_row, ws, ws_bytes, stream);
+}
+
+int moe_permute_capacity(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k,
+                         int append_shared, int capacity, int xp_dtype, void* xp, float* xp_scales, int32_t* counts,
+                         int32_t* offsets, int32_t* row_to_token, int32_t* token_to_row, void* ws, size_t ws_bytes,
+                         void* stream) {
+  return permute_impl(x, x_dtype, topk_idx, T, d, E, k, append_shared, capacity, xp_dtype, xp, xp_scales, counts,
+                      offsets, row_to_token, token_to_row, ws, ws_bytes, stream);
 }
 
 // ------------------------------------------------------------------ grouped GEMM
@@ -312,6 +332,17 @@ int moe_combine(const void* Y, const int32_t* token_to_row, const float* topk_w,
   return launch_combine(Y, token_to_row, topk_w, has_shared, T, d, k, out, out_dtype, as_stream(stream));
 }
 
+int moe_combine_plan(const void* Y, const int32_t* token_to_row, const float* topk_w, const int32_t* offsets, int E,
+                     int has_shared, int T, int d, int k, void* out, int out_dtype, void* stream) {
+  if (T < 0 || d <= 0 || k <= 0 || k > kMaxTopK || E <= 0 || E > kMaxExperts) return MOE_ERR_INVALID;
+  if (d % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (out_dtype != MOE_F32 && out_dtype != MOE_BF16) return MOE_ERR_INVALID;
+  if (T > 0 && (!Y || !token_to_row || !topk_w || !out || !offsets)) return MOE_ERR_INVALID;
+  if (!aligned(Y, 16) || !aligned(out, 16)) return MOE_ERR_INVALID;
+  return launch_combine(Y, token_to_row, topk_w, has_shared, T, d, k, out, out_dtype, as_stream(stream),
+                        T > 0 ? offsets + E : nullptr);
+}
+
 // ------------------------------------------------------------------ FP8 weights
 int moe_quantize_weights_fp8(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, void* stream) {
   if (G < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID;
@@ -393,6 +424,7 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   pa.token_to_row = t2r;
   pa.block_base = reinterpret_cast<int32_t*>(base + L.base);
   pa.status = status;
+  pa.capacity = c.capacity;
   st = launch_permute(pa, s);
   if (st != MOE_OK) return st;
   if ((st = mark(2)) != MOE_OK) return st;
@@ -446,7 +478,7 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   if (st != MOE_OK) return st;
   if ((st = mark(4)) != MOE_OK) return st;
 
-  st = launch_combine(base + L.y, t2r, w, shared ? 1 : 0, T, d, k, out, c.out_dtype, s);
+  st = launch_combine(base + L.y, t2r, w, shared ? 1 : 0, T, d, k, out, c.out_dtype, s, offsets + E);
   if (st != MOE_OK) return st;
   if ((st = mark(5)) != MOE_OK) return st;
   if (counts_out) MOE_CUDA_CHECK(cudaMemcpyAsync(counts_out, counts, sizeof(int32_t) * E, cudaMemcpyDeviceToDevice, s));

@@ -11,8 +11,13 @@
 //           offsets[e] + sum_{b' < b} cnt[b'][e], plus counts / offsets;
 //   scatter block b ranks its pairs by token order inside the block and
 //           copies each token's row to its k destinations (and, for the
-//           shared expert, to row R + t), casting to bf16 or quantising to
-//           E4M3 with one scale per 128 columns on the way.
+//           shared expert, to row offsets[E] + t), casting to bf16 or
+//           quantising to E4M3 with one scale per 128 columns on the way.
+// With a capacity C ("Dense GEMM -> GroupedGEMM -> TP MoE" §5.1: a capacity
+// factor caps each expert's tokens, the rest take a fallback path) an expert
+// keeps its first C pairs in token order: the scan counts min(n_e, C) rows
+// per expert, and a pair whose rank in its expert reaches C gets no row
+// (token_to_row = -1); the shared expert's rows follow the kept rows.
 #include <mutex>
 
 #include "common.cuh"
@@ -55,8 +60,8 @@ __global__ void __launch_bounds__(kPermThreads) hist_kernel(const int32_t* __res
 // of a batch are in flight together.
 constexpr int kScanBatch = 8;
 
-__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, int nblk, int E, int R, int T,
-                                                    int shared, int32_t* __restrict__ counts,
+__global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, int nblk, int E, int T,
+                                                    int shared, int capacity, int32_t* __restrict__ counts,
                                                     int32_t* __restrict__ offsets) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
@@ -90,7 +95,8 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, 
   __syncthreads();
   // exclusive scan of s_tot[0..E) by the whole block (one value per thread)
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int mine = threadIdx.x < E ? s_tot[threadIdx.x] : 0;
+  // rows an expert keeps: all of its pairs, or the first `capacity` of them
+  const int mine = threadIdx.x < E ? (capacity > 0 ? min(s_tot[threadIdx.x], capacity) : s_tot[threadIdx.x]) : 0;
   int incl = mine;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
@@ -116,9 +122,11 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, 
     counts[threadIdx.x] = mine;
     offsets[threadIdx.x] = excl;
   }
-  if (threadIdx.x == 0) {
-    offsets[E] = R;
-    if (shared) offsets[E + 1] = R + T;
+  if (threadIdx.x == E - 1) {  // E <= 1024 = blockDim.x
+    // the kept rows end where the last expert's do; the shared rows follow them
+    const int used = excl + mine;
+    offsets[E] = used;
+    if (shared) offsets[E + 1] = used + T;
   }
   __syncthreads();
   if (active) {
@@ -161,7 +169,9 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   const int rows_total = R + (a.shared ? a.T : 0);
   const int nd = k + (a.shared ? 1 : 0);  // destinations per token
   const bool writer = blockIdx.y == 0;   // one column block writes the index maps
+  __shared__ int s_used;  // rows the experts keep: the shared rows start there
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) s_idx[p] = a.idx[static_cast<size_t>(t0) * k + p];
+  if (threadIdx.x == 0) s_used = a.offsets[E];
   __syncthreads();
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
     const int tl = p / k, j = p % k;
@@ -171,19 +181,26 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
       int rank = 0;
       for (int q = 0; q < tl * k; ++q) rank += (s_idx[q] == e);
       row = a.block_base[static_cast<size_t>(b) * E + e] + rank;
-      if (row < 0 || row >= R) row = 0;  // only reachable with invalid ids (status already set)
+      // past the expert's capacity: the pair overflows and gets no row
+      if (a.capacity > 0 && row - a.offsets[e] >= a.capacity) row = -1;
+      if (row >= R) row = 0;  // only reachable with invalid ids (status already set)
     }
     s_row[tl * nd + j] = row;
     if (writer) {
       a.token_to_row[static_cast<size_t>(t0 + tl) * k + j] = row;
-      a.row_to_token[row] = t0 + tl;
+      if (row >= 0) a.row_to_token[row] = t0 + tl;
     }
   }
   if (a.shared)
     for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) {
-      s_row[tl * nd + k] = R + t0 + tl;
-      if (writer) a.row_to_token[R + t0 + tl] = t0 + tl;
+      s_row[tl * nd + k] = s_used + t0 + tl;
+      if (writer) a.row_to_token[s_used + t0 + tl] = t0 + tl;
     }
+  if (writer && a.capacity > 0) {  // rows left unused by the overflowing pairs belong to no token
+    const int end = s_used + (a.shared ? a.T : 0);
+    for (int r = end + b * blockDim.x + threadIdx.x; r < rows_total; r += gridDim.x * blockDim.x)
+      a.row_to_token[r] = -1;
+  }
   __syncthreads();
 
   const int d = a.d;
@@ -220,8 +237,10 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         if (tl[u] < 0) continue;
-        for (int j = 0; j < nd; ++j)
-          *reinterpret_cast<uint4*>(xp + static_cast<size_t>(s_row[tl[u] * nd + j]) * d + c[u]) = v[u];
+        for (int j = 0; j < nd; ++j) {
+          const int row = s_row[tl[u] * nd + j];
+          if (row >= 0) *reinterpret_cast<uint4*>(xp + static_cast<size_t>(row) * d + c[u]) = v[u];
+        }
       }
     }
   } else {
@@ -274,6 +293,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
       if (!act) continue;
       for (int j = 0; j < nd; ++j) {
         const int row = s_row[tl * nd + j];
+        if (row < 0) continue;  // overflowed its expert's capacity
         *reinterpret_cast<uint2*>(xp + static_cast<size_t>(row) * d + c) = qv;
         if (sub == 0) a.xp_scales[static_cast<size_t>(gi) * rows_total + row] = s;
       }
@@ -296,8 +316,8 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
   int st = launch_pdl("hist_kernel", hist_kernel, dim3(nblk), dim3(kPermThreads), sizeof(int) * a.E, s, a.idx, a.T,
                       a.E, a.k, a.block_base, a.status);
   if (st != MOE_OK) return st;
-  st = launch_pdl("scan_kernel", scan_kernel, dim3(1), dim3(1024), 0, s, a.block_base, nblk, a.E, a.T * a.k, a.T,
-                  a.shared, a.counts, a.offsets);
+  st = launch_pdl("scan_kernel", scan_kernel, dim3(1), dim3(1024), 0, s, a.block_base, nblk, a.E, a.T, a.shared,
+                  a.capacity, a.counts, a.offsets);
   if (st != MOE_OK) return st;
   const bool fp8 = a.xp_dtype == MOE_E4M3;
   const dim3 grid(nblk, (a.d + kScatterCols - 1) / kScatterCols);

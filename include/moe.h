@@ -38,7 +38,7 @@
 extern "C" {
 #endif
 
-#define MOE_ABI_VERSION 1
+#define MOE_ABI_VERSION 2
 
 typedef enum moe_status {
   MOE_OK = 0,
@@ -64,11 +64,20 @@ typedef enum moe_epilogue {
  * d and inter are multiples of 128 (E4M3 experts: d a multiple of 256).
  * renormalize = 0 weights each expert by its softmax value p_i (MegaMoE §2.1);
  * 1 divides by the sum over the selected experts (route_tokens in
- * Dense GEMM -> GroupedGEMM -> TP MoE §4.2). */
+ * Dense GEMM -> GroupedGEMM -> TP MoE §4.2).
+ * capacity = 0: no limit; > 0: each expert takes at most `capacity` of the
+ * batch's (token, slot) pairs, the first ones in token order, and a pair
+ * over it adds nothing to its token's output (the token keeps the shared
+ * expert and its other experts, weights unchanged).  This is the capacity
+ * factor of Dense GEMM -> GroupedGEMM -> TP MoE §5.1 (tokens over an
+ * expert's capacity take a fallback path) and DeepSeek MoE architecture
+ * overview §3.2 (a bound on one expert's share of a forward's tokens);
+ * capacity = ceil(factor * T * k / E) for a capacity factor `factor`. */
 typedef struct moe_config {
   int T, d, E, k, inter, shared_inter;
   int x_dtype, router_dtype, expert_dtype, out_dtype;
   int renormalize;
+  int capacity;
 } moe_config;
 
 /* Human-readable name of a status code (static string). */
@@ -135,6 +144,21 @@ int moe_permute(const void* x, int x_dtype, const int32_t* topk_idx, int T, int 
                 int append_shared, int xp_dtype, void* xp, float* xp_scales, int32_t* counts,
                 int32_t* offsets, int32_t* row_to_token, int32_t* token_to_row, void* ws, size_t ws_bytes,
                 void* stream);
+
+/* moe_permute with a capacity limit (capacity = 0: none): each expert keeps
+ * its first `capacity` (token, slot) pairs in token order, as moe_config's
+ * capacity describes.  A pair over its expert's capacity gets no row
+ * (token_to_row = -1); counts[e] are the kept rows, offsets their exclusive
+ * scan, offsets[E] the kept total R_kept, and with append_shared the shared
+ * expert's rows are R_kept .. R_kept+T-1 (offsets[E+1] = R_kept + T).  Rows
+ * from there up to R' - 1 belong to no token (row_to_token = -1).  The
+ * buffers keep moe_permute's sizes (R' = T*k (+ T) rows).  The pairs with
+ * token_to_row = -1 are the overflow: a caller may send them to another
+ * path (moe_combine_plan skips them).  capacity < 0: MOE_ERR_INVALID. */
+int moe_permute_capacity(const void* x, int x_dtype, const int32_t* topk_idx, int T, int d, int E, int k,
+                         int append_shared, int capacity, int xp_dtype, void* xp, float* xp_scales,
+                         int32_t* counts, int32_t* offsets, int32_t* row_to_token, int32_t* token_to_row,
+                         void* ws, size_t ws_bytes, void* stream);
 
 /* Allocation-free variant of moe_permute, for callers that cannot give the
  * library any device memory of its own: a plugin whose host runtime owns all
@@ -226,6 +250,13 @@ int moe_selftest_stalled_pipeline(void* ws, size_t ws_bytes, unsigned long long 
 int moe_combine(const void* Y, const int32_t* token_to_row, const float* topk_w, int has_shared, int T,
                 int d, int k, void* out, int out_dtype, void* stream);
 
+/* moe_combine over a plan from moe_permute_capacity: the shared expert's row
+ * of token t is offsets[E] + t (offsets: the permute's DEVICE array), and a
+ * slot with token_to_row[t, j] < 0 (its pair overflowed an expert's
+ * capacity) adds nothing.  Otherwise as moe_combine. */
+int moe_combine_plan(const void* Y, const int32_t* token_to_row, const float* topk_w, const int32_t* offsets, int E,
+                     int has_shared, int T, int d, int k, void* out, int out_dtype, void* stream);
+
 /* ---------------------------------------------------------------- FP8 weights
  * Quantise bf16 weights W [G, N, K] per 128x128 block ("MegaMoE ..." §2.3,
  * §5.1): s = amax(block)/448 (1 if the block is zero), Wq = e4m3_rn_satfinite(W/s).
@@ -241,7 +272,8 @@ int moe_quantize_weights_fp8(const void* W, int G, int N, int K, uint8_t* Wq, fl
  *   BF16 experts: W1 [E, 2I, d], W2 [E, d, I] bf16, *_scales NULL
  *   E4M3 experts: W1/W2 as moe_quantize_weights_fp8 output with their scales
  *   W1_shared [2I, d], W2_shared [d, I] (+ scales) or NULL
- *   out [T, d] cfg->out_dtype;  counts_out [E] int32 (tokens per expert) or NULL
+ *   out [T, d] cfg->out_dtype;  counts_out [E] int32 (rows each expert took:
+ *       its tokens, or at most cfg->capacity of them) or NULL
  *   ws  moe_workspace_size(cfg) bytes: status, routing, permutation plan and
  *       the intermediates Xp [R', d], H [R', I], Y [R', d].
  * No host synchronisation and no host<->device copy: the call can be

@@ -1,5 +1,7 @@
 """FP8 (E4M3) path: the grouped GEMM with per-128-K scale promotion and the
-whole layer with E4M3 experts, against the quantisation-simulating oracle.
+whole layer with E4M3 experts, against the quantisation-simulating oracle;
+at full size the layer is compared on 512+ tokens that together route to
+every non-empty group, and the GEMMs at the fine-grained layer's real shapes.
 
 Bars: bf16 outputs within 2e-3 relative Frobenius of the oracle's blockwise
 fp64 product of the SAME quantised operands; E4M3 outputs (the intermediate
@@ -84,7 +86,7 @@ def test_grouped_gemm_fp8(sizes, N, K, epi, cdt):
         rq, rs = ofp8.quantize_1x128(ref.astype(np.float32))
         np.testing.assert_allclose(gs, rs, rtol=1e-5)
         same = gq == rq
-        assert same.mean() > 0.99, same.mean()
+        assert same.mean() >= 1 - 1e-3, same.mean()  # at most one code in a thousand flips
         diff = np.abs(ofp8.e4m3_decode(gq).astype(np.float64) - ofp8.e4m3_decode(rq))
         step = np.abs(ofp8.e4m3_decode(rq)) * 2.0 ** -3 + 2.0 ** -9
         assert np.all(diff[~same] <= step[~same] * 1.01)
@@ -143,19 +145,134 @@ def test_fp8_layer_every_element(T, E, k, I, shared, xdt):
     assert err < 1e-2, err
 
 
-@pytest.mark.parametrize("name,nsample", [("fine_fp8", 3), ("fine_fp8_skew", 3)])
-def test_fp8_full_size_sampled_tokens(name, nsample):
+# Oracle-quantised expert weights of the full-size fine-grained layer, kept
+# for the module: the balanced and skewed FP8 workloads draw the same weights
+# (same seed and shapes; only the router bias differs).
+_QUANTISED = {}
+
+
+def _oracle_quantised(s, inp, experts):
+    from concurrent.futures import ThreadPoolExecutor
+    from threadpoolctl import threadpool_limits
+    from _util import StreamedExperts, host_threads
+    key = (s.d, s.E, s.inter, 1234)
+    cache = _QUANTISED.setdefault(key, {})
+    W1, W2 = StreamedExperts(inp["W1"]), StreamedExperts(inp["W2"])
+    need = [int(e) for e in experts if int(e) not in cache]
+    with threadpool_limits(1), ThreadPoolExecutor(host_threads()) as ex:
+        for e, q in zip(need, ex.map(lambda e: ofp8.quantize_expert(W1[e], W2[e]), need)):
+            cache[e] = q
+    return cache
+
+
+@pytest.mark.parametrize("name", ["fine_fp8", "fine_fp8_skew"])
+def test_fp8_full_size_tokens_covering_every_group(name):
+    from threadpoolctl import threadpool_limits
+    from _util import check_plan_full_size, host_threads, tokens_covering_every_group
     s = shape_of(name)
     inp = make_inputs(s, seed=1234, device=DEV)
+    gidx = check_plan_full_size(gg, s, inp)
     cfg = _cfg(s)
     w = _fp8_weights(inp)
     ws = torch.empty(gg.workspace_size(cfg), dtype=torch.uint8, device=DEV)
-    out = gg.moe_forward(cfg, inp["x"], inp["W_r"], inp["bias"], w, ws=ws)
+    counts = torch.empty(s.E, dtype=torch.int32, device=DEV)
+    out = gg.moe_forward(cfg, inp["x"], inp["W_r"], inp["bias"], w, counts_out=counts, ws=ws)
     torch.cuda.synchronize()
     assert gg.read_device_status(ws) == 0
-    tokens = np.sort(np.random.default_rng(5).choice(s.T, size=nsample, replace=False))
-    ref = _oracle_fp8(s, inp, tokens)["out"]
-    err = rel_fro(f64(out[torch.from_numpy(tokens).to(DEV)]), ref)
-    assert err < TOL_FP8, err
+    assert np.array_equal(counts.cpu().numpy(), oracle.expert_counts(gidx, s.E))
+    tokens = tokens_covering_every_group(gidx, s.E, 512)
+    assert len(tokens) >= 512
+    # together the tokens route to every non-empty group (the shared expert takes them all)
+    assert set(np.unique(gidx[tokens]).tolist()) == set(np.unique(gidx).tolist())
+    xs = inp["x"][torch.from_numpy(tokens).to(DEV)]
+    r = oracle.route(xs, inp["W_r"], inp["bias"], s.k, s.renormalize)
+    idx, adopted, bad = adopt_near_ties(r["logits"], r["idx"], gidx[tokens], s.k)
+    assert not bad
+    q = _oracle_quantised(s, inp, np.unique(idx))
+    with threadpool_limits(1):
+        ref = ofp8.moe_forward_fp8(xs, inp["W_r"], inp["bias"], None, None, f64(inp["W1s"]), f64(inp["W2s"]),
+                                   k=s.k, renormalize=s.renormalize, idx=idx, quantized=q,
+                                   workers=host_threads())["out"]
+    got = f64(out[torch.from_numpy(tokens).to(DEV)])
+    err = rel_fro(got, ref)
+    assert err < TOL_FP8, (err, len(adopted))
+    per_token = np.linalg.norm(got - ref, axis=1) / np.maximum(np.linalg.norm(ref, axis=1), 1e-30)
+    assert per_token.max() < 2 * TOL_FP8, (int(per_token.argmax()), per_token.max())
     del inp, w
     torch.cuda.empty_cache()
+
+
+# ---------------------------------------------------------------- the fine-grained layer's FP8 GEMM shapes
+# 257 groups (256 routed experts + the shared one) with Zipf-skewed sizes
+# summing to T*k + T = 36864 rows, at the real K / N of the up (K = 7168,
+# N = 2048, SiLU gate, E4M3 h out) and down (K = 2048, N = 7168, bf16 out)
+# projections.  Operands are random E4M3 codes with random fp32 scales; the
+# oracle computes sampled rows covering every 128-row block of every group.
+def _fine_sizes(seed=3):
+    rng = np.random.default_rng(seed)
+    w = 1.0 / (1.0 + np.arange(256)) ** 0.85
+    w = w[rng.permutation(256)]
+    sizes = np.floor(w / w.sum() * 32768).astype(int)
+    sizes[rng.choice(256, size=6, replace=False)] = 0  # a few empty experts
+    sizes[0] += 32768 - sizes.sum()
+    return [int(v) for v in sizes] + [4096]          # + the shared expert's group
+
+
+def _random_codes(shape, gen):
+    c = torch.randint(0, 256, shape, dtype=torch.uint8, device=DEV, generator=gen)
+    return torch.where((c & 0x7F) == 0x7F, c - 1, c)  # no NaN codes
+
+
+@pytest.mark.parametrize("N,K,epi,cdt", [(2048, 7168, gg.EPI_SILU_GATE, torch.uint8),
+                                          (7168, 2048, gg.EPI_NONE, torch.bfloat16)])
+def test_grouped_gemm_fp8_fine_shapes(N, K, epi, cdt):
+    from concurrent.futures import ThreadPoolExecutor
+    from threadpoolctl import threadpool_limits
+    from _util import host_threads, rows_in_every_block
+    sizes = _fine_sizes()
+    G = len(sizes)
+    rows = sum(sizes)
+    Nb = 2 * N if epi == gg.EPI_SILU_GATE else N
+    gen = torch.Generator(device=DEV).manual_seed(N + K)
+    Aq = _random_codes((rows, K), gen)
+    Bq = _random_codes((G, Nb, K), gen)
+    As = (torch.rand((K // 128, rows), device=DEV, generator=gen) + 0.5) * 2.0 ** -9
+    Bs = (torch.rand((G, Nb // 128, K // 128), device=DEV, generator=gen) + 0.5) * 2.0 ** -9
+    offsets = torch.tensor(np.concatenate([[0], np.cumsum(sizes)]).astype(np.int32), device=DEV)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    res = gg.grouped_gemm(Aq, Bq, offsets, N, epilogue=epi, c_dtype=cdt, A_scales=As, B_scales=Bs, ws=ws)
+    assert gg.read_device_status(ws) == 0
+    sample = rows_in_every_block(sizes, np.random.default_rng(K), per_block=1)
+    bounds = np.concatenate([[0], np.cumsum(sizes)])
+    qa = Aq[torch.from_numpy(sample).to(DEV)].cpu().numpy()
+    sa = As.T[torch.from_numpy(sample).to(DEV)].cpu().numpy()
+
+    def group_ref(g):
+        sel = np.nonzero((sample >= bounds[g]) & (sample < bounds[g + 1]))[0]
+        if not len(sel):
+            return sel, None
+        c = ofp8.fp8_gemm(qa[sel], sa[sel], Bq[g].cpu().numpy(), Bs[g].cpu().numpy())
+        if epi == gg.EPI_SILU_GATE:
+            c = c[:, :N] / (1 + np.exp(-c[:, :N])) * c[:, N:]
+        return sel, c
+
+    ref = np.zeros((len(sample), N))
+    with threadpool_limits(1), ThreadPoolExecutor(host_threads()) as ex:
+        for sel, c in ex.map(group_ref, range(G)):
+            if c is not None:
+                ref[sel] = c
+    idx = torch.from_numpy(sample).to(DEV)
+    if cdt == torch.uint8:
+        C, Cs = res
+        gq = C[idx].cpu().numpy()
+        gs = Cs.T[idx].cpu().numpy()
+        rq, rs = ofp8.quantize_1x128(ref.astype(np.float32))
+        np.testing.assert_allclose(gs, rs, rtol=1e-5)
+        same = gq == rq
+        assert same.mean() >= 1 - 1e-3, same.mean()
+        diff = np.abs(ofp8.e4m3_decode(gq) - ofp8.e4m3_decode(rq))
+        step = np.abs(ofp8.e4m3_decode(rq)) * 2.0 ** -3 + 2.0 ** -9
+        assert np.all(diff[~same] <= step[~same] * 1.01)
+    else:
+        err = rel_fro(f64(res[idx]), ref)
+        assert err < 2e-3, err

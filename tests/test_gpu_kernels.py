@@ -307,3 +307,46 @@ def test_selftest_rejects_bad_arguments():
     ws = torch.zeros(L.moe_selftest_workspace_size(), dtype=torch.uint8, device=DEV)
     assert L.moe_selftest_stalled_pipeline(gg._ptr(ws), 100, 50_000_000, gg._stream()) == -3
     assert L.moe_selftest_stalled_pipeline(gg._ptr(ws), ws.numel(), 10, gg._stream()) == -1
+
+
+# ---------------------------------------------------------------- the full-size layers' GEMM shapes
+# The Mixtral-shaped layer's two GEMMs at their real sizes (CTA pairs, K = 4096
+# and K = 14336 main loops, Zipf-skewed groups summing to T*k = 8192 rows),
+# compared on sampled rows that cover every 128-row block of every group.
+MIXTRAL_SIZES = [561, 2121, 1280, 700, 950, 1105, 620, 855]
+
+
+@pytest.mark.parametrize("N,K,epi", [(14336, 4096, gg.EPI_SILU_GATE), (4096, 14336, gg.EPI_NONE)])
+def test_grouped_gemm_bf16_mixtral_shapes(N, K, epi):
+    from _util import rows_in_every_block
+    sizes = MIXTRAL_SIZES
+    assert "cta-pair" in gg.grouped_gemm_plan(len(sizes), sum(sizes), N, K, epilogue=epi)
+    torch.manual_seed(N + K)
+    rows = sum(sizes) + 3
+    G = len(sizes)
+    Nb = 2 * N if epi == gg.EPI_SILU_GATE else N
+    A = torch.randn((rows, K), device=DEV).to(torch.bfloat16)
+    B = (torch.randn((G, Nb, K), device=DEV) * 0.02).to(torch.bfloat16)
+    C = torch.full((rows, N), 7.0, dtype=torch.bfloat16, device=DEV)
+    ws = torch.empty(256, dtype=torch.uint8, device=DEV)
+    gg.grouped_gemm(A, B, _offsets(sizes), N, epilogue=epi, out=C, ws=ws)
+    assert gg.read_device_status(ws) == 0
+    sample = rows_in_every_block(sizes, np.random.default_rng(N), per_block=2)
+    bounds = np.concatenate([[0], np.cumsum(sizes)])
+    got, ref = [], []
+    for g in range(G):
+        r = sample[(sample >= bounds[g]) & (sample < bounds[g + 1])]
+        if not len(r):
+            continue
+        Ar = f64(A[torch.from_numpy(r).to(DEV)])
+        Bg = B[g].to(torch.float64).cpu().numpy()  # exact widening
+        if epi == gg.EPI_SILU_GATE:
+            gt, up = Ar @ Bg[:N].T, Ar @ Bg[N:].T
+            ref.append(gt / (1 + np.exp(-gt)) * up)
+        else:
+            ref.append(Ar @ Bg.T)
+        got.append(f64(C[torch.from_numpy(r).to(DEV)]))
+    got, ref = np.concatenate(got), np.concatenate(ref)
+    err = rel_fro(got, ref)
+    assert err < 2e-3, err
+    assert torch.all(C[sum(sizes):] == 7.0)
