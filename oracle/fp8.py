@@ -18,6 +18,14 @@ Readings (the pages leave these open):
   * the intermediate h = silu(gate) * up is rounded to fp32 and quantised per
     row per 128 columns before the down projection;
   * the router stays in bf16; the shared expert runs in FP8 like the others.
+
+MX variant (pow2=True): the same groups (1x128 per token, 128x128 per weight
+block), but each scale is the smallest power of two s = 2^p with
+448 * s >= amax (s = 1 when amax = 0; 2^-127 <= s <= 2^127, the range of an
+8-bit exponent), so that the tensor core can apply it as a UE8M0 block
+scale ([MegaMoE] §5.1 folds the scales into the GEMM; with power-of-two
+scales the MMA does it in hardware).  q = E4M3(fp32(a / s)) as before; a / s
+is exact in fp32.  The GEMM is the same blockwise sum, with these scales.
 """
 from __future__ import annotations
 
@@ -26,7 +34,7 @@ import numpy as np
 from .moe_oracle import as_f64, bf16_round, route
 
 __all__ = [
-    "E4M3_MAX", "e4m3_magnitudes", "e4m3_decode", "e4m3_encode", "quantize_1x128",
+    "E4M3_MAX", "e4m3_magnitudes", "e4m3_decode", "e4m3_encode", "pow2_scale_of", "quantize_1x128",
     "quantize_128x128", "dequantize_1x128", "dequantize_128x128", "fp8_gemm",
     "swiglu_ffn_fp8", "quantize_expert", "moe_forward_fp8",
 ]
@@ -76,26 +84,45 @@ def _scale_of(amax32: np.ndarray) -> np.ndarray:
     return np.where(amax32 == 0, np.float32(1.0), s).astype(np.float32)
 
 
-def quantize_1x128(a) -> tuple[np.ndarray, np.ndarray]:
-    """Per row, per 128-column group: (codes [M, K], scales [M, K/128] fp32)."""
+def pow2_scale_of(amax32) -> np.ndarray:
+    """Smallest power of two s = 2^p with 448 * s >= amax (exact comparisons in
+    fp64), p clamped to the UE8M0 exponent range [-127, 127]; s = 1 for amax = 0."""
+    amax = np.asarray(amax32, dtype=np.float32).astype(np.float64)
+    safe = np.where(amax > 0, amax, E4M3_MAX)
+    p = np.ceil(np.log2(safe / E4M3_MAX)).astype(np.int64)
+    # log2 is rounded: settle p by exact comparisons against 448 * 2^p
+    p = np.where(np.ldexp(E4M3_MAX, p) < safe, p + 1, p)
+    p = np.where(np.ldexp(E4M3_MAX, p - 1) >= safe, p - 1, p)
+    p = np.clip(np.where(amax > 0, p, 0), -127, 127)
+    return np.ldexp(np.float64(1.0), p).astype(np.float32)
+
+
+def quantize_1x128(a, pow2: bool = False) -> tuple[np.ndarray, np.ndarray]:
+    """Per row, per 128-column group: (codes [M, K], scales [M, K/128] fp32).
+
+    pow2: power-of-two (MX) scales instead of amax/448."""
     a = np.asarray(a, dtype=np.float32)
     M, K = a.shape
     if K % 128:
         raise ValueError("K must be a multiple of 128")
     g = a.reshape(M, K // 128, 128)
-    s = _scale_of(np.abs(g).max(axis=2))
+    amax = np.abs(g).max(axis=2)
+    s = pow2_scale_of(amax) if pow2 else _scale_of(amax)
     q = e4m3_encode((g / s[:, :, None]).astype(np.float32))
     return q.reshape(M, K), s
 
 
-def quantize_128x128(W) -> tuple[np.ndarray, np.ndarray]:
-    """Per 128x128 block: (codes [N, K], scales [N/128, K/128] fp32)."""
+def quantize_128x128(W, pow2: bool = False) -> tuple[np.ndarray, np.ndarray]:
+    """Per 128x128 block: (codes [N, K], scales [N/128, K/128] fp32).
+
+    pow2: power-of-two (MX) scales instead of amax/448."""
     W = np.asarray(W, dtype=np.float32)
     N, K = W.shape
     if N % 128 or K % 128:
         raise ValueError("N and K must be multiples of 128")
     b = W.reshape(N // 128, 128, K // 128, 128)
-    s = _scale_of(np.abs(b).max(axis=(1, 3)))
+    amax = np.abs(b).max(axis=(1, 3))
+    s = pow2_scale_of(amax) if pow2 else _scale_of(amax)
     q = e4m3_encode((b / s[:, None, :, None]).astype(np.float32))
     return q.reshape(N, K), s
 
@@ -127,26 +154,26 @@ def fp8_gemm(qa, sa, qb, sb) -> np.ndarray:
     return C
 
 
-def swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2) -> dict:
-    """SiLU-gated FFN on quantised operands; h is re-quantised 1x128."""
+def swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2, pow2: bool = False) -> dict:
+    """SiLU-gated FFN on quantised operands; h is re-quantised 1x128 (power-of-two scales with pow2)."""
     I = W1q.shape[0] // 2
     gu = fp8_gemm(xq, sx, W1q, s1)
     g, u = gu[:, :I], gu[:, I:]
     h = g / (1.0 + np.exp(-g)) * u
-    hq, sh = quantize_1x128(h.astype(np.float32))
+    hq, sh = quantize_1x128(h.astype(np.float32), pow2)
     return dict(h=h, hq=hq, sh=sh, y=fp8_gemm(hq, sh, W2q, s2))
 
 
-def quantize_expert(W1e, W2e) -> tuple:
+def quantize_expert(W1e, W2e, pow2: bool = False) -> tuple:
     """One expert's weights (bf16 values) quantised per 128x128 block: (W1q, s1, W2q, s2)."""
-    W1q, s1 = quantize_128x128(as_f64(W1e))
-    W2q, s2 = quantize_128x128(as_f64(W2e))
+    W1q, s1 = quantize_128x128(as_f64(W1e), pow2)
+    W2q, s2 = quantize_128x128(as_f64(W2e), pow2)
     return W1q, s1, W2q, s2
 
 
 def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
                     renormalize: bool = False, tokens=None, idx=None, w=None,
-                    quantized=None, workers: int = 1, capacity: int = 0) -> dict:
+                    quantized=None, workers: int = 1, capacity: int = 0, pow2: bool = False) -> dict:
     """FP8 variant of oracle.moe_forward: same routing, quantised expert GEMMs.
 
     Each expert's W1[e] / W2[e] (bf16 values) is quantised per 128x128 block;
@@ -157,7 +184,8 @@ def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
     with one thread and the weighted outputs are still added in ascending
     expert order, so the result does not depend on `workers`.  `capacity`
     drops the pairs over an expert's capacity exactly as oracle.moe_forward
-    does (kept_mask).
+    does (kept_mask).  pow2 selects the MX variant: every scale (x, the
+    weights, h) is a power of two (pow2_scale_of).
     """
     from .moe_oracle import kept_mask
     if capacity > 0 and tokens is not None:
@@ -172,16 +200,16 @@ def moe_forward_fp8(x, W_r, bias, W1, W2, W1s=None, W2s=None, k: int = 2,
     kept = kept_mask(sel, capacity)
     r["kept"] = kept
     xe = bf16_round(as_f64(xs)).astype(np.float32)
-    xq, sx = quantize_1x128(xe)
+    xq, sx = quantize_1x128(xe, pow2)
     out = np.zeros(xe.shape, dtype=np.float64)
     if W1s is not None:
-        W1q, s1, W2q, s2 = quantize_expert(W1s, W2s)
-        out += swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2)["y"]
+        W1q, s1, W2q, s2 = quantize_expert(W1s, W2s, pow2)
+        out += swiglu_ffn_fp8(xq, sx, W1q, s1, W2q, s2, pow2)["y"]
 
     def expert_rows(e):
         t_rows, slots = np.nonzero((sel == e) & kept)
-        q = quantized[int(e)] if quantized is not None else quantize_expert(W1[int(e)], W2[int(e)])
-        y = swiglu_ffn_fp8(xq[t_rows], sx[t_rows], *q)["y"]
+        q = quantized[int(e)] if quantized is not None else quantize_expert(W1[int(e)], W2[int(e)], pow2)
+        y = swiglu_ffn_fp8(xq[t_rows], sx[t_rows], *q, pow2=pow2)["y"]
         return t_rows, wts[t_rows, slots][:, None] * y
 
     experts = np.unique(sel[kept])
