@@ -87,7 +87,7 @@ def workload_desc(s) -> str:
     parts = [f"{s.name}: T={s.T} d={s.d} E={s.E} top-{s.k} I={s.inter}"]
     if s.shared_inter:
         parts.append(f"+1 shared (I={s.shared_inter})")
-    parts.append("fp8 e4m3 experts" if s.fp8 else "bf16")
+    parts.append(("mx-e4m3 experts (power-of-two scales)" if s.mx else "fp8 e4m3 experts") if s.fp8 else "bf16")
     parts.append(f"Zipf s={s.zipf_s} logit bias" if s.zipf_s else "balanced router")
     return ", ".join(parts)
 
@@ -215,8 +215,8 @@ def make_cfg(gg, s):
     xdt = gg.MOE_F32 if s.x_dtype == "f32" else gg.MOE_BF16
     rdt = gg.MOE_F32 if s.router_dtype == "f32" else gg.MOE_BF16
     odt = gg.MOE_F32 if s.x_dtype == "f32" else gg.MOE_BF16
-    return gg.make_config(s.T, s.d, s.E, s.k, s.inter, s.shared_inter, xdt, rdt,
-                          gg.MOE_E4M3 if s.fp8 else gg.MOE_BF16, odt, s.renormalize)
+    edt = (gg.MOE_MXE4M3 if s.mx else gg.MOE_E4M3) if s.fp8 else gg.MOE_BF16
+    return gg.make_config(s.T, s.d, s.E, s.k, s.inter, s.shared_inter, xdt, rdt, edt, odt, s.renormalize)
 
 
 HOLD_CYCLES = 2_000_000  # ~1 ms spin queued ahead of each timed step
@@ -398,10 +398,11 @@ class OracleRunner:
             need = np.unique(o.route(xs, self.inp["W_r"], self.inp["bias"], s.k)["idx"])
             self.W1.stage(need)
             self.W2.stage(need)
+        kw = dict(pow2=s.mx) if s.fp8 else {}
         fwd = o.moe_forward_fp8 if s.fp8 else o.moe_forward
         t0 = time.perf_counter()
         fwd(xs, self.inp["W_r"], self.inp["bias"], self.W1, self.W2, self.W1s, self.W2s, k=s.k,
-            renormalize=s.renormalize)
+            renormalize=s.renormalize, **kw)
         return time.perf_counter() - t0
 
     def describe(self, batches, spent) -> str:
@@ -434,12 +435,13 @@ def prepare(gg, s, dev, seed):
     cfg = make_cfg(gg, s)
     ws = torch.empty(gg.workspace_size(cfg) + gg.host_staging_size(cfg), dtype=torch.uint8, device=dev)
     if s.fp8:  # weights quantised once per 128x128 block (offline, outside the timed region)
-        W1q, W1sc = gg.quantize_weights_fp8(inp["W1"])
-        W2q, W2sc = gg.quantize_weights_fp8(inp["W2"])
+        quant = gg.quantize_weights_mx if s.mx else gg.quantize_weights_fp8
+        W1q, W1sc = quant(inp["W1"])
+        W2q, W2sc = quant(inp["W2"])
         weights = gg.ExpertWeights(W1=W1q, W2=W2q, W1_scales=W1sc, W2_scales=W2sc)
         if s.shared_inter:
-            weights.W1s, weights.W1s_scales = gg.quantize_weights_fp8(inp["W1s"])
-            weights.W2s, weights.W2s_scales = gg.quantize_weights_fp8(inp["W2s"])
+            weights.W1s, weights.W1s_scales = quant(inp["W1s"])
+            weights.W2s, weights.W2s_scales = quant(inp["W2s"])
     else:
         weights = gg.ExpertWeights(W1=inp["W1"], W2=inp["W2"], W1s=inp["W1s"], W2s=inp["W2s"])
     out = torch.empty((s.T, s.d), dtype=torch.bfloat16 if s.x_dtype != "f32" else torch.float32, device=dev)
@@ -518,7 +520,8 @@ def layer_report(s, r, peaks, peak_kind, world):
     gemm_tf = s.gemm_flops() / (gemm_us * 1e-6) / 1e12
     tensor_peak = float(peaks["bf16_tflops"]) * (2.0 if s.fp8 else 1.0)
     c = r["counts"]
-    rep = {"workload": workload_desc(s), "tokens_per_step": T, "dtype": "e4m3" if s.fp8 else "bf16",
+    rep = {"workload": workload_desc(s), "tokens_per_step": T,
+           "dtype": ("mx-e4m3" if s.mx else "e4m3") if s.fp8 else "bf16",
            "ms_per_step": round(r["ms"], 4), "value": round(job_tokens_per_s(T, world, r["ms"]), 1),
            "unit": "tokens/s",
            # grouped-GEMM FLOP over the two GEMM kernels' own time, against the dense tensor peak
@@ -536,7 +539,7 @@ def layer_report(s, r, peaks, peak_kind, world):
     return rep
 
 
-SIDE_WORKLOADS = ("fine", "fine_skew", "fine_fp8", "fine_fp8_skew", "decode", "tiny")
+SIDE_WORKLOADS = ("fine", "fine_skew", "fine_fp8", "fine_fp8_skew", "fine_mx", "fine_mx_skew", "decode", "tiny")
 
 
 def main():

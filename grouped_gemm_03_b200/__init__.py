@@ -21,12 +21,13 @@ __all__ = [
     "router_topk", "topk_logits", "permute", "grouped_gemm", "combine", "quantize_weights_fp8",
     "capacity_from_factor",
     "workspace_size", "moe_forward", "moe_forward_marked", "moe_forward_host", "host_staging_size", "read_device_status",
-    "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "EPI_NONE", "EPI_SILU_GATE",
+    "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "MOE_MXE4M3", "EPI_NONE", "EPI_SILU_GATE",
+    "quantize_weights_mx",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
-MOE_F32, MOE_F16, MOE_BF16, MOE_E4M3 = 0, 1, 2, 3
+MOE_F32, MOE_F16, MOE_BF16, MOE_E4M3, MOE_MXE4M3 = 0, 1, 2, 3, 4
 EPI_NONE, EPI_SILU_GATE = 0, 1
 _STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WORKSPACE",
            -4: "MOE_ERR_CUDA", -5: "MOE_ERR_BAD_OFFSETS", -6: "MOE_ERR_TIMEOUT"}
@@ -73,6 +74,7 @@ _SIGS = {
     "moe_selftest_workspace_size": (_sz, []),
     "moe_selftest_stalled_pipeline": (_i, [_vp, _sz, ctypes.c_ulonglong, _vp]),
     "moe_quantize_weights_fp8": (_i, [_vp, _i, _i, _i, _vp, _fp, _vp]),
+    "moe_quantize_weights_mx": (_i, [_vp, _i, _i, _i, _vp, _fp, _vp]),
     "moe_workspace_size": (_sz, [_CFG]),
     "moe_forward": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _ip, _vp, _sz, _vp]),
     "moe_forward_marked": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _ip, _vp, _sz,
@@ -190,8 +192,9 @@ def topk_logits(logits, k: int, renormalize: bool = False, out_idx=None, out_w=N
 
 # ---------------------------------------------------------------- permute
 def permute(x, topk_idx, E: int, append_shared: bool = False, fp8: bool = False, ws=None, stream=None,
-            capacity: int = 0) -> dict:
-    """Histogram, scan and scatter (moe_permute; moe_permute_capacity when capacity > 0)."""
+            capacity: int = 0, mx: bool = False) -> dict:
+    """Histogram, scan and scatter (moe_permute; moe_permute_capacity when capacity > 0).
+    fp8: E4M3 rows with 1x128 scales (mx: power-of-two scales)."""
     _cuda(x, topk_idx)
     T, d = x.shape
     k = topk_idx.shape[1]
@@ -208,36 +211,43 @@ def permute(x, topk_idx, E: int, append_shared: bool = False, fp8: bool = False,
         ws = _scratch(L.moe_permute_workspace_size(T, E), dev)
     if capacity:
         _check(L.moe_permute_capacity(_ptr(x), _dt(x), _ptr(topk_idx), T, d, E, k, int(append_shared), int(capacity),
-                                      MOE_E4M3 if fp8 else MOE_BF16, _ptr(xp), _ptr(xps), _ptr(counts),
+                                      (MOE_MXE4M3 if mx else MOE_E4M3) if fp8 else MOE_BF16, _ptr(xp), _ptr(xps),
+                                      _ptr(counts),
                                       _ptr(offsets), _ptr(r2t), _ptr(t2r), _ptr(ws), ws.numel(), _stream(stream)),
                "moe_permute_capacity")
     else:
         _check(L.moe_permute(_ptr(x), _dt(x), _ptr(topk_idx), T, d, E, k, int(append_shared),
-                             MOE_E4M3 if fp8 else MOE_BF16, _ptr(xp), _ptr(xps), _ptr(counts), _ptr(offsets),
+                             (MOE_MXE4M3 if mx else MOE_E4M3) if fp8 else MOE_BF16, _ptr(xp), _ptr(xps),
+                             _ptr(counts), _ptr(offsets),
                              _ptr(r2t), _ptr(t2r), _ptr(ws), ws.numel(), _stream(stream)), "moe_permute")
     return dict(xp=xp, xp_scales=xps, counts=counts, offsets=offsets, row_to_token=r2t, token_to_row=t2r, ws=ws)
 
 
 # ---------------------------------------------------------------- grouped GEMM
 def grouped_gemm(A, B, offsets, N: int, epilogue: int = EPI_NONE, c_dtype=torch.bfloat16, A_scales=None,
-                 B_scales=None, out=None, out_scales=None, ws=None, stream=None):
-    """C [rows, N] for groups offsets[g]..offsets[g+1] of A against B[g] ([G, Nb, K])."""
+                 B_scales=None, out=None, out_scales=None, ws=None, stream=None, mx: bool = False):
+    """C [rows, N] for groups offsets[g]..offsets[g+1] of A against B[g] ([G, Nb, K]).
+
+    E4M3 operands are uint8 codes with fp32 scales; mx=True says the scales are
+    powers of two (MOE_MXE4M3: applied by the tensor core), and an E4M3 C then
+    gets power-of-two scales too."""
     _cuda(A, B, offsets, A_scales, B_scales)
     rows, K = A.shape
     G = B.shape[0]
     fp8 = A.dtype in (torch.uint8, torch.float8_e4m3fn)
-    cdt = {torch.bfloat16: MOE_BF16, torch.float32: MOE_F32, torch.uint8: MOE_E4M3}[c_dtype]
+    q8 = MOE_MXE4M3 if mx else MOE_E4M3
+    cdt = {torch.bfloat16: MOE_BF16, torch.float32: MOE_F32, torch.uint8: q8}[c_dtype]
     C = out if out is not None else torch.empty((rows, N), dtype=c_dtype, device=A.device)
     Cs = out_scales
-    if cdt == MOE_E4M3 and Cs is None:
+    if cdt == q8 and Cs is None:
         Cs = torch.empty((N // 128, rows), dtype=torch.float32, device=A.device)
     L = lib()
     if ws is None:
         ws = _scratch(L.moe_grouped_gemm_workspace_size(), A.device)
     _check(L.moe_grouped_gemm(_ptr(A), _ptr(A_scales), _ptr(B), _ptr(B_scales), _ptr(offsets), G, rows, N, K,
-                              MOE_E4M3 if fp8 else MOE_BF16, epilogue, _ptr(C), cdt, _ptr(Cs), _ptr(ws), ws.numel(),
+                              q8 if fp8 else MOE_BF16, epilogue, _ptr(C), cdt, _ptr(Cs), _ptr(ws), ws.numel(),
                               _stream(stream)), "moe_grouped_gemm")
-    return (C, Cs) if cdt == MOE_E4M3 else C
+    return (C, Cs) if cdt == q8 else C
 
 
 # ---------------------------------------------------------------- combine
@@ -277,6 +287,19 @@ def quantize_weights_fp8(W, stream=None):
     s = torch.empty((G, N // 128, K // 128), dtype=torch.float32, device=W.device)
     _check(lib().moe_quantize_weights_fp8(_ptr(W3), G, N, K, _ptr(q), _ptr(s), _stream(stream)),
            "moe_quantize_weights_fp8")
+    return (q[0], s[0]) if squeeze else (q, s)
+
+
+def quantize_weights_mx(W, stream=None):
+    """As quantize_weights_fp8, with power-of-two block scales (MOE_MXE4M3)."""
+    _cuda(W)
+    squeeze = W.dim() == 2
+    W3 = W.unsqueeze(0) if squeeze else W
+    G, N, K = W3.shape
+    q = torch.empty((G, N, K), dtype=torch.uint8, device=W.device)
+    s = torch.empty((G, N // 128, K // 128), dtype=torch.float32, device=W.device)
+    _check(lib().moe_quantize_weights_mx(_ptr(W3), G, N, K, _ptr(q), _ptr(s), _stream(stream)),
+           "moe_quantize_weights_mx")
     return (q[0], s[0]) if squeeze else (q, s)
 
 

@@ -47,7 +47,34 @@ __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
   return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
+// Scale of a quantisation group with largest magnitude amax.
+//   fp32 scales:  s = amax / 448 (IEEE division), 1 for amax = 0;
+//   MX (pow2):    s = 2^p with p the smallest integer such that 448 * 2^p >= amax,
+//                 clamped to [-127, 127] (an 8-bit exponent carries it), 1 for amax = 0.
+// With amax = (1 + m / 2^23) 2^e and 448 = 1.75 * 2^8: amax / 448 lies in
+// (2^(e-9), 2^(e-8)] when 1 + m / 2^23 <= 1.75 (mantissa bits <= 0x600000),
+// else in (2^(e-8), 2^(e-7)); a subnormal amax gives p below -127.
+__device__ __forceinline__ int pow2_exponent(float amax) {
+  const uint32_t b = __float_as_uint(amax) & 0x7fffffffu;
+  const int ef = static_cast<int>(b >> 23);
+  if (ef == 0) return b ? -127 : 0;
+  const int p = ef - 127 - 8 + ((b & 0x7fffffu) > 0x600000u ? 1 : 0);
+  return p < -127 ? -127 : p;
+}
+__device__ __forceinline__ float pow2_value(int p) {  // 2^p for -127 <= p <= 127
+  return p >= -126 ? __uint_as_float(static_cast<uint32_t>(p + 127) << 23) : __uint_as_float(0x00400000u);
+}
+template <bool kPow2>
+__device__ __forceinline__ float group_scale(float amax) {
+  if constexpr (kPow2) {
+    return amax > 0.f ? pow2_value(pow2_exponent(amax)) : 1.0f;
+  } else {
+    return amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  }
+}
+
 inline size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+inline bool is_e4m3(int dt) { return dt == MOE_E4M3 || dt == MOE_MXE4M3; }
 
 // ---------------------------------------------------------------- launchers
 // Each returns a moe_status; they assume arguments were validated.
@@ -111,7 +138,9 @@ const char* gemm_variant_name(int variant);
 // slots that overflowed an expert's capacity and are skipped.
 int launch_combine(const void* Y, const int32_t* t2r, const float* w, int has_shared, int T, int d, int k,
                    void* out, int out_dtype, cudaStream_t s, const int32_t* shared_base = nullptr);
-int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, cudaStream_t s);
+// pow2: power-of-two (MX) block scales instead of amax / 448
+int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, cudaStream_t s,
+                            bool pow2 = false);
 
 int num_sms();
 

@@ -1365,6 +1365,393 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
   }
 }
 
+// ------------------------------------------------------------------ MX FP8 (block-scaled E4M3) kernel
+// E4M3 operands whose scales are powers of two ("MegaMoE ..." §2.3 / §5.1
+// groups: 1x128 per token, 128x128 per weight block).  The tensor core takes
+// them as UE8M0 block scales (tcgen05.mma kind::mxf8f6f4, one scale per row
+// per 32 K elements), so the whole K reduction of a tile accumulates in TMEM
+// with no promotion step: D = sum_k qa * qb * 2^(ea[m, k/128] + eb[n/128, k/128]).
+// The four 32-wide sub-blocks of a 128-wide K block share one scale, so
+// byte 0 of each scale-factor word serves every MMA of the block.
+//
+// Per k-step (128 K): a TMA thread loads A [128 x 128 B] and B [256 x 128 B];
+// a scale-factor warp writes the step's scale factors into shared memory as
+// 32 x 16-byte atoms (lane i, word c = the scale of row i + 32c, in each of
+// its four bytes): one atom for A's 128 rows, two for B's 256; the MMA
+// thread copies them to TMEM with tcgen05.cp (32x128b.warpx4) and issues
+// four block-scaled MMAs 128 x 256 x 32.  TMEM holds one 256-column fp32
+// accumulator (the scale factors take 12 columns after it), so the epilogue
+// of a tile holds the next tile's MMAs back; the TMA ring keeps loading
+// meanwhile.  Eight epilogue warps read the accumulator (two per TMEM lane
+// quarter, each half of the columns), release it, then convert and store.
+constexpr int kThreadsMX = 352;  // TMA producer, MMA issuer, 8 epilogue warps, scale-factor warp
+constexpr int kMXSfWarp = 10;
+
+template <int EPI>
+struct MXSmem {
+  static constexpr int A_BYTES = BM * 128;
+  static constexpr int B_BYTES = 256 * 128;
+  static constexpr int SF_BYTES = 3 * 512;  // A atom, two B atoms
+  static constexpr int STAGES = 4;
+  static constexpr int SB = STAGES * A_BYTES;                   // B ring
+  static constexpr int SFR = SB + STAGES * B_BYTES;             // scale-factor ring
+  static constexpr int BARS = SFR + STAGES * SF_BYTES;          // barriers and flags
+  static constexpr int TABLES = BARS + 512;                     // group offsets and tile prefix
+  static constexpr int AMAX = TABLES + 2 * (kMaxGroups + 2) * 4;  // [2 parity][2 halves][128 rows]
+  static constexpr int SMEM = AMAX + 2 * 2 * 128 * 4 + 1024;    // + alignment slack
+  static_assert(SMEM <= 227 * 1024, "shared memory budget");
+};
+
+// The UE8M0 byte of a power-of-two fp32 scale (2^-127 .. 2^127), repeated in
+// the four bytes of a word.
+__device__ __forceinline__ uint32_t ue8m0_word(float s) {
+  return ((__float_as_uint(s) >> 23) & 0xffu) * 0x01010101u;
+}
+
+template <int EPI, int OUT>  // EPI 1: SiLU gate (OUT 0 bf16 / 2 MX e4m3); EPI 0: OUT 0 bf16
+__global__ void __launch_bounds__(kThreadsMX, 1)
+    gg_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                 const __grid_constant__ CUtensorMap tmBx, const Params p) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
+  using L = MXSmem<EPI>;
+  constexpr int MMA_N = 256;
+  constexpr int OUT_COLS = EPI ? 128 : 256;
+  constexpr uint32_t IDESC = ptx::make_idesc_mx(BM, MMA_N);
+  constexpr uint32_t SFA_COL = 256, SFB_COL = 260;  // TMEM columns of the scale factors
+
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* sA = smem;
+  uint8_t* sB = smem + L::SB;
+  uint8_t* sSF = smem + L::SFR;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::BARS);
+  uint64_t* empty = full + L::STAGES;
+  uint64_t* tfull = empty + L::STAGES;
+  uint64_t* tempty = tfull + 1;
+  uint64_t* drain = tempty + 1;
+  uint64_t* xchg = drain + 1;  // [4]: the two epilogue warps of a lane quarter swap row amax (E4M3 out)
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(xchg + 4);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  int* s_bad = reinterpret_cast<int*>(tmem_slot + 2);
+  int* s_off = reinterpret_cast<int*>(smem + L::TABLES);
+  int* s_tile = s_off + kMaxGroups + 2;
+  float* s_amax = reinterpret_cast<float*>(smem + L::AMAX);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = p.G_total;
+  const int nt = p.N / OUT_COLS;
+
+  if (warp == 0) {
+    for (int g = lane; g <= G; g += 32) s_off[g] = p.offsets ? p.offsets[g] : (g == 0 ? 0 : p.rows);
+    __syncwarp();
+    const int per = (G + 31) / 32;
+    const int g0 = min(G, lane * per), g1 = min(G, g0 + per);
+    int bad = 0, mine = 0;
+    for (int g = g0; g < g1; ++g) {
+      const int m = s_off[g + 1] - s_off[g];
+      if (m < 0) bad = 1;
+      mine += (max(m, 0) + BM - 1) / BM * nt;
+    }
+    int incl = mine;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    int run = incl - mine;
+    for (int g = g0; g < g1; ++g) {
+      s_tile[g] = run;
+      run += (max(s_off[g + 1] - s_off[g], 0) + BM - 1) / BM * nt;
+    }
+    if (lane == 31) s_tile[G] = incl;
+    if (lane == 0 && (s_off[0] != 0 || s_off[G] > p.rows)) bad = 1;
+    bad = __any_sync(0xffffffffu, bad);
+    if (lane == 0) {
+      *s_bad = bad;
+      *abort_flag = 0;
+      if (bad && blockIdx.x == 0) set_status(p.status, MOE_ERR_BAD_OFFSETS);
+    }
+  }
+  __syncthreads();
+  if (*s_bad) return;
+
+  if (warp == 0 && lane == 0) {
+    for (int s = 0; s < L::STAGES; ++s) {
+      ptx::mbar_init(&full[s], 2);  // the TMA bytes and the scale-factor warp
+      ptx::mbar_init(&empty[s], 1);
+    }
+    ptx::mbar_init(tfull, 1);
+    ptx::mbar_init(tempty, 8);  // one arrival per epilogue warp
+    ptx::mbar_init(drain, 1);
+    for (int i = 0; i < 4; ++i) ptx::mbar_init(&xchg[i], 2);
+    ptx::fence_mbar_init();
+    ptx::prefetch_tmap(&tmA);
+    ptx::prefetch_tmap(&tmB);
+    ptx::prefetch_tmap(&tmBx);
+  }
+  if (warp == 1) {
+    ptx::tmem_alloc(tmem_slot, 512);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const int total = s_tile[G];
+  const int nk = p.K / 128;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ TMA producer
+      uint32_t stage = 0, phase = 0, issued = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+        const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+        const int g = tc.g, nb = tc.nb;
+        const int a_row = s_off[g] + tc.mb * BM;
+        const bool extra = g >= p.G_main;
+        const CUtensorMap* mB = extra ? &tmBx : &tmB;
+        const int gb = extra ? 0 : g;
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
+          ptx::tma_load_2d(sA + stage * L::A_BYTES, &tmA, &full[stage], kb * 128, a_row);
+          if (EPI) {
+            const int brow = gb * 2 * p.N + nb * 128;
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, brow);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES + 128 * 128, mB, &full[stage], kb * 128, brow + p.N);
+          } else {
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, gb * p.N + nb * 256);
+          }
+          ++issued;
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        const uint32_t pending = issued < static_cast<uint32_t>(L::STAGES) ? issued : L::STAGES;
+        uint32_t s2 = stage, ph = phase;
+        for (uint32_t i = 0; i < pending; ++i) {
+          if (s2 == 0) {
+            s2 = L::STAGES - 1;
+            ph ^= 1;
+          } else {
+            --s2;
+          }
+          ptx::mbar_wait(&full[s2], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+        }
+      }
+    }
+  } else if (warp == kMXSfWarp) {
+    // -------------------------------------------------------------- scale-factor warp
+    // Lane i writes word c of row i of each atom: A's scale of tile row i + 32c,
+    // and B's scale of its 128-row weight block (one value per atom).
+    uint32_t stage = 0, phase = 0;
+    bool ok = true;
+    const size_t rstride = static_cast<size_t>(p.rows);
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+      const int g = tc.g, nb = tc.nb;
+      const int a_row = s_off[g] + tc.mb * BM;
+      const float* bsc = g >= p.G_main ? p.Bx_scales
+                                       : p.B_scales + static_cast<size_t>(g) * ((EPI ? 2 : 1) * p.N / 128) * nk;
+      const float* sb0 = bsc + static_cast<size_t>(EPI ? nb : 2 * nb) * nk;          // gate / first half
+      const float* sb1 = bsc + static_cast<size_t>(EPI ? p.N / 128 + nb : 2 * nb + 1) * nk;  // up / second half
+      int rowc[4];
+#pragma unroll
+      for (int c = 0; c < 4; ++c) rowc[c] = min(a_row + lane + 32 * c, p.rows - 1);  // rows past A: any value
+      for (int kb = 0; kb < nk; ++kb) {
+        float sa[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) sa[c] = __ldg(p.A_scales + kb * rstride + rowc[c]);
+        const float b0 = __ldg(sb0 + kb), b1 = __ldg(sb1 + kb);
+        if (!ptx::mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        uint8_t* sf = sSF + stage * L::SF_BYTES;
+        *reinterpret_cast<uint4*>(sf + lane * 16) =
+            make_uint4(ue8m0_word(sa[0]), ue8m0_word(sa[1]), ue8m0_word(sa[2]), ue8m0_word(sa[3]));
+        const uint32_t w0 = ue8m0_word(b0), w1 = ue8m0_word(b1);
+        *reinterpret_cast<uint4*>(sf + 512 + lane * 16) = make_uint4(w0, w0, w0, w0);
+        *reinterpret_cast<uint4*>(sf + 1024 + lane * 16) = make_uint4(w1, w1, w1, w1);
+        ptx::fence_proxy_async_smem();  // visible to tcgen05.cp (async proxy)
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&full[stage]);
+        if (++stage == L::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      set_status(p.status, MOE_ERR_TIMEOUT);
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      uint32_t stage = 0, phase = 0;
+      bool ok = true;
+      int it = 0;
+      const uint32_t sfa = tmem_base + SFA_COL, sfb = tmem_base + SFB_COL;
+      for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x, ++it) {
+        if (!ptx::mbar_wait(tempty, (static_cast<uint32_t>(it) & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+          ok = false;
+          break;
+        }
+        ptx::tc_fence_after();
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!ptx::mbar_wait(&full[stage], phase, abort_flag, kWaitLimitNs)) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          const uint32_t sf = ptx::smem_u32(sSF + stage * L::SF_BYTES);
+          ptx::tmem_cp_32x128b_warpx4(sfa, ptx::plain_16B_rows_desc(sf));
+          ptx::tmem_cp_32x128b_warpx4(sfb, ptx::plain_16B_rows_desc(sf + 512));
+          ptx::tmem_cp_32x128b_warpx4(sfb + 4, ptx::plain_16B_rows_desc(sf + 1024));
+          const uint64_t adesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sA + stage * L::A_BYTES));
+          const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sB + stage * L::B_BYTES));
+#pragma unroll
+          for (int kk = 0; kk < 4; ++kk)
+            ptx::umma_mxf8(tmem_base, adesc + 2 * kk, bdesc + 2 * kk, IDESC, sfa, sfb, (kb | kk) != 0);
+          ptx::umma_commit(&empty[stage]);
+          if (++stage == L::STAGES) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        ptx::umma_commit(tfull);
+      }
+      if (!ok) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+      }
+      ptx::umma_commit(drain);
+      ptx::mbar_wait(drain, 0, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+    }
+  } else {
+    // -------------------------------------------------------------- epilogue (warps 2..9)
+    const int q = warp & 3;         // TMEM lane quarter this warp may access
+    const int hf = (warp - 2) >> 2;  // which half of the tile's columns
+    const int row_t = q * 32 + lane;
+    const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
+      const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+      const int g = tc.g, nb = tc.nb;
+      const int r_in = tc.mb * BM + row_t;
+      const bool valid = r_in < tc.m_g;
+      const size_t grow = static_cast<size_t>(s_off[g] + r_in);
+      if (!ptx::mbar_wait_warp(tfull, static_cast<uint32_t>(it) & 1, abort_flag, kWaitLimitNs)) {
+        *abort_flag = 1;
+        set_status(p.status, MOE_ERR_TIMEOUT);
+        break;
+      }
+      ptx::tc_fence_after();
+      if constexpr (EPI == 1) {
+        // gate columns [64 hf, 64 hf + 64) and the matching up columns 128 + ...
+        float h[64];
+#pragma unroll
+        for (int c = 0; c < 64; c += 32) {
+          uint32_t gv[32], uv[32];
+          ptx::tmem_ld_32x32b_x32(lane_base + 64 * hf + c, gv);
+          ptx::tmem_ld_32x32b_x32(lane_base + 128 + 64 * hf + c, uv);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 32; ++i) h[c + i] = silu(__uint_as_float(gv[i])) * __uint_as_float(uv[i]);
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(tempty);  // the values are in registers: release the accumulator
+        if constexpr (OUT == 2) {
+          // E4M3 with one power-of-two scale per row per 128 columns: the two halves exchange amax
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 64; ++i) amax = fmaxf(amax, fabsf(h[i]));
+          float* xa = s_amax + (it & 1) * 256;  // by tile parity: a slot is rewritten only after both read it
+          xa[hf * 128 + row_t] = amax;
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&xchg[q]);
+          if (!ptx::mbar_wait_warp(&xchg[q], static_cast<uint32_t>(it) & 1, abort_flag, kWaitLimitNs)) {
+            *abort_flag = 1;
+            set_status(p.status, MOE_ERR_TIMEOUT);
+            break;
+          }
+          amax = fmaxf(amax, xa[(hf ^ 1) * 128 + row_t]);
+          const float sc = group_scale<true>(amax);
+          uint32_t qw[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const uint16_t lo = f32x2_to_e4m3x2(__fdiv_rn(h[4 * i], sc), __fdiv_rn(h[4 * i + 1], sc));
+            const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(h[4 * i + 2], sc), __fdiv_rn(h[4 * i + 3], sc));
+            qw[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
+          }
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.C) + grow * p.N + nb * 128 + hf * 64);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) dst[v] = make_uint4(qw[4 * v], qw[4 * v + 1], qw[4 * v + 2], qw[4 * v + 3]);
+            if (hf == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
+          }
+        } else {
+          if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 128 + hf * 64);
+#pragma unroll
+            for (int v = 0; v < 8; ++v) {
+              uint32_t pk[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(h[8 * v + 2 * i], h[8 * v + 2 * i + 1]);
+                pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
+              }
+              dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
+            }
+          }
+        }
+      } else {
+        // columns [128 hf, 128 hf + 128) as bf16
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 32) {
+          uint32_t v[32];
+          ptx::tmem_ld_32x32b_x32(lane_base + 128 * hf + c, v);
+          ptx::tmem_ld_wait();
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+            pk[c / 2 + i] = *reinterpret_cast<const uint32_t*>(&hb);
+          }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(tempty);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 256 + hf * 128);
+#pragma unroll
+          for (int v = 0; v < 16; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
+        }
+      }
+    }
+  }
+
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem_base, 512);
+  }
+}
+
 // ------------------------------------------------------------------ host side
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
@@ -1624,6 +2011,41 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
                     p);
 }
 
+
+template <int EPI, int OUT>
+int run_mx(const GemmArgs& a, cudaStream_t s) {
+  constexpr int kSmem = MXSmem<EPI>::SMEM;
+  const int nb_rows = EPI ? 2 * a.N : a.N;
+  const uint32_t box_b = EPI ? 128 : 256;
+  CUtensorMap mA, mB, mBx;
+  if (!make_map(&mA, a.A, 1, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
+  if (!make_map(&mB, a.B, 1, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 1, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  static bool attr_set[64] = {};
+  int dev = 0;
+  MOE_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  if (!attr_set[dev]) {
+    MOE_CUDA_CHECK(cudaFuncSetAttribute(gg_mx_kernel<EPI, OUT>, cudaFuncAttributeMaxDynamicSharedMemorySize, kSmem));
+    attr_set[dev] = true;
+  }
+  Params p{};
+  p.offsets = a.offsets;
+  p.G_total = a.G + a.has_extra;
+  p.G_main = a.G;
+  p.N = a.N;
+  p.K = a.K;
+  p.rows = a.rows;
+  p.ksplit = 1;
+  p.C = a.C;
+  p.status = a.status;
+  p.A_scales = a.A_scales;
+  p.B_scales = a.B_scales;
+  p.Bx_scales = a.has_extra ? a.B_extra_scales : a.B_scales;
+  p.C_scales = a.C_scales;
+  return launch_pdl(__func__, gg_mx_kernel<EPI, OUT>, dim3(num_sms()), dim3(kThreadsMX), kSmem, s, mA, mB, mBx, p);
+}
+
 }  // namespace
 
 // Which kernel a grouped GEMM runs on: decided on the host from shapes alone
@@ -1635,7 +2057,8 @@ enum GemmVariant {
   kPairNone, kPairNoneF32,                    // no epilogue on CTA pairs (bf16 / fp32 out)
   kNone256, kNone128, kNone64,                // single-CTA, bf16 out
   kNone256F32, kNone128F32, kNone64F32,       // single-CTA, fp32 out (router logits, split-K)
-  kFp8GateE4M3, kFp8GateBf16, kFp8None        // E4M3 operands, per-128-K promotion
+  kFp8GateE4M3, kFp8GateBf16, kFp8None,       // E4M3 operands, per-128-K promotion
+  kMxGateE4M3, kMxGateBf16, kMxNone           // E4M3 with power-of-two scales applied by the MMA
 };
 
 int plan_grouped_gemm(const GemmArgs& a, int sms) {
@@ -1669,6 +2092,16 @@ int plan_grouped_gemm(const GemmArgs& a, int sms) {
     if ((want == 0 || want == 256) && a.N % 256 == 0) return out ? kNone256F32 : kNone256;
     if ((want == 0 || want == 128) && a.N % 128 == 0) return out ? kNone128F32 : kNone128;
     if ((want == 0 || want == 64) && a.N % 64 == 0) return out ? kNone64F32 : kNone64;
+    return kUnsupported;
+  }
+  if (a.ab_dtype == MOE_MXE4M3) {
+    if (a.ksplit > 1) return kUnsupported;
+    if (a.epilogue == MOE_EPI_SILU_GATE && a.N % 128 == 0) {
+      if (a.c_dtype == MOE_MXE4M3) return kMxGateE4M3;
+      if (a.c_dtype == MOE_BF16) return kMxGateBf16;
+      return kUnsupported;
+    }
+    if (a.epilogue == MOE_EPI_NONE && a.N % 256 == 0 && a.c_dtype == MOE_BF16) return kMxNone;
     return kUnsupported;
   }
   if (a.ab_dtype == MOE_E4M3) {
@@ -1705,12 +2138,15 @@ const char* gemm_variant_name(int v) {
     case kFp8GateE4M3: return "e4m3 128x256 silu-gate e4m3-out";
     case kFp8GateBf16: return "e4m3 128x256 silu-gate";
     case kFp8None: return "e4m3 128x256";
+    case kMxGateE4M3: return "mx-e4m3 128x256 silu-gate mx-e4m3-out";
+    case kMxGateBf16: return "mx-e4m3 128x256 silu-gate";
+    case kMxNone: return "mx-e4m3 128x256";
     default: return "unknown";
   }
 }
 
 int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
-  if (a.ab_dtype == MOE_E4M3 && (!a.A_scales || !a.B_scales || (a.has_extra && !a.B_extra_scales)))
+  if (is_e4m3(a.ab_dtype) && (!a.A_scales || !a.B_scales || (a.has_extra && !a.B_extra_scales)))
     return MOE_ERR_UNSUPPORTED;
   switch (plan_grouped_gemm(a, num_sms())) {
     case kEmpty: return MOE_OK;
@@ -1730,6 +2166,9 @@ int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s) {
     case kFp8GateE4M3: return a.C_scales ? run_fp8<1, 2>(a, s) : MOE_ERR_INVALID;
     case kFp8GateBf16: return run_fp8<1, 0>(a, s);
     case kFp8None: return run_fp8<0, 0>(a, s);
+    case kMxGateE4M3: return a.C_scales ? run_mx<1, 2>(a, s) : MOE_ERR_INVALID;
+    case kMxGateBf16: return run_mx<1, 0>(a, s);
+    case kMxNone: return run_mx<0, 0>(a, s);
     default: return MOE_ERR_UNSUPPORTED;
   }
 }

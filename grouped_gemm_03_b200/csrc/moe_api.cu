@@ -41,6 +41,7 @@ size_t dtype_bytes(int dt) {
     case MOE_F16: return 2;
     case MOE_BF16: return 2;
     case MOE_E4M3: return 1;
+    case MOE_MXE4M3: return 1;
     default: return 0;
   }
 }
@@ -59,7 +60,7 @@ FwdLayout fwd_layout(const moe_config& c) {
   };
   const size_t T = c.T, k = c.k, E = c.E, d = c.d, I = c.inter;
   const size_t R = T * k, Rp = R + (c.shared_inter ? T : 0);
-  const bool fp8 = c.expert_dtype == MOE_E4M3;
+  const bool fp8 = is_e4m3(c.expert_dtype);
   const size_t eb = fp8 ? 1 : 2;
   L.status = take(256);
   L.idx = take(T * k * 4);
@@ -87,10 +88,10 @@ int check_config(const moe_config* c) {
   if (c->shared_inter != 0 && c->shared_inter != c->inter) return MOE_ERR_UNSUPPORTED;
   if (c->x_dtype != MOE_F32 && c->x_dtype != MOE_BF16) return MOE_ERR_INVALID;
   if (c->router_dtype != MOE_F32 && c->router_dtype != MOE_BF16) return MOE_ERR_INVALID;
-  if (c->expert_dtype != MOE_BF16 && c->expert_dtype != MOE_E4M3) return MOE_ERR_INVALID;
+  if (c->expert_dtype != MOE_BF16 && !is_e4m3(c->expert_dtype)) return MOE_ERR_INVALID;
   if (c->out_dtype != MOE_F32 && c->out_dtype != MOE_BF16) return MOE_ERR_INVALID;
   if (c->d % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
-  if (c->expert_dtype == MOE_E4M3 && c->d % 256 != 0) return MOE_ERR_UNSUPPORTED;
+  if (is_e4m3(c->expert_dtype) && c->d % 256 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->capacity < 0) return MOE_ERR_INVALID;
   const long long rows = static_cast<long long>(c->T) * (c->k + 1);
   if (rows * c->d > (1ll << 40) || rows > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
@@ -186,11 +187,11 @@ int permute_impl(const void* x, int x_dtype, const int32_t* topk_idx, int T, int
   if (static_cast<long long>(T) * (k + 1) > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
   if (capacity < 0) return MOE_ERR_INVALID;
   if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID;
-  if (xp_dtype != MOE_BF16 && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID;
-  if (d % 8 != 0 || (xp_dtype == MOE_E4M3 && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (xp_dtype != MOE_BF16 && !is_e4m3(xp_dtype)) return MOE_ERR_INVALID;
+  if (d % 8 != 0 || (is_e4m3(xp_dtype) && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;
   if (!counts || !offsets) return MOE_ERR_INVALID;
   if (T > 0 && (!x || !topk_idx || !xp || !row_to_token || !token_to_row)) return MOE_ERR_INVALID;
-  if (T > 0 && xp_dtype == MOE_E4M3 && !xp_scales) return MOE_ERR_INVALID;
+  if (T > 0 && is_e4m3(xp_dtype) && !xp_scales) return MOE_ERR_INVALID;
   if (!aligned(x, 16) || !aligned(xp, 16)) return MOE_ERR_INVALID;
   if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_permute_workspace_size(T, E)) return MOE_ERR_WORKSPACE;
@@ -243,12 +244,13 @@ int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const 
   if (G <= 0 || rows < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID;
   if (G > kMaxGroups) return MOE_ERR_UNSUPPORTED;
   if (!A || !B || !offsets || !C) return MOE_ERR_INVALID;
-  if (ab_dtype != MOE_BF16 && ab_dtype != MOE_E4M3) return MOE_ERR_INVALID;
+  if (ab_dtype != MOE_BF16 && !is_e4m3(ab_dtype)) return MOE_ERR_INVALID;
   if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SILU_GATE) return MOE_ERR_INVALID;
-  if (ab_dtype == MOE_E4M3 && (!A_scales || !B_scales)) return MOE_ERR_INVALID;
-  if (c_dtype == MOE_E4M3 && !C_scales) return MOE_ERR_INVALID;
+  if (is_e4m3(ab_dtype) && (!A_scales || !B_scales)) return MOE_ERR_INVALID;
+  if (is_e4m3(c_dtype) && !C_scales) return MOE_ERR_INVALID;
+  if (is_e4m3(c_dtype) && c_dtype != ab_dtype) return MOE_ERR_UNSUPPORTED;  // h keeps the operands' scale kind
   if (ab_dtype == MOE_BF16 && K % 64 != 0) return MOE_ERR_UNSUPPORTED;
-  if (ab_dtype == MOE_E4M3 && K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (is_e4m3(ab_dtype) && K % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16)) return MOE_ERR_INVALID;
   if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_grouped_gemm_workspace_size()) return MOE_ERR_WORKSPACE;
@@ -352,6 +354,14 @@ int moe_quantize_weights_fp8(const void* W, int G, int N, int K, uint8_t* Wq, fl
   return launch_quantize_weights(W, G, N, K, Wq, scales, as_stream(stream));
 }
 
+int moe_quantize_weights_mx(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, void* stream) {
+  if (G < 0 || N <= 0 || K <= 0) return MOE_ERR_INVALID;
+  if (N % 128 != 0 || K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (G > 0 && (!W || !Wq || !scales)) return MOE_ERR_INVALID;
+  if (!aligned(W, 16) || !aligned(Wq, 16)) return MOE_ERR_INVALID;
+  return launch_quantize_weights(W, G, N, K, Wq, scales, as_stream(stream), true);
+}
+
 // ------------------------------------------------------------------ whole layer
 size_t moe_workspace_size(const moe_config* cfg) {
   if (check_config(cfg) != MOE_OK) return 0;
@@ -369,7 +379,8 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   int st = check_config(cfg);
   if (st != MOE_OK) return st;
   const moe_config c = *cfg;
-  const bool fp8 = c.expert_dtype == MOE_E4M3;
+  const bool fp8 = is_e4m3(c.expert_dtype);
+  const int qdt = c.expert_dtype;  // MOE_E4M3 or MOE_MXE4M3 when fp8
   const bool shared = c.shared_inter != 0;
   if (c.T > 0 && (!x || !W_r || !W1 || !W2 || !out)) return MOE_ERR_INVALID;
   if (shared && (!W1_shared || !W2_shared)) return MOE_ERR_INVALID;
@@ -415,7 +426,7 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   pa.E = E;
   pa.k = k;
   pa.shared = shared ? 1 : 0;
-  pa.xp_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
+  pa.xp_dtype = fp8 ? qdt : MOE_BF16;
   pa.xp = base + L.xp;
   pa.xp_scales = fp8 ? reinterpret_cast<float*>(base + L.xps) : nullptr;
   pa.counts = counts;
@@ -439,9 +450,9 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   up.rows = Rp;
   up.N = I;
   up.K = d;
-  up.ab_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
+  up.ab_dtype = fp8 ? qdt : MOE_BF16;
   up.epilogue = MOE_EPI_SILU_GATE;
-  up.c_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
+  up.c_dtype = fp8 ? qdt : MOE_BF16;
   up.C = base + L.h;
   up.status = status;
   if (fp8) {
@@ -464,7 +475,7 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   dn.rows = Rp;
   dn.N = d;
   dn.K = I;
-  dn.ab_dtype = fp8 ? MOE_E4M3 : MOE_BF16;
+  dn.ab_dtype = fp8 ? qdt : MOE_BF16;
   dn.epilogue = MOE_EPI_NONE;
   dn.c_dtype = MOE_BF16;
   dn.C = base + L.y;

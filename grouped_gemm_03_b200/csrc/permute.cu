@@ -155,7 +155,7 @@ __device__ __forceinline__ void load_row8(const float* p, float (&f)[8]) {
 // kScatterCols) so that even a few hundred tokens keep every SM busy.
 constexpr int kScatterCols = 512;
 
-template <typename XT, bool kFp8>
+template <typename XT, bool kFp8, bool kPow2 = false>
 __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
@@ -281,7 +281,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
       for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
 #pragma unroll
       for (int o = 8; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-      const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+      const float s = group_scale<kPow2>(amax);
       uint32_t q[2];
 #pragma unroll
       for (int i = 0; i < 2; ++i) {
@@ -319,14 +319,18 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
   st = launch_pdl("scan_kernel", scan_kernel, dim3(1), dim3(1024), 0, s, a.block_base, nblk, a.E, a.T, a.shared,
                   a.capacity, a.counts, a.offsets);
   if (st != MOE_OK) return st;
-  const bool fp8 = a.xp_dtype == MOE_E4M3;
+  const bool fp8 = is_e4m3(a.xp_dtype);
+  const bool mx = a.xp_dtype == MOE_MXE4M3;
   const dim3 grid(nblk, (a.d + kScatterCols - 1) / kScatterCols);
   const dim3 block(kPermThreads);
-  if (a.x_dtype == MOE_BF16)
-    return fp8 ? launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true>, grid, block, 0, s, a)
-               : launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, false>, grid, block, 0, s, a);
-  return fp8 ? launch_pdl("scatter_kernel", scatter_kernel<float, true>, grid, block, 0, s, a)
-             : launch_pdl("scatter_kernel", scatter_kernel<float, false>, grid, block, 0, s, a);
+  if (a.x_dtype == MOE_BF16) {
+    if (!fp8) return launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, false>, grid, block, 0, s, a);
+    return mx ? launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true, true>, grid, block, 0, s, a)
+              : launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true>, grid, block, 0, s, a);
+  }
+  if (!fp8) return launch_pdl("scatter_kernel", scatter_kernel<float, false>, grid, block, 0, s, a);
+  return mx ? launch_pdl("scatter_kernel", scatter_kernel<float, true, true>, grid, block, 0, s, a)
+            : launch_pdl("scatter_kernel", scatter_kernel<float, true>, grid, block, 0, s, a);
 }
 
 }  // namespace moe
@@ -437,11 +441,11 @@ extern "C" int moe_permute_noalloc(const void* x, int x_dtype, const int32_t* to
   if (static_cast<size_t>(permute_blocks(T)) * static_cast<size_t>(E) > kNoAllocCountWords)
     return MOE_ERR_UNSUPPORTED;  // beyond the built-in scratch: use moe_permute with a workspace
   if (x_dtype != MOE_F32 && x_dtype != MOE_BF16) return MOE_ERR_INVALID;
-  if (xp_dtype != MOE_BF16 && xp_dtype != MOE_E4M3) return MOE_ERR_INVALID;
-  if (d % 8 != 0 || (xp_dtype == MOE_E4M3 && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;
+  if (xp_dtype != MOE_BF16 && !is_e4m3(xp_dtype)) return MOE_ERR_INVALID;
+  if (d % 8 != 0 || (is_e4m3(xp_dtype) && d % 128 != 0)) return MOE_ERR_UNSUPPORTED;
   if (!counts || !offsets) return MOE_ERR_INVALID;
   if (T > 0 && (!x || !topk_idx || !xp || !row_to_token || !token_to_row)) return MOE_ERR_INVALID;
-  if (T > 0 && xp_dtype == MOE_E4M3 && !xp_scales) return MOE_ERR_INVALID;
+  if (T > 0 && is_e4m3(xp_dtype) && !xp_scales) return MOE_ERR_INVALID;
   if (reinterpret_cast<uintptr_t>(x) % 16 || reinterpret_cast<uintptr_t>(xp) % 16) return MOE_ERR_INVALID;
   int32_t* scratch = nullptr;
   const int st = noalloc_scratch(&scratch);

@@ -203,6 +203,46 @@ __device__ __forceinline__ void umma_f8(uint32_t d_tmem, uint64_t adesc, uint64_
       : "memory");
 }
 
+// Block-scaled 8-bit MMA (kind::mxf8f6f4, one UE8M0 scale per 32 K elements
+// of each row of A and of B): D[tmem] (+)= (A * 2^sfa) (B * 2^sfb)^T, fp32
+// accumulate, K = 32 per instruction.  sfa_tmem / sfb_tmem are the TMEM
+// addresses of the scale factors (written by tcgen05.cp); the scale-factor
+// ids in idesc select which byte of each 32-bit TMEM word is used.
+__device__ __forceinline__ void umma_mxf8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                          uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+      : "memory");
+}
+
+// Copy 32 rows x 128 bits of shared memory (described by `sdesc`) into TMEM
+// lanes [0, 32) x 4 columns at `taddr`, repeated in each of the four 32-lane
+// quarters (the layout the block-scaled MMA reads its scale factors from).
+__device__ __forceinline__ void tmem_cp_32x128b_warpx4(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+// Shared-memory descriptor of a K-major operand without swizzling whose
+// rows are 16 bytes and contiguous (8-row core matrices 128 bytes apart):
+// the 32 x 16-byte scale-factor atoms tcgen05.cp reads.
+__device__ __forceinline__ uint64_t plain_16B_rows_desc(uint32_t smem_addr) {
+  uint64_t d = 0;
+  d |= static_cast<uint64_t>((smem_addr & 0x3FFFFu) >> 4);  // start address  [0,14)
+  d |= static_cast<uint64_t>(128 >> 4) << 16;                // leading offset [16,30)
+  d |= static_cast<uint64_t>(128 >> 4) << 32;                // stride offset  [32,46): next 8 rows
+  d |= static_cast<uint64_t>(1) << 46;                       // descriptor version (tcgen05)
+  return d;                                                  // layout type 0: no swizzle
+}
+
+// Instruction descriptor of the block-scaled MMA: E4M3 A and B (format 0),
+// K-major, UE8M0 scale factors (bit 23), scale-factor ids 0, shape M x N.
+__host__ __device__ constexpr uint32_t make_idesc_mx(int M, int N) {
+  return (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) | (static_cast<uint32_t>(M >> 4) << 24);
+}
+
 // Arrive once on `bar` when every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void umma_commit(uint64_t* bar) {
   asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(

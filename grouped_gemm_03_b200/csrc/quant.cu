@@ -1,12 +1,15 @@
 // Weight quantisation to E4M3 with one fp32 scale per 128x128 block
 // ("MegaMoE ..." §2.3 / §5.1: per-block scaling of the weights).
 //   s = amax(block) / 448  (1 for an all-zero block),  q = e4m3_rn_satfinite(w / s)
+// or, for the MX variant, s = the smallest power of two with 448 s >= amax
+// (group_scale<true>); w / s is then exact before the E4M3 rounding.
 // One CTA per block; each thread owns 64 contiguous elements of one row.
 #include "common.cuh"
 
 namespace moe {
 namespace {
 
+template <bool kPow2>
 __global__ void __launch_bounds__(256) quant_block_kernel(const __nv_bfloat16* __restrict__ W, int N, int K,
                                                           uint8_t* __restrict__ Wq, float* __restrict__ scales) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
@@ -38,7 +41,7 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const __nv_bfloat16* _
   amax = s_max[0];
 #pragma unroll
   for (int i = 1; i < 8; ++i) amax = fmaxf(amax, s_max[i]);
-  const float s = amax > 0.f ? __fdiv_rn(amax, 448.0f) : 1.0f;
+  const float s = group_scale<kPow2>(amax);
   uint4* dst = reinterpret_cast<uint4*>(Wq + off);
 #pragma unroll
   for (int v = 0; v < 4; ++v) {
@@ -58,11 +61,13 @@ __global__ void __launch_bounds__(256) quant_block_kernel(const __nv_bfloat16* _
 
 }  // namespace
 
-int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, cudaStream_t s) {
+int launch_quantize_weights(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, cudaStream_t s,
+                            bool pow2) {
   if (G == 0) return MOE_OK;
   dim3 grid(K / 128, N / 128, G);
-  return launch_pdl(__func__, quant_block_kernel, grid, dim3(256), 0, s, static_cast<const __nv_bfloat16*>(W), N, K, Wq,
-                    scales);
+  const __nv_bfloat16* w = static_cast<const __nv_bfloat16*>(W);
+  return pow2 ? launch_pdl(__func__, quant_block_kernel<true>, grid, dim3(256), 0, s, w, N, K, Wq, scales)
+              : launch_pdl(__func__, quant_block_kernel<false>, grid, dim3(256), 0, s, w, N, K, Wq, scales);
 }
 
 }  // namespace moe

@@ -50,7 +50,14 @@ typedef enum moe_status {
   MOE_ERR_TIMEOUT = -6       /* a kernel pipeline wait exceeded its time limit      */
 } moe_status;
 
-typedef enum moe_dtype { MOE_F32 = 0, MOE_F16 = 1, MOE_BF16 = 2, MOE_E4M3 = 3 } moe_dtype;
+/* MOE_E4M3: E4M3 codes with fp32 scales s = amax/448, one per 128 elements
+ * along K (activations) or per 128x128 block (weights); a GEMM promotes each
+ * 128-wide K block's partial product by its scales ("MegaMoE ..." §2.3, §5.1).
+ * MOE_MXE4M3: the same codes and groups with power-of-two scales, the
+ * smallest 2^p (p in [-127, 127]) with 448 * 2^p >= amax, still stored as
+ * fp32 values; a GEMM hands them to the tensor core as UE8M0 block scales
+ * (tcgen05.mma kind::mxf8f6f4), which applies them itself. */
+typedef enum moe_dtype { MOE_F32 = 0, MOE_F16 = 1, MOE_BF16 = 2, MOE_E4M3 = 3, MOE_MXE4M3 = 4 } moe_dtype;
 
 typedef enum moe_epilogue {
   MOE_EPI_NONE = 0,      /* C = A B^T                                                   */
@@ -59,9 +66,10 @@ typedef enum moe_epilogue {
 
 /* One layer's shape.  x_dtype: MOE_F32 | MOE_BF16.  router_dtype (W_r):
  * MOE_F32 | MOE_BF16 (an fp32 router needs fp32 x).  expert_dtype: MOE_BF16 |
- * MOE_E4M3 (the expert GEMMs run in E4M3 with fp32 scales).  out_dtype:
+ * MOE_E4M3 (the expert GEMMs run in E4M3 with fp32 scales) | MOE_MXE4M3
+ * (E4M3 with power-of-two scales the tensor core applies).  out_dtype:
  * MOE_F32 | MOE_BF16.  shared_inter is 0 (no shared expert) or equal to inter.
- * d and inter are multiples of 128 (E4M3 experts: d a multiple of 256).
+ * d and inter are multiples of 128 (E4M3 / MX experts: d a multiple of 256).
  * renormalize = 0 weights each expert by its softmax value p_i (MegaMoE §2.1);
  * 1 divides by the sum over the selected experts (route_tokens in
  * Dense GEMM -> GroupedGEMM -> TP MoE §4.2).
@@ -129,9 +137,10 @@ int moe_topk_logits(const void* logits, int dtype, int N, int E, int k, int reno
  *   topk_idx     [T, k] int32 in [0, E), distinct within a token
  *   xp_dtype     MOE_BF16 (x rounded to bf16) | MOE_E4M3 (quantised once per
  *                token per 128 columns: s = amax/448, q = e4m3_rn_satfinite(x/s))
+ *                | MOE_MXE4M3 (the same with power-of-two s, see moe_dtype)
  *   xp           [R', d] (R' = R + T if append_shared else R)
  *   xp_scales    [d/128][R'] fp32 (K-block-major: scale of row r, block b at
- *                b*R' + r) when xp_dtype == MOE_E4M3, else NULL
+ *                b*R' + r) when xp_dtype is MOE_E4M3 / MOE_MXE4M3, else NULL
  *   counts       [E] int32; offsets [E+1] (+1 with append_shared): offsets[e]
  *                = sum of counts before e, offsets[E] = R, offsets[E+1] = R+T
  *   row_to_token [R'] int32;  token_to_row [T, k] int32
@@ -197,18 +206,21 @@ int moe_permute_noalloc(const void* x, int x_dtype, const int32_t* topk_idx, int
  * shared N, K; "Dense GEMM -> GroupedGEMM -> TP MoE" §2.3: the
  * grouped_gemm(A_ptrs, B_ptrs, C_ptrs, expert_sizes, N, K, workspace, stream)
  * call, with the pointer arrays replaced by base + device offsets.)
- *   A        [rows, K] ab_dtype (MOE_BF16 | MOE_E4M3), row-major
- *   A_scales [K/128][rows] fp32 (E4M3 only, else NULL)
+ *   A        [rows, K] ab_dtype (MOE_BF16 | MOE_E4M3 | MOE_MXE4M3), row-major
+ *   A_scales [K/128][rows] fp32 (E4M3 / MX only, else NULL)
  *   B        [G, Nb, K] ab_dtype, K-major, Nb = N (NONE) or 2N (SILU_GATE:
  *            rows 0..N-1 gate, N..2N-1 up)
- *   B_scales [G][Nb/128][K/128] fp32 (E4M3 only, else NULL)
+ *   B_scales [G][Nb/128][K/128] fp32 (E4M3 / MX only, else NULL)
  *   offsets  [G+1] int32 DEVICE array, offsets[0] = 0, non-decreasing,
  *            offsets[G] <= rows; checked on the device (MOE_ERR_BAD_OFFSETS,
  *            nothing written)
  *   C        [rows, N] c_dtype: MOE_BF16 | MOE_F32 (NONE, bf16 inputs) or
- *            MOE_BF16 | MOE_E4M3 (SILU_GATE); rows outside every group untouched
- *   C_scales [N/128][rows] fp32 when c_dtype == MOE_E4M3 (per row per 128 columns)
+ *            MOE_BF16 | ab_dtype's E4M3 kind (SILU_GATE); rows outside every group untouched
+ *   C_scales [N/128][rows] fp32 when C is E4M3 (per row per 128 columns)
  *   ws       moe_grouped_gemm_workspace_size() bytes (status word)
+ * MOE_MXE4M3 operands: the power-of-two scales go to the tensor core as
+ * UE8M0 block scales (tcgen05.mma kind::mxf8f6f4), which applies them
+ * itself; an MX C gets power-of-two scales.  Same shape rules as E4M3.
  * E4M3 operands: the scales vary along K, so each 128-wide K block's partial
  * product is scaled by sa[row, kb] * sb[n/128, kb] and accumulated in fp32
  * ("MegaMoE ..." §5.1); an E4M3 C is quantised per row per 128 columns
@@ -264,6 +276,11 @@ int moe_combine_plan(const void* Y, const int32_t* token_to_row, const float* to
  * N % 128 == 0, K % 128 == 0. */
 int moe_quantize_weights_fp8(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, void* stream);
 
+/* As moe_quantize_weights_fp8, with power-of-two block scales (MOE_MXE4M3):
+ * s = the smallest 2^p with 448 * 2^p >= amax(block), p in [-127, 127]
+ * (1 if the block is zero); w / s is exact, then rounded to E4M3. */
+int moe_quantize_weights_mx(const void* W, int G, int N, int K, uint8_t* Wq, float* scales, void* stream);
+
 /* ---------------------------------------------------------------- whole layer
  * moe_forward runs the whole layer: router, permute, up grouped GEMM with the
  * SiLU-gate epilogue, down grouped GEMM, combine.  The shared expert (if
@@ -271,6 +288,7 @@ int moe_quantize_weights_fp8(const void* W, int G, int N, int K, uint8_t* Wq, fl
  *   x [T, d] cfg->x_dtype;  W_r [E, d] cfg->router_dtype;  router_bias [E] or NULL
  *   BF16 experts: W1 [E, 2I, d], W2 [E, d, I] bf16, *_scales NULL
  *   E4M3 experts: W1/W2 as moe_quantize_weights_fp8 output with their scales
+ *   MX experts:   W1/W2 as moe_quantize_weights_mx output with their scales
  *   W1_shared [2I, d], W2_shared [d, I] (+ scales) or NULL
  *   out [T, d] cfg->out_dtype;  counts_out [E] int32 (rows each expert took:
  *       its tokens, or at most cfg->capacity of them) or NULL

@@ -46,6 +46,7 @@ class MoEShape:
     x_dtype: str = "bf16"   # "f32" | "bf16"
     router_dtype: str = "bf16"
     fp8: bool = False       # expert GEMMs in E4M3 with 1x128 / 128x128 scales
+    mx: bool = False        # with fp8: power-of-two (MX) scales the tensor core applies
     zipf_s: float = 0.0     # 0 = balanced router
     renormalize: bool = False
 
@@ -76,6 +77,11 @@ CONFIGS: dict[str, MoEShape] = {
                          fp8=True),
     "fine_fp8_skew": MoEShape("fine_fp8_skew", T=4096, d=7168, E=256, k=8, inter=2048,
                               shared_inter=2048, fp8=True, zipf_s=1.2),
+    # the same FP8 layers with power-of-two (MX) scales
+    "fine_mx": MoEShape("fine_mx", T=4096, d=7168, E=256, k=8, inter=2048, shared_inter=2048,
+                        fp8=True, mx=True),
+    "fine_mx_skew": MoEShape("fine_mx_skew", T=4096, d=7168, E=256, k=8, inter=2048,
+                             shared_inter=2048, fp8=True, mx=True, zipf_s=1.2),
     "decode": MoEShape("decode", T=128, d=2048, E=64, k=2, inter=1408, zipf_s=1.5),
 }
 
