@@ -53,7 +53,6 @@ from workload.gen import ROUTER_MICRO  # noqa: E402
 
 METRIC = "MoE-layer tokens/s at 1 B200; grouped-GEMM TFLOP/s as % of dense tensor peak"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNELS_PER_FORWARD = 8  # router logits, top-k, hist, scan, scatter, up GEMM, down GEMM, combine
 
 
 def log(*a):
@@ -594,7 +593,7 @@ def main():
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)", "config": config_block(s),
             "gemm_tflops": rep["gemm_tflops"], "gemm_frac_of_peak": rep["gemm_frac_of_peak"],
             "roofline": rep["roofline"], "kernels": rep["kernels"], "e2e": rep["e2e"], "graph": rep["graph"],
-            "gpu_launches": KERNELS_PER_FORWARD * args.steps, "clocks": rep["clocks"],
+            "gpu_launches": gg.forward_launches(make_cfg(gg, s)) * args.steps, "clocks": rep["clocks"],
             "expert_counts": rep["expert_counts"]}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
             result["cpu_baseline"] = cpu_baseline(s, r["inp"])

@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "LIB_PATH", "MoEError", "MoEConfig", "lib", "exported_symbols", "status_string", "device_info",
     "router_topk", "topk_logits", "permute", "grouped_gemm", "combine", "quantize_weights_fp8",
-    "capacity_from_factor",
+    "capacity_from_factor", "forward_launches",
     "workspace_size", "moe_forward", "moe_forward_marked", "moe_forward_host", "host_staging_size", "read_device_status",
     "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "MOE_MXE4M3", "EPI_NONE", "EPI_SILU_GATE",
     "quantize_weights_mx",
@@ -80,6 +80,7 @@ _SIGS = {
     "moe_forward_marked": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _ip, _vp, _sz,
                                 ctypes.POINTER(ctypes.c_void_p), _vp]),
     "moe_host_staging_size": (_sz, [_CFG]),
+    "moe_forward_launches": (_i, [_CFG]),
     "moe_forward_host": (_i, [_CFG, _vp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _fp, _vp, _vp, _sz, _vp]),
 }
 
@@ -325,6 +326,11 @@ def workspace_size(cfg: MoEConfig) -> int:
 
 def host_staging_size(cfg: MoEConfig) -> int:
     return lib().moe_host_staging_size(ctypes.byref(cfg))
+
+
+def forward_launches(cfg: MoEConfig) -> int:
+    """Kernels one moe_forward of this shape launches (host arithmetic)."""
+    return lib().moe_forward_launches(ctypes.byref(cfg))
 
 
 @dataclass

@@ -85,6 +85,7 @@ int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, cons
                   int k, int renorm, float* logits_out, int32_t* idx, float* w, float* parts, int* status,
                   cudaStream_t s);
 bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E);
+bool router_is_fused(int T, int d, int E);  // one launch (logits + softmax + top-k on chip)
 int router_padded_experts(int E);  // logits columns the tensor-core router computes
 int launch_topk_logits(const void* logits, int dtype, int N, int E, int k, int renorm, int32_t* idx,
                        float* w, cudaStream_t s);

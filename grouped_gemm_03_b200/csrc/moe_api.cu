@@ -518,6 +518,13 @@ int moe_forward_marked(const moe_config* cfg, const void* x, const void* W_r, co
                       W2s_scales, out, counts_out, ws, ws_bytes, stream, stage_events);
 }
 
+int moe_forward_launches(const moe_config* cfg) {
+  if (check_config(cfg) != MOE_OK) return -1;
+  if (cfg->T == 0) return 0;
+  const int router = router_is_fused(cfg->T, cfg->d, cfg->E) ? 1 : 2;  // fused, or logits + selection
+  return router + 3 /* histogram, scan, scatter */ + 2 /* grouped GEMMs */ + 1 /* combine */;
+}
+
 size_t moe_host_staging_size(const moe_config* cfg) {
   if (check_config(cfg) != MOE_OK) return 0;
   const size_t td = static_cast<size_t>(cfg->T) * cfg->d;

@@ -2,7 +2,9 @@
 //
 // "MegaMoE math model -> DeepGEMM source walk-through" §2.1 (p = Softmax(W_r x_t),
 // keep the k best) and "Dense GEMM -> GroupedGEMM -> TP MoE" §4.2 (route_tokens).
-// Two launches:
+// Up to 64 experts with a modest T*d*E: one launch, router_fused_kernel
+// (below), which streams x once and keeps every logit on chip.  Otherwise
+// two launches:
 //   logits  either the grouped-GEMM kernel on the tensor cores (bf16, large
 //           E and d: the logits GEMM is then near the compute ridge), split
 //           along K into fp32 partial products, or a SIMT kernel that keeps
@@ -363,6 +365,228 @@ int finish_dispatch(const void* parts, int nsplit, size_t stride, int pstride, c
   return MOE_ERR_UNSUPPORTED;
 }
 
+// ------------------------------------------------------------------ fused router (E <= 64)
+// One launch: logits, softmax and top-k ("MegaMoE ..." §2.1; the fused
+// logits + softmax kernel of "DeepSeek-R1 deployment on A100" §3.2 and the
+// warp-level top-k of "DeepSeek MoE architecture overview" §2.2).  The
+// logits of a few experts are a short dot product per token, bound by
+// reading x once: a warp takes TPW = 32 / EP tokens at a time (EP = E
+// rounded up to a power of two, at least 8; one token when EP = 64) and its
+// lanes split d into 16-byte chunks, lane l owning chunks l, l + 32, ...;
+// every lane accumulates TPW x EP partial logits in fp32 (packed FMAs), the
+// W_r chunk it needs coming through L1 and reused by the warp's TPW tokens,
+// and the next two chunks of x in flight.  A butterfly reduce-scatter over
+// the lanes leaves lane l with the full logit of (token l / EP, expert
+// l % EP) (EP = 64: experts 2l and 2l + 1 of the warp's one token), and the
+// EP lanes of a token run the softmax and k rounds of an arg-max on packed
+// (logit, ~index) keys, so ties go to the lower expert index.
+constexpr int kFusedWarps = 8;
+
+template <typename T>
+struct Chunk8;  // 8 consecutive elements as raw 16- or 32-byte words
+template <>
+struct Chunk8<__nv_bfloat16> {
+  uint4 w;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { w = __ldg(reinterpret_cast<const uint4*>(p)); }
+  __device__ __forceinline__ void zero() { w = make_uint4(0, 0, 0, 0); }
+  __device__ __forceinline__ float2 pair(int i) const {  // elements 2i, 2i+1
+    const uint32_t u = i == 0 ? w.x : i == 1 ? w.y : i == 2 ? w.z : w.w;
+    return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+  }
+};
+template <>
+struct Chunk8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = __ldg(reinterpret_cast<const float4*>(p));
+    b = __ldg(reinterpret_cast<const float4*>(p) + 1);
+  }
+  __device__ __forceinline__ void zero() { a = b = make_float4(0.f, 0.f, 0.f, 0.f); }
+  __device__ __forceinline__ float2 pair(int i) const {
+    return i == 0 ? make_float2(a.x, a.y) : i == 1 ? make_float2(a.z, a.w) : i == 2 ? make_float2(b.x, b.y)
+                                                                                     : make_float2(b.z, b.w);
+  }
+};
+
+// One level of the butterfly reduce-scatter: lanes with `bit` clear keep the
+// lower half of v[0, S), the others the upper half, each adding the
+// partner's copy of the half it keeps; the kept half moves to v[0, S/2).
+template <int S>
+__device__ __forceinline__ void rs_level(float (&v)[64], int lane, int bit) {
+  const bool up = lane & bit;
+#pragma unroll
+  for (int i = 0; i < S / 2; ++i) {
+    const float send = up ? v[i] : v[S / 2 + i];
+    const float keep = up ? v[S / 2 + i] : v[i];
+    v[i] = keep + __shfl_xor_sync(0xffffffffu, send, bit);
+  }
+}
+
+template <typename XT, typename WT, int EP>
+__global__ void __launch_bounds__(kFusedWarps * 32) router_fused_kernel(const XT* __restrict__ x,
+                                                                      const WT* __restrict__ Wr,
+                                                                      const float* __restrict__ bias, int T, int d,
+                                                                      int E, int k, int renorm,
+                                                                      float* __restrict__ logits_out,
+                                                                      int32_t* __restrict__ idx_out,
+                                                                      float* __restrict__ w_out) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
+  constexpr int TPW = EP >= 32 ? 1 : 32 / EP;
+  constexpr int NV = TPW * EP;          // partial logits per lane: 32, or 64 when EP = 64
+  constexpr int PER = NV / 32;          // logits per lane after the reduce-scatter
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int lane = threadIdx.x & 31;
+  const int nwarps = gridDim.x * kFusedWarps;
+  const int nchunk = d / 8;             // 8-element chunks per row
+  for (int t0 = (blockIdx.x * kFusedWarps + (threadIdx.x >> 5)) * TPW; t0 < T; t0 += nwarps * TPW) {
+    // fp32 sums per (token, expert); with EP <= 32 two running sums (even and
+    // odd columns, packed FMAs) added at the end
+    constexpr bool kPair = NV == 32;
+    float2 acc2[kPair ? NV : 1];
+    float acc[64];
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+      if constexpr (kPair) acc2[i] = make_float2(0.f, 0.f);
+      acc[i] = 0.f;
+    }
+    auto fetch = [&](Chunk8<XT>(&dst)[TPW], int c) {
+#pragma unroll
+      for (int j = 0; j < TPW; ++j) {
+        if (c < nchunk && t0 + j < T)
+          dst[j].load(x + static_cast<size_t>(t0 + j) * d + c * 8);
+        else
+          dst[j].zero();
+      }
+    };
+    // three steps of x in flight per lane: this one, the next and the one after
+    Chunk8<XT> cur[TPW], nxt[TPW];
+    fetch(cur, lane);
+    fetch(nxt, lane + 32);
+    for (int c0 = 0; c0 < nchunk; c0 += 32) {  // warp-uniform trip count
+      const int c = c0 + lane;
+      Chunk8<XT> after[TPW];
+      fetch(after, c + 64);
+#pragma unroll
+      for (int e = 0; e < EP; ++e) {
+        Chunk8<WT> w;
+        if (c < nchunk && e < E)
+          w.load(Wr + static_cast<size_t>(e) * d + c * 8);
+        else
+          w.zero();
+#pragma unroll
+        for (int j = 0; j < TPW; ++j) {
+          if constexpr (kPair) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) acc2[j * EP + e] = __ffma2_rn(cur[j].pair(i), w.pair(i), acc2[j * EP + e]);
+          } else {
+            float2 a2 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a2 = __ffma2_rn(cur[j].pair(i), w.pair(i), a2);
+            acc[j * EP + e] += a2.x + a2.y;
+          }
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < TPW; ++j) {
+        cur[j] = nxt[j];
+        nxt[j] = after[j];
+      }
+    }
+    if constexpr (kPair) {
+#pragma unroll
+      for (int i = 0; i < NV; ++i) acc[i] = acc2[i].x + acc2[i].y;
+    }
+    // reduce-scatter: afterwards acc[0, PER) of lane l are the logits of
+    // partial index [PER l, PER l + PER) (token (PER l) / EP, experts (PER l) % EP ...)
+    if constexpr (NV == 64) rs_level<64>(acc, lane, 16);
+    rs_level<32>(acc, lane, NV == 64 ? 8 : 16);
+    if constexpr (NV == 64) {
+      rs_level<16>(acc, lane, 4);
+      rs_level<8>(acc, lane, 2);
+      rs_level<4>(acc, lane, 1);
+    } else {
+      rs_level<16>(acc, lane, 8);
+      rs_level<8>(acc, lane, 4);
+      rs_level<4>(acc, lane, 2);
+      rs_level<2>(acc, lane, 1);
+    }
+    // the EP / PER lanes of a token: consecutive lanes, group size G
+    constexpr int G = EP / PER;
+    const int t = t0 + (lane * PER) / EP;
+    const int e_base = (lane * PER) % EP;
+    const bool tok = t < T;
+    float v[PER];
+    uint64_t key[PER];
+    float m = -INFINITY;
+#pragma unroll
+    for (int i = 0; i < PER; ++i) {
+      const int e = e_base + i;
+      v[i] = acc[i];
+      if (!tok || e >= E) {
+        v[i] = -INFINITY;
+        key[i] = 0ull;
+      } else {
+        if (bias) v[i] += bias[e];
+        if (logits_out) logits_out[static_cast<size_t>(t) * E + e] = v[i];
+        key[i] = sel_key(v[i], e);
+      }
+      m = fmaxf(m, v[i]);
+    }
+#pragma unroll
+    for (int o = G / 2; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    float sum = 0.f;
+#pragma unroll
+    for (int i = 0; i < PER; ++i)
+      if (e_base + i < E) sum += exp2f((v[i] - m) * kLog2e);
+#pragma unroll
+    for (int o = G / 2; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
+    const float inv_sum = 1.0f / sum;
+    const bool leader = (lane % G) == 0;
+    float psum = 0.f;
+    for (int r = 0; r < k; ++r) {
+      uint64_t best = 0;
+#pragma unroll
+      for (int i = 0; i < PER; ++i) best = key[i] > best ? key[i] : best;
+#pragma unroll
+      for (int o = G / 2; o; o >>= 1) {
+        const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
+        best = other > best ? other : best;
+      }
+      const float pr = exp2f((key_value(best) - m) * kLog2e) * inv_sum;
+      psum += pr;
+      if (tok && leader) {
+        idx_out[static_cast<size_t>(t) * k + r] = key_index(best);
+        w_out[static_cast<size_t>(t) * k + r] = pr;
+      }
+#pragma unroll
+      for (int i = 0; i < PER; ++i) key[i] = key[i] == best ? 0ull : key[i];
+    }
+    if (renorm && tok && leader)
+      for (int r = 0; r < k; ++r) w_out[static_cast<size_t>(t) * k + r] /= psum;
+  }
+}
+
+template <typename XT, typename WT, int EP>
+int fused_launch(const void* x, const void* Wr, const float* bias, int T, int d, int E, int k, int renorm,
+                 float* logits_out, int32_t* idx, float* w, cudaStream_t s) {
+  constexpr int TPW = EP >= 32 ? 1 : 32 / EP;
+  const int warps_needed = (T + TPW - 1) / TPW;
+  const int blocks = max(1, min((warps_needed + kFusedWarps - 1) / kFusedWarps, num_sms() * 8));
+  return launch_pdl("router_fused_kernel", router_fused_kernel<XT, WT, EP>, dim3(blocks), dim3(kFusedWarps * 32), 0,
+                    s, static_cast<const XT*>(x), static_cast<const WT*>(Wr), bias, T, d, E, k, renorm, logits_out,
+                    idx, w);
+}
+
+template <typename XT, typename WT>
+int fused_dispatch(const void* x, const void* Wr, const float* bias, int T, int d, int E, int k, int renorm,
+                   float* lo, int32_t* idx, float* w, cudaStream_t s) {
+  if (E <= 8) return fused_launch<XT, WT, 8>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
+  if (E <= 16) return fused_launch<XT, WT, 16>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
+  if (E <= 32) return fused_launch<XT, WT, 32>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
+  return fused_launch<XT, WT, 64>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
+}
+
 template <typename XT, typename WT>
 int simt_logits(const void* x, const void* Wr, int T, int d, int E, float* logits, cudaStream_t s) {
   dim3 grid((T + kRTok - 1) / kRTok, (E + kREC - 1) / kREC);
@@ -382,10 +606,25 @@ bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E) {
 
 int router_padded_experts(int E) { return (E + 63) / 64 * 64; }
 
+bool router_is_fused(int T, int d, int E) {
+  return E <= 64 && (E <= 16 || static_cast<double>(T) * d * E <= static_cast<double>(1ll << 30));
+}
+
 int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d, int E,
                   int k, int renorm, float* logits_out, int32_t* idx, float* w, float* parts, int* status,
                   cudaStream_t s) {
   if (T == 0) return MOE_OK;
+  if (router_is_fused(T, d, E)) {
+    if (x_dtype == MOE_BF16 && w_dtype == MOE_BF16)
+      return fused_dispatch<__nv_bfloat16, __nv_bfloat16>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
+    if (x_dtype == MOE_F32 && w_dtype == MOE_F32)
+      return fused_dispatch<float, float>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
+    if (x_dtype == MOE_F32 && w_dtype == MOE_BF16)
+      return fused_dispatch<float, __nv_bfloat16>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
+    if (x_dtype == MOE_BF16 && w_dtype == MOE_F32)
+      return fused_dispatch<__nv_bfloat16, float>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
+    return MOE_ERR_UNSUPPORTED;
+  }
   int nsplit = 1;
   int pstride = E;
   int st;

@@ -315,6 +315,12 @@ int moe_forward_marked(const moe_config* cfg, const void* x, const void* W_r, co
                        const float* W2s_scales, void* out, int32_t* counts_out, void* ws, size_t ws_bytes,
                        void* const* stage_events, void* stream);
 
+/* How many kernels one moe_forward of this shape launches (host arithmetic
+ * only, no device needed): the router (1 when it runs fused, else 2), the
+ * permute's 3, the 2 grouped GEMMs and the combine; 0 for T = 0, -1 for an
+ * invalid config.  (Status-word resets are memsets, not kernels.) */
+int moe_forward_launches(const moe_config* cfg);
+
 /* As moe_forward, but x_host and out_host are HOST buffers (page-locked for
  * the copies to overlap): x is copied into the workspace, the layer runs,
  * and out is copied back, all on `stream`.  The call returns without

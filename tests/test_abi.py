@@ -163,3 +163,16 @@ def test_grouped_gemm_plan_edges(L):
     assert P(8, 8 * 256, 1024, 1024, epilogue=gg.EPI_SILU_GATE, num_sms=148) == \
         "bf16 128x128 silu-gate (64 out cols)"
     assert P(8, 8 * 256, 4096, 1024, epilogue=gg.EPI_SILU_GATE, num_sms=148) == "bf16 128x256 silu-gate"
+
+
+def test_forward_launch_count():
+    L = gg.lib()
+    import ctypes
+    mixtral = gg.make_config(T=4096, d=4096, E=8, k=2, inter=14336)
+    fine = gg.make_config(T=4096, d=7168, E=256, k=8, inter=2048, shared_inter=2048)
+    decode = gg.make_config(T=128, d=2048, E=64, k=2, inter=1408)
+    assert L.moe_forward_launches(ctypes.byref(mixtral)) == 7   # fused router
+    assert L.moe_forward_launches(ctypes.byref(decode)) == 7
+    assert L.moe_forward_launches(ctypes.byref(fine)) == 8      # tensor-core logits + selection
+    assert L.moe_forward_launches(ctypes.byref(gg.make_config(T=0, d=256, E=8, k=2, inter=512))) == 0
+    assert L.moe_forward_launches(ctypes.byref(gg.make_config(T=4, d=100, E=8, k=2, inter=512))) == -1

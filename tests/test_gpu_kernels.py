@@ -94,6 +94,39 @@ def test_router_topk(name, T, renorm):
     np.testing.assert_allclose(w.cpu().numpy(), want_w, rtol=2e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("T,d,E,k,xdt,wdt", [(1000, 264, 5, 2, torch.bfloat16, torch.bfloat16),
+                                           (333, 4096, 16, 4, torch.bfloat16, torch.bfloat16),
+                                           (70, 1024, 33, 3, torch.bfloat16, torch.bfloat16),
+                                           (129, 512, 64, 8, torch.float32, torch.bfloat16),
+                                           (513, 256, 8, 2, torch.bfloat16, torch.float32),
+                                           (1, 8, 7, 7, torch.float32, torch.float32)])
+def test_fused_router_shapes(T, d, E, k, xdt, wdt):
+    # the one-launch router (E <= 64): ragged d, E not a power of two, mixed operand types
+    g = torch.Generator(device=DEV).manual_seed(T + d + E)
+    x = torch.randn((T, d), device=DEV, generator=g).to(xdt)
+    W = (torch.randn((E, d), device=DEV, generator=g) * 0.05).to(wdt)
+    bias = torch.randn(E, device=DEV, generator=g)
+    idx, w, logits = gg.router_topk(x, W, k, bias=bias, want_logits=True)
+    torch.cuda.synchronize()
+    gl = f64(logits)
+    ol = oracle.router_logits(x, W, bias)
+    np.testing.assert_allclose(gl, ol, rtol=1e-4, atol=2e-5 * np.sqrt(d))
+    want = oracle.topk_select(gl, k)
+    assert np.array_equal(idx.cpu().numpy(), want)
+    np.testing.assert_allclose(w.cpu().numpy(), oracle.gate_weights(oracle.softmax(gl), want), rtol=2e-6, atol=1e-7)
+
+
+@pytest.mark.parametrize("E,k", [(8, 2), (32, 5), (64, 8)])
+def test_fused_router_ties_go_to_the_lower_index(E, k):
+    # every expert row equal: all logits tie, so the selection is experts 0..k-1 in order
+    x = torch.randn((300, 512), device=DEV).to(torch.bfloat16)
+    W = (torch.randn((1, 512), device=DEV) * 0.05).to(torch.bfloat16).repeat(E, 1).contiguous()
+    idx, w = gg.router_topk(x, W, k)
+    torch.cuda.synchronize()
+    assert np.array_equal(idx.cpu().numpy(), np.tile(np.arange(k), (300, 1)))
+    np.testing.assert_allclose(w.cpu().numpy(), 1.0 / E, rtol=1e-6)
+
+
 # ---------------------------------------------------------------- permute
 def _check_plan(res, idx_np, E, shared):
     plan = oracle.permutation(idx_np, E, shared=shared)
