@@ -19,7 +19,7 @@ import torch
 __all__ = [
     "LIB_PATH", "MoEError", "MoEConfig", "lib", "exported_symbols", "status_string", "device_info",
     "router_topk", "topk_logits", "permute", "grouped_gemm", "combine", "quantize_weights_fp8",
-    "capacity_from_factor", "forward_launches",
+    "capacity_from_factor", "forward_launches", "grouped_gemm_gather",
     "workspace_size", "moe_forward", "moe_forward_marked", "moe_forward_host", "host_staging_size", "read_device_status",
     "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "MOE_MXE4M3", "EPI_NONE", "EPI_SILU_GATE",
     "quantize_weights_mx",
@@ -69,6 +69,8 @@ _SIGS = {
     "moe_grouped_gemm_workspace_size": (_sz, []),
     "moe_grouped_gemm_plan": (ctypes.c_char_p, [_i, _i, _i, _i, _i, _i, _i, _i, _i]),
     "moe_grouped_gemm": (_i, [_vp, _fp, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _vp, _i, _fp, _vp, _sz, _vp]),
+    "moe_grouped_gemm_gather": (_i, [_vp, _fp, _i, _ip, _vp, _fp, _ip, _i, _i, _i, _i, _i, _i, _vp, _i, _fp, _vp, _sz,
+                                     _vp]),
     "moe_combine": (_i, [_vp, _ip, _fp, _i, _i, _i, _i, _vp, _i, _vp]),
     "moe_combine_plan": (_i, [_vp, _ip, _fp, _ip, _i, _i, _i, _i, _i, _vp, _i, _vp]),
     "moe_selftest_workspace_size": (_sz, []),
@@ -248,6 +250,30 @@ def grouped_gemm(A, B, offsets, N: int, epilogue: int = EPI_NONE, c_dtype=torch.
     _check(L.moe_grouped_gemm(_ptr(A), _ptr(A_scales), _ptr(B), _ptr(B_scales), _ptr(offsets), G, rows, N, K,
                               q8 if fp8 else MOE_BF16, epilogue, _ptr(C), cdt, _ptr(Cs), _ptr(ws), ws.numel(),
                               _stream(stream)), "moe_grouped_gemm")
+    return (C, Cs) if cdt == q8 else C
+
+
+def grouped_gemm_gather(A, A_rows, B, offsets, N: int, epilogue: int = EPI_NONE, c_dtype=torch.bfloat16,
+                        A_scales=None, B_scales=None, out=None, out_scales=None, ws=None, stream=None,
+                        mx: bool = False):
+    """grouped_gemm whose A row r is row A_rows[r] of A (moe_grouped_gemm_gather); C has len(A_rows) rows."""
+    _cuda(A, A_rows, B, offsets, A_scales, B_scales)
+    src_rows, K = A.shape
+    rows = A_rows.numel()
+    G = B.shape[0]
+    fp8 = A.dtype in (torch.uint8, torch.float8_e4m3fn)
+    q8 = MOE_MXE4M3 if mx else MOE_E4M3
+    cdt = {torch.bfloat16: MOE_BF16, torch.float32: MOE_F32, torch.uint8: q8}[c_dtype]
+    C = out if out is not None else torch.empty((rows, N), dtype=c_dtype, device=A.device)
+    Cs = out_scales
+    if cdt == q8 and Cs is None:
+        Cs = torch.empty((N // 128, rows), dtype=torch.float32, device=A.device)
+    L = lib()
+    if ws is None:
+        ws = _scratch(L.moe_grouped_gemm_workspace_size(), A.device)
+    _check(L.moe_grouped_gemm_gather(_ptr(A), _ptr(A_scales), src_rows, _ptr(A_rows), _ptr(B), _ptr(B_scales),
+                                     _ptr(offsets), G, rows, N, K, q8 if fp8 else MOE_BF16, epilogue, _ptr(C), cdt,
+                                     _ptr(Cs), _ptr(ws), ws.numel(), _stream(stream)), "moe_grouped_gemm_gather")
     return (C, Cs) if cdt == q8 else C
 
 

@@ -104,6 +104,10 @@ struct PermuteArgs {
   int32_t* block_base;  // scratch [nblocks * E]
   int* status;
   int capacity = 0;     // > 0: an expert keeps only its first `capacity` pairs in token order
+  // 1: the grouped GEMM gathers its A rows through row_to_token, so xp is
+  // [T, d] with each token's row once (cast / quantised as xp_dtype says,
+  // scales [d/128][T]); with bf16 x and a bf16 xp nothing is copied at all
+  int gather = 0;
 };
 int permute_blocks(int T);  // number of token blocks the permute kernels use
 int launch_permute(const PermuteArgs& a, cudaStream_t s);
@@ -116,6 +120,8 @@ struct GemmArgs {
   const void* B_extra;      // optional extra group (index G) with its own [Nb, K] weights
   const float* B_extra_scales;
   const int32_t* offsets;   // [G + has_extra + 1]
+  const int32_t* a_rows;    // gather: A row r is row a_rows[r] of A (< 0: any row); A has a_src_rows rows
+  int a_src_rows;
   int G, has_extra, rows, N, K;
   int B_rows;               // > 0: rows of B actually present (G == 1); rows past it read as zero
   int ksplit;               // > 1: fp32 partial products of K slices at C + s * rows * N (no epilogue)
@@ -132,6 +138,7 @@ struct GemmArgs {
 };
 int launch_grouped_gemm(const GemmArgs& a, cudaStream_t s);
 int plan_grouped_gemm(const GemmArgs& a, int sms);  // host-only choice of kernel (see gemm_variant_name)
+bool plan_takes_gathered_a(int variant);            // the variant can load A rows through a_rows
 const char* gemm_variant_name(int variant);
 
 // shared_base: device int32 holding the first shared row (offsets[E] of the

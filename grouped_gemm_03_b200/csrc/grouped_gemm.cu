@@ -81,7 +81,29 @@ struct Params {
   float* C_scales;         // [N/128][rows] when C is E4M3
   uint64_t wait_ns;        // limit of every pipeline wait
   int stall;               // self-test: the epilogue first waits on a barrier no thread arrives at
+  // gathered A ("permute in the load"): A row r of the grouped problem is row
+  // a_rows[r] of the a_src_rows-row tensor tmA maps (box one row high); < 0: any row
+  const int32_t* a_rows;
+  int a_src_rows;
 };
+
+// Source rows of the 4 A rows lane `lane` gathers for the tile starting at
+// row a_row: rows past the problem or without a token read row 0 (never stored).
+__device__ __forceinline__ void gather_rows(const Params& p, int a_row, int lane, int (&tok)[4]) {
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int r = a_row + 4 * lane + i;
+    const int v = r < p.rows ? __ldg(p.a_rows + r) : 0;
+    tok[i] = (v < 0 || v >= p.a_src_rows) ? 0 : v;
+  }
+}
+
+// Source row of A row r (gathered or not), for per-row A scales.
+__device__ __forceinline__ int a_source_row(const Params& p, int r) {
+  if (!p.a_rows) return r;
+  const int v = r < p.rows ? __ldg(p.a_rows + r) : 0;
+  return (v < 0 || v >= p.a_src_rows) ? 0 : v;
+}
 
 struct TileCoord {
   int g, mb, nb, ks, m_g;
@@ -208,7 +230,65 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int total = s_tile[G];
   const int nk = p.K / 64;
 
-  if (warp == 0) {
+  if (warp == 0 && p.a_rows) {
+    // -------------------------------------------------------------- producer, gathered A
+    // lane l brings A rows 4l..4l+3 of the tile (one tile::gather4 each k-step);
+    // lane 0 also waits for the stage and loads B
+    uint32_t stage = 0, phase = 0, issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+      const int g = tc.g, nb = tc.nb;
+      int tok[4];
+      gather_rows(p, s_off[g] + tc.mb * BM, lane, tok);
+      const bool extra = g >= p.G_main;
+      const CUtensorMap* mB = extra ? &tmBx : &tmB;
+      const int gb = extra ? 0 : g;
+      const int kb0 = tc.ks * nk / p.ksplit, kb1 = (tc.ks + 1) * nk / p.ksplit;
+      for (int kb = kb0; kb < kb1; ++kb) {
+        int go = 1;
+        if (lane == 0) {
+          go = ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, p.wait_ns);
+          if (go) ptx::mbar_arrive_expect_tx(&full[stage], L::STAGE_BYTES);
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
+        ptx::tma_gather4(sA + stage * L::A_BYTES + lane * 512, &tmA, &full[stage], kb * 64, tok[0], tok[1], tok[2],
+                         tok[3]);
+        if (lane == 0) {
+          if (EPI) {
+            const int brow = gb * 2 * p.N + nb * (MMA_N / 2);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 64, brow);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES + (MMA_N / 2) * 128, mB, &full[stage], kb * 64, brow + p.N);
+          } else {
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 64, gb * p.N + nb * MMA_N);
+          }
+        }
+        ++issued;
+        if (++stage == L::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      set_status(p.status, MOE_ERR_TIMEOUT);
+      const uint32_t pending = issued < static_cast<uint32_t>(L::STAGES) ? issued : L::STAGES;
+      uint32_t s2 = stage, ph = phase;
+      for (uint32_t i = 0; i < pending; ++i) {
+        if (s2 == 0) {
+          s2 = L::STAGES - 1;
+          ph ^= 1;
+        } else {
+          --s2;
+        }
+        ptx::mbar_wait(&full[s2], ph, reinterpret_cast<volatile int*>(s_bad), p.wait_ns);
+      }
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       uint32_t stage = 0, phase = 0;
@@ -1096,7 +1176,64 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
   const int total = s_tile[G];
   const int nk = p.K / 128;
 
-  if (warp == 0) {
+  if (warp == 0 && p.a_rows) {
+    // -------------------------------------------------------------- producer, gathered A
+    // lane l brings A rows 4l..4l+3 of the tile (one tile::gather4 each k-step);
+    // lane 0 also waits for the stage and loads B
+    uint32_t stage = 0, phase = 0, issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+      const int g = tc.g, nb = tc.nb;
+      int tok[4];
+      gather_rows(p, s_off[g] + tc.mb * BM, lane, tok);
+      const bool extra = g >= p.G_main;
+      const CUtensorMap* mB = extra ? &tmBx : &tmB;
+      const int gb = extra ? 0 : g;
+      for (int kb = 0; kb < nk; ++kb) {
+        int go = 1;
+        if (lane == 0) {
+          go = ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs);
+          if (go) ptx::mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
+        ptx::tma_gather4(sA + stage * L::A_BYTES + lane * 512, &tmA, &full[stage], kb * 128, tok[0], tok[1], tok[2],
+                         tok[3]);
+        if (lane == 0) {
+          if (EPI) {
+            const int brow = gb * 2 * p.N + nb * 128;
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, brow);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES + 128 * 128, mB, &full[stage], kb * 128, brow + p.N);
+          } else {
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, gb * p.N + nb * 256);
+          }
+        }
+        ++issued;
+        if (++stage == L::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      set_status(p.status, MOE_ERR_TIMEOUT);
+      const uint32_t pending = issued < static_cast<uint32_t>(L::STAGES) ? issued : L::STAGES;
+      uint32_t s2 = stage, ph = phase;
+      for (uint32_t i = 0; i < pending; ++i) {
+        if (s2 == 0) {
+          s2 = L::STAGES - 1;
+          ph ^= 1;
+        } else {
+          --s2;
+        }
+        ptx::mbar_wait(&full[s2], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+      }
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ producer
       uint32_t stage = 0, phase = 0, issued = 0;
@@ -1212,8 +1349,8 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
       // Scales are fetched ahead of use so that no K block waits on a global
       // load: the row's sa[kb] through a 2-deep register queue, the two
       // weight-block scales one K block ahead (the same address in every lane).
-      const float* sa_p = p.A_scales + grow;
-      const size_t rstride = static_cast<size_t>(p.rows);
+      const float* sa_p = p.A_scales + a_source_row(p, static_cast<int>(grow));
+      const size_t rstride = static_cast<size_t>(p.a_rows ? p.a_src_rows : p.rows);
       float sa0 = valid ? __ldg(sa_p) : 0.f;
       float sa1 = (valid && 1 < nbk) ? __ldg(sa_p + rstride) : 0.f;
       sa_p += 2 * rstride;
@@ -1501,7 +1638,64 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
   const int total = s_tile[G];
   const int nk = p.K / 128;
 
-  if (warp == 0) {
+  if (warp == 0 && p.a_rows) {
+    // -------------------------------------------------------------- producer, gathered A
+    // lane l brings A rows 4l..4l+3 of the tile (one tile::gather4 each k-step);
+    // lane 0 also waits for the stage and loads B
+    uint32_t stage = 0, phase = 0, issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
+      const int g = tc.g, nb = tc.nb;
+      int tok[4];
+      gather_rows(p, s_off[g] + tc.mb * BM, lane, tok);
+      const bool extra = g >= p.G_main;
+      const CUtensorMap* mB = extra ? &tmBx : &tmB;
+      const int gb = extra ? 0 : g;
+      for (int kb = 0; kb < nk; ++kb) {
+        int go = 1;
+        if (lane == 0) {
+          go = ptx::mbar_wait(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs);
+          if (go) ptx::mbar_arrive_expect_tx(&full[stage], L::A_BYTES + L::B_BYTES);
+        }
+        if (!__shfl_sync(0xffffffffu, go, 0)) {
+          ok = false;
+          break;
+        }
+        ptx::tma_gather4(sA + stage * L::A_BYTES + lane * 512, &tmA, &full[stage], kb * 128, tok[0], tok[1], tok[2],
+                         tok[3]);
+        if (lane == 0) {
+          if (EPI) {
+            const int brow = gb * 2 * p.N + nb * 128;
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, brow);
+            ptx::tma_load_2d(sB + stage * L::B_BYTES + 128 * 128, mB, &full[stage], kb * 128, brow + p.N);
+          } else {
+            ptx::tma_load_2d(sB + stage * L::B_BYTES, mB, &full[stage], kb * 128, gb * p.N + nb * 256);
+          }
+        }
+        ++issued;
+        if (++stage == L::STAGES) {
+          stage = 0;
+          phase ^= 1;
+        }
+      }
+    }
+    if (!ok && lane == 0) {
+      *abort_flag = 1;
+      set_status(p.status, MOE_ERR_TIMEOUT);
+      const uint32_t pending = issued < static_cast<uint32_t>(L::STAGES) ? issued : L::STAGES;
+      uint32_t s2 = stage, ph = phase;
+      for (uint32_t i = 0; i < pending; ++i) {
+        if (s2 == 0) {
+          s2 = L::STAGES - 1;
+          ph ^= 1;
+        } else {
+          --s2;
+        }
+        ptx::mbar_wait(&full[s2], ph, reinterpret_cast<volatile int*>(s_bad), kWaitLimitNs);
+      }
+    }
+  } else if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------ TMA producer
       uint32_t stage = 0, phase = 0, issued = 0;
@@ -1556,7 +1750,7 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
     // and B's scale of its 128-row weight block (one value per atom).
     uint32_t stage = 0, phase = 0;
     bool ok = true;
-    const size_t rstride = static_cast<size_t>(p.rows);
+    const size_t rstride = static_cast<size_t>(p.a_rows ? p.a_src_rows : p.rows);
     for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
       const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
       const int g = tc.g, nb = tc.nb;
@@ -1567,7 +1761,7 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
       const float* sb1 = bsc + static_cast<size_t>(EPI ? p.N / 128 + nb : 2 * nb + 1) * nk;  // up / second half
       int rowc[4];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) rowc[c] = min(a_row + lane + 32 * c, p.rows - 1);  // rows past A: any value
+      for (int c = 0; c < 4; ++c) rowc[c] = a_source_row(p, min(a_row + lane + 32 * c, p.rows - 1));  // past A: any
       for (int kb = 0; kb < nk; ++kb) {
         float sa[4];
 #pragma unroll
@@ -1842,6 +2036,14 @@ bool make_gateup_map(CUtensorMap* m, const void* base, int G, int N, int K) {
   return true;
 }
 
+// The A operand's map: [rows, K] in 128-row boxes, or, when A rows are
+// gathered, the source [a_src_rows, K] in one-row boxes for tile::gather4.
+bool a_map(CUtensorMap* m, const GemmArgs& a, int ebytes) {
+  if (a.a_rows)
+    return make_map(m, a.A, ebytes, static_cast<uint64_t>(a.a_src_rows > 0 ? a.a_src_rows : 1), a.K, 1);
+  return make_map(m, a.A, ebytes, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM);
+}
+
 template <int MMA_N, int EPI, int OUT>
 int run_bf16(const GemmArgs& a, cudaStream_t s) {
   using L = Tile<MMA_N>;
@@ -1849,7 +2051,7 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   const int nb_rows = EPI ? 2 * a.N : a.N;
   const uint32_t box_b = EPI ? MMA_N / 2 : MMA_N;
   CUtensorMap mA, mB, mBx;
-  if (!make_map(&mA, a.A, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
+  if (!a_map(&mA, a, 2)) return MOE_ERR_CUDA;
   const uint64_t b_rows = a.B_rows > 0 ? static_cast<uint64_t>(a.B_rows)
                                        : static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows;
   if (!make_map(&mB, a.B, 2, b_rows, a.K, box_b)) return MOE_ERR_CUDA;
@@ -1876,6 +2078,8 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   p.status = a.status;
   p.wait_ns = a.wait_ns ? a.wait_ns : kWaitLimitNs;
   p.stall = a.stall;
+  p.a_rows = a.a_rows;
+  p.a_src_rows = a.a_src_rows;
   return launch_pdl(__func__, gg_bf16_kernel<MMA_N, EPI, OUT>, dim3(a.grid > 0 ? a.grid : num_sms()), dim3(kThreads),
                     L::SMEM, s, mA, mB, mBx, p);
 }
@@ -1978,7 +2182,7 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
   const int nb_rows = EPI ? 2 * a.N : a.N;
   const uint32_t box_b = EPI ? 128 : 256;
   CUtensorMap mA, mB, mBx;
-  if (!make_map(&mA, a.A, 1, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
+  if (!a_map(&mA, a, 1)) return MOE_ERR_CUDA;
   if (!make_map(&mB, a.B, 1, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 1, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   // output boxes of one warp's 32 rows: 64 bf16 columns (128-byte swizzle), or 32 columns of the gated output
@@ -2007,6 +2211,8 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
   p.B_scales = a.B_scales;
   p.Bx_scales = a.has_extra ? a.B_extra_scales : a.B_scales;
   p.C_scales = a.C_scales;
+  p.a_rows = a.a_rows;
+  p.a_src_rows = a.a_src_rows;
   return launch_pdl(__func__, gg_fp8_kernel<EPI, OUT>, dim3(num_sms()), dim3(kThreadsF8), kF8Smem, s, mA, mB, mBx, mC,
                     p);
 }
@@ -2018,7 +2224,7 @@ int run_mx(const GemmArgs& a, cudaStream_t s) {
   const int nb_rows = EPI ? 2 * a.N : a.N;
   const uint32_t box_b = EPI ? 128 : 256;
   CUtensorMap mA, mB, mBx;
-  if (!make_map(&mA, a.A, 1, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, BM)) return MOE_ERR_CUDA;
+  if (!a_map(&mA, a, 1)) return MOE_ERR_CUDA;
   if (!make_map(&mB, a.B, 1, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 1, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   static bool attr_set[64] = {};
@@ -2043,6 +2249,8 @@ int run_mx(const GemmArgs& a, cudaStream_t s) {
   p.B_scales = a.B_scales;
   p.Bx_scales = a.has_extra ? a.B_extra_scales : a.B_scales;
   p.C_scales = a.C_scales;
+  p.a_rows = a.a_rows;
+  p.a_src_rows = a.a_src_rows;
   return launch_pdl(__func__, gg_mx_kernel<EPI, OUT>, dim3(num_sms()), dim3(kThreadsMX), kSmem, s, mA, mB, mBx, p);
 }
 
@@ -2067,8 +2275,9 @@ int plan_grouped_gemm(const GemmArgs& a, int sms) {
   if (a.ab_dtype == MOE_BF16) {
     // CTA pairs pay off when tiles of 256 rows are mostly full: large groups on average;
     // groups of a few tokens (decode) put the weights on the 128-row side instead
-    const bool pairs = a.pair_tiles > 0 || (a.pair_tiles == 0 && a.rows >= 512 * groups);
-    const bool swap = a.swap_ab > 0 || (a.swap_ab == 0 && a.rows < 32 * groups);
+    // gathered A rows (tile::gather4) are loaded by the single-CTA kernels only
+    const bool pairs = !a.a_rows && (a.pair_tiles > 0 || (a.pair_tiles == 0 && a.rows >= 512 * groups));
+    const bool swap = !a.a_rows && (a.swap_ab > 0 || (a.swap_ab == 0 && a.rows < 32 * groups));
     if (swap && a.ksplit <= 1 && a.c_dtype == MOE_BF16) {
       if (a.epilogue == MOE_EPI_SILU_GATE && a.N % 64 == 0) return kSwapGate;
       if (a.epilogue == MOE_EPI_NONE && a.N % 128 == 0) return kSwapNone;
@@ -2115,6 +2324,11 @@ int plan_grouped_gemm(const GemmArgs& a, int sms) {
     return kUnsupported;
   }
   return kUnsupported;
+}
+
+bool plan_takes_gathered_a(int v) {
+  return v == kGate64 || v == kGate128 || v == kNone256 || v == kNone128 || v == kNone64 || v == kFp8GateE4M3 ||
+         v == kFp8GateBf16 || v == kFp8None || v == kMxGateE4M3 || v == kMxGateBf16 || v == kMxNone;
 }
 
 const char* gemm_variant_name(int v) {

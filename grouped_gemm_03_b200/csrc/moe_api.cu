@@ -276,6 +276,47 @@ int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const 
   return launch_grouped_gemm(a, s);
 }
 
+int moe_grouped_gemm_gather(const void* A, const float* A_scales, int A_src_rows, const int32_t* A_rows,
+                            const void* B, const float* B_scales, const int32_t* offsets, int G, int rows, int N,
+                            int K, int ab_dtype, int epilogue, void* C, int c_dtype, float* C_scales, void* ws,
+                            size_t ws_bytes, void* stream) {
+  if (G <= 0 || rows < 0 || N <= 0 || K <= 0 || A_src_rows <= 0) return MOE_ERR_INVALID;
+  if (G > kMaxGroups) return MOE_ERR_UNSUPPORTED;
+  if (!A || !B || !offsets || !C || !A_rows) return MOE_ERR_INVALID;
+  if (ab_dtype != MOE_BF16 && !is_e4m3(ab_dtype)) return MOE_ERR_INVALID;
+  if (epilogue != MOE_EPI_NONE && epilogue != MOE_EPI_SILU_GATE) return MOE_ERR_INVALID;
+  if (is_e4m3(ab_dtype) && (!A_scales || !B_scales)) return MOE_ERR_INVALID;
+  if (is_e4m3(c_dtype) && !C_scales) return MOE_ERR_INVALID;
+  if (is_e4m3(c_dtype) && c_dtype != ab_dtype) return MOE_ERR_UNSUPPORTED;
+  if (ab_dtype == MOE_BF16 && K % 64 != 0) return MOE_ERR_UNSUPPORTED;
+  if (is_e4m3(ab_dtype) && K % 128 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!aligned(A, 16) || !aligned(B, 16) || !aligned(C, 16)) return MOE_ERR_INVALID;
+  if (!ws || !aligned(ws, 256)) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_grouped_gemm_workspace_size()) return MOE_ERR_WORKSPACE;
+  GemmArgs a{};
+  a.A = A;
+  a.A_scales = A_scales;
+  a.a_rows = A_rows;
+  a.a_src_rows = A_src_rows;
+  a.B = B;
+  a.B_scales = B_scales;
+  a.offsets = offsets;
+  a.G = G;
+  a.rows = rows;
+  a.N = N;
+  a.K = K;
+  a.ab_dtype = ab_dtype;
+  a.epilogue = epilogue;
+  a.c_dtype = c_dtype;
+  a.C = C;
+  a.C_scales = C_scales;
+  if (!plan_takes_gathered_a(plan_grouped_gemm(a, num_sms()))) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = as_stream(stream);
+  MOE_CUDA_CHECK(cudaMemsetAsync(ws, 0, sizeof(int), s));
+  a.status = static_cast<int*>(ws);
+  return launch_grouped_gemm(a, s);
+}
+
 // ------------------------------------------------------------------ failure-detection self-test
 size_t moe_selftest_workspace_size(void) { return 1024 + (16 + 128 + 256) * 1024; }
 
@@ -417,6 +458,27 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   if (st != MOE_OK) return st;
   if ((st = mark(1)) != MOE_OK) return st;
 
+  // "Permute in the load": when the up GEMM runs on a single-CTA kernel it
+  // gathers its A rows through row_to_token (tile::gather4), so the permute
+  // writes only the plan (plus, for E4M3 experts or fp32 x, each token's row
+  // once, quantised or cast) and the expert-ordered copy of x is never made.
+  GemmArgs up{};
+  up.B = W1;
+  up.B_extra = W1_shared;
+  up.offsets = offsets;
+  up.G = E;
+  up.has_extra = shared ? 1 : 0;
+  up.rows = Rp;
+  up.N = I;
+  up.K = d;
+  up.ab_dtype = fp8 ? qdt : MOE_BF16;
+  up.epilogue = MOE_EPI_SILU_GATE;
+  up.c_dtype = fp8 ? qdt : MOE_BF16;
+  up.C = base + L.h;
+  up.status = status;
+  const bool gather = plan_takes_gathered_a(plan_grouped_gemm(up, num_sms()));
+  const bool x_as_is = gather && !fp8 && c.x_dtype == MOE_BF16;  // the GEMM reads x itself
+
   PermuteArgs pa;
   pa.x = x;
   pa.x_dtype = c.x_dtype;
@@ -436,25 +498,16 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   pa.block_base = reinterpret_cast<int32_t*>(base + L.base);
   pa.status = status;
   pa.capacity = c.capacity;
+  pa.gather = gather ? 1 : 0;
   st = launch_permute(pa, s);
   if (st != MOE_OK) return st;
   if ((st = mark(2)) != MOE_OK) return st;
 
-  GemmArgs up{};
-  up.A = base + L.xp;
-  up.B = W1;
-  up.B_extra = W1_shared;
-  up.offsets = offsets;
-  up.G = E;
-  up.has_extra = shared ? 1 : 0;
-  up.rows = Rp;
-  up.N = I;
-  up.K = d;
-  up.ab_dtype = fp8 ? qdt : MOE_BF16;
-  up.epilogue = MOE_EPI_SILU_GATE;
-  up.c_dtype = fp8 ? qdt : MOE_BF16;
-  up.C = base + L.h;
-  up.status = status;
+  up.A = x_as_is ? x : base + L.xp;
+  if (gather) {
+    up.a_rows = pa.row_to_token;
+    up.a_src_rows = T;
+  }
   if (fp8) {
     up.A_scales = reinterpret_cast<const float*>(base + L.xps);
     up.B_scales = W1_scales;

@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   const int k = a.k, E = a.E;
   const int R = a.T * k;
   const int rows_total = R + (a.shared ? a.T : 0);
-  const int nd = k + (a.shared ? 1 : 0);  // destinations per token
+  // destinations per token: its k rows (and shared row), or with gather its own row once
+  const int nd = a.gather ? 1 : k + (a.shared ? 1 : 0);
+  const int xp_rows = a.gather ? a.T : rows_total;  // leading dimension of xp_scales
   const bool writer = blockIdx.y == 0;   // one column block writes the index maps
   __shared__ int s_used;  // rows the experts keep: the shared rows start there
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) s_idx[p] = a.idx[static_cast<size_t>(t0) * k + p];
@@ -185,7 +187,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
       if (a.capacity > 0 && row - a.offsets[e] >= a.capacity) row = -1;
       if (row >= R) row = 0;  // only reachable with invalid ids (status already set)
     }
-    s_row[tl * nd + j] = row;
+    if (!a.gather) s_row[tl * nd + j] = row;
     if (writer) {
       a.token_to_row[static_cast<size_t>(t0 + tl) * k + j] = row;
       if (row >= 0) a.row_to_token[row] = t0 + tl;
@@ -193,9 +195,11 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   }
   if (a.shared)
     for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) {
-      s_row[tl * nd + k] = s_used + t0 + tl;
+      if (!a.gather) s_row[tl * nd + k] = s_used + t0 + tl;
       if (writer) a.row_to_token[s_used + t0 + tl] = t0 + tl;
     }
+  if (a.gather)
+    for (int tl = threadIdx.x; tl < nt; tl += blockDim.x) s_row[tl] = t0 + tl;
   if (writer && a.capacity > 0) {  // rows left unused by the overflowing pairs belong to no token
     const int end = s_used + (a.shared ? a.T : 0);
     for (int r = end + b * blockDim.x + threadIdx.x; r < rows_total; r += gridDim.x * blockDim.x)
@@ -203,6 +207,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   }
   __syncthreads();
 
+  if (a.gather && !kFp8 && sizeof(XT) == 2) return;  // the GEMM reads x itself: no copy
   const int d = a.d;
   const int cbeg = blockIdx.y * kScatterCols;
   const int cw = min(kScatterCols, d - cbeg);
@@ -295,7 +300,7 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
         const int row = s_row[tl * nd + j];
         if (row < 0) continue;  // overflowed its expert's capacity
         *reinterpret_cast<uint2*>(xp + static_cast<size_t>(row) * d + c) = qv;
-        if (sub == 0) a.xp_scales[static_cast<size_t>(gi) * rows_total + row] = s;
+        if (sub == 0) a.xp_scales[static_cast<size_t>(gi) * xp_rows + row] = s;
       }
     }
   }
@@ -321,7 +326,8 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
   if (st != MOE_OK) return st;
   const bool fp8 = is_e4m3(a.xp_dtype);
   const bool mx = a.xp_dtype == MOE_MXE4M3;
-  const dim3 grid(nblk, (a.d + kScatterCols - 1) / kScatterCols);
+  const bool copies = !(a.gather && !fp8 && a.x_dtype == MOE_BF16);
+  const dim3 grid(nblk, copies ? (a.d + kScatterCols - 1) / kScatterCols : 1);
   const dim3 block(kPermThreads);
   if (a.x_dtype == MOE_BF16) {
     if (!fp8) return launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, false>, grid, block, 0, s, a);

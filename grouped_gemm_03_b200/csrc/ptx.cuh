@@ -106,6 +106,19 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
+// Four rows r0..r3 of a 2-D tensor (box: one row of 128 bytes) into four
+// consecutive 128-byte rows of this CTA's shared memory at smem_dst, the
+// 128-byte swizzle applied by destination address as for a tiled load;
+// completion counted in bytes on `bar`.  x is the element column.
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const CUtensorMap* m, uint64_t* bar, int x, int r0,
+                                            int r1, int r2, int r3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(x), "r"(r0), "r"(r1), "r"(r2), "r"(r3)
+      : "memory");
+}
+
 // 2-D tiled bulk store of a box from this CTA's shared memory to global
 // memory, tracked as a bulk async-group of the issuing thread.  x must be a
 // multiple of 16 bytes and neither coordinate may be negative.

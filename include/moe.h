@@ -238,6 +238,22 @@ int moe_grouped_gemm(const void* A, const float* A_scales, const void* B, const 
                      const int32_t* offsets, int G, int rows, int N, int K, int ab_dtype, int epilogue,
                      void* C, int c_dtype, float* C_scales, void* ws, size_t ws_bytes, void* stream);
 
+/* moe_grouped_gemm whose A rows are gathered in the load: row r of the
+ * grouped problem (r < rows, in offsets order) is row A_rows[r] of the
+ * source A [A_src_rows, K] (an entry < 0 or >= A_src_rows reads row 0 and
+ * must belong to no group's valid rows), so an expert-contiguous copy of the
+ * tokens never has to be written ("Dense GEMM -> GroupedGEMM -> TP MoE"
+ * §2.2 names steps 3-4, prefix sum and scatter, as hotspots; here the
+ * scatter folds into the GEMM's TMA loads, tile::gather4).  A_rows is a
+ * DEVICE int32 array of `rows` entries (moe_permute's row_to_token);
+ * A_scales, for E4M3 / MX operands, is [K/128][A_src_rows].  Everything else
+ * as moe_grouped_gemm.  The shapes the CTA-pair and swap-AB kernels would
+ * take run on the single-CTA kernels here; an fp32 C is MOE_ERR_UNSUPPORTED. */
+int moe_grouped_gemm_gather(const void* A, const float* A_scales, int A_src_rows, const int32_t* A_rows,
+                            const void* B, const float* B_scales, const int32_t* offsets, int G, int rows, int N,
+                            int K, int ab_dtype, int epilogue, void* C, int c_dtype, float* C_scales, void* ws,
+                            size_t ws_bytes, void* stream);
+
 /* ---------------------------------------------------------------- failure detection
  * Self-test of the grouped GEMM's failure path (no counterpart on the source
  * pages): launches the bf16 grouped-GEMM kernel on one CTA over a small
