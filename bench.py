@@ -88,6 +88,8 @@ def workload_desc(s) -> str:
         parts.append(f"+1 shared (I={s.shared_inter})")
     parts.append(("mx-e4m3 experts (power-of-two scales)" if s.mx else "fp8 e4m3 experts") if s.fp8 else "bf16")
     parts.append(f"Zipf s={s.zipf_s} logit bias" if s.zipf_s else "balanced router")
+    if s.gather:
+        parts.append("up GEMM gathers its A rows in the load")
     return ", ".join(parts)
 
 
@@ -215,7 +217,8 @@ def make_cfg(gg, s):
     rdt = gg.MOE_F32 if s.router_dtype == "f32" else gg.MOE_BF16
     odt = gg.MOE_F32 if s.x_dtype == "f32" else gg.MOE_BF16
     edt = (gg.MOE_MXE4M3 if s.mx else gg.MOE_E4M3) if s.fp8 else gg.MOE_BF16
-    return gg.make_config(s.T, s.d, s.E, s.k, s.inter, s.shared_inter, xdt, rdt, edt, odt, s.renormalize)
+    return gg.make_config(s.T, s.d, s.E, s.k, s.inter, s.shared_inter, xdt, rdt, edt, odt, s.renormalize,
+                          flags=gg.MOE_FLAG_GATHER_A if s.gather else 0)
 
 
 HOLD_CYCLES = 2_000_000  # ~1 ms spin queued ahead of each timed step
@@ -538,7 +541,8 @@ def layer_report(s, r, peaks, peak_kind, world):
     return rep
 
 
-SIDE_WORKLOADS = ("fine", "fine_skew", "fine_fp8", "fine_fp8_skew", "fine_mx", "fine_mx_skew", "decode", "tiny")
+SIDE_WORKLOADS = ("fine", "fine_skew", "fine_fp8", "fine_fp8_skew", "fine_mx", "fine_mx_skew", "fine_gather",
+                  "decode", "tiny")
 
 
 def main():

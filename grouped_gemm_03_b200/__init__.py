@@ -21,13 +21,14 @@ __all__ = [
     "router_topk", "topk_logits", "permute", "grouped_gemm", "combine", "quantize_weights_fp8",
     "capacity_from_factor", "forward_launches", "grouped_gemm_gather",
     "workspace_size", "moe_forward", "moe_forward_marked", "moe_forward_host", "host_staging_size", "read_device_status",
-    "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "MOE_MXE4M3", "EPI_NONE", "EPI_SILU_GATE",
+    "MOE_F32", "MOE_F16", "MOE_BF16", "MOE_E4M3", "MOE_MXE4M3", "MOE_FLAG_GATHER_A", "EPI_NONE", "EPI_SILU_GATE",
     "quantize_weights_mx",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmoe.so")
 
 MOE_F32, MOE_F16, MOE_BF16, MOE_E4M3, MOE_MXE4M3 = 0, 1, 2, 3, 4
+MOE_FLAG_GATHER_A = 1
 EPI_NONE, EPI_SILU_GATE = 0, 1
 _STATUS = {0: "MOE_OK", -1: "MOE_ERR_INVALID", -2: "MOE_ERR_UNSUPPORTED", -3: "MOE_ERR_WORKSPACE",
            -4: "MOE_ERR_CUDA", -5: "MOE_ERR_BAD_OFFSETS", -6: "MOE_ERR_TIMEOUT"}
@@ -46,7 +47,7 @@ class MoEConfig(ctypes.Structure):
     """Mirror of `moe_config` in include/moe.h."""
     _fields_ = [(n, ctypes.c_int) for n in ("T", "d", "E", "k", "inter", "shared_inter", "x_dtype",
                                             "router_dtype", "expert_dtype", "out_dtype", "renormalize",
-                                            "capacity")]
+                                            "capacity", "flags")]
 
 
 _vp, _i, _sz, _fp, _ip = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p
@@ -332,9 +333,9 @@ def quantize_weights_mx(W, stream=None):
 
 # ---------------------------------------------------------------- whole layer
 def make_config(T, d, E, k, inter, shared_inter=0, x_dtype=MOE_BF16, router_dtype=MOE_BF16,
-                expert_dtype=MOE_BF16, out_dtype=MOE_BF16, renormalize=False, capacity=0) -> MoEConfig:
+                expert_dtype=MOE_BF16, out_dtype=MOE_BF16, renormalize=False, capacity=0, flags=0) -> MoEConfig:
     return MoEConfig(T, d, E, k, inter, shared_inter, x_dtype, router_dtype, expert_dtype, out_dtype,
-                     int(renormalize), int(capacity))
+                     int(renormalize), int(capacity), int(flags))
 
 
 def capacity_from_factor(factor: float, T: int, k: int, E: int) -> int:

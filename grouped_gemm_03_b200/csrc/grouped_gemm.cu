@@ -53,16 +53,21 @@ constexpr int BM = 128;
 constexpr int kThreads = 192;
 constexpr int kSmemBudget = 220 * 1024;
 
-template <int MMA_N>
+// Shared memory of the single-CTA bf16 kernel.  With bf16 output each of the
+// four epilogue warps stages its 32 rows in two 4 KB boxes (32 rows x 64
+// columns, 128-byte swizzled) for bulk tensor stores, at OUTB.
+template <int MMA_N, bool kStageOut>
 struct Tile {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = MMA_N * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TABLE_BYTES = 2 * (kMaxGroups + 2) * 4;
-  static constexpr int STAGES_RAW = (kSmemBudget - 1024 - TABLE_BYTES - 512) / STAGE_BYTES;
+  static constexpr int OUT_WARP = kStageOut ? 8192 : 0;
+  static constexpr int STAGES_RAW = (kSmemBudget - 2048 - TABLE_BYTES - 512 - 4 * OUT_WARP) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = 2 * MMA_N;
-  static constexpr int SMEM = 1024 + STAGES * STAGE_BYTES + 512 + TABLE_BYTES;
+  static constexpr int OUTB = (STAGES * STAGE_BYTES + 512 + TABLE_BYTES + 1023) / 1024 * 1024;
+  static constexpr int SMEM = 1024 + OUTB + 4 * OUT_WARP;
 };
 
 struct Params {
@@ -139,10 +144,10 @@ __device__ __forceinline__ TileCoord decode_tile(const int* s_tile, const int* s
 template <int MMA_N, int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gg_bf16_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                   const __grid_constant__ CUtensorMap tmBx, const Params p) {
+                   const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC, const Params p) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
-  using L = Tile<MMA_N>;
+  using L = Tile<MMA_N, OUT == 0>;
   constexpr int OUT_COLS = EPI ? MMA_N / 2 : MMA_N;
   constexpr uint32_t IDESC = ptx::make_idesc(BM, MMA_N, 1);
 
@@ -412,62 +417,84 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       ptx::tc_fence_after();
       const uint32_t tacc = lane_base + acc * MMA_N;
-      if constexpr (EPI == 1) {
-        __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS;
+      if constexpr (OUT == 0) {
+        // bf16 output in 64-column boxes.  A warp whose 32 rows all belong to
+        // the group stages each box (128-byte swizzled, two buffers in turn)
+        // and writes it with a bulk tensor store; a slice crossing the
+        // group's end stores its valid rows directly.
+        const int r0 = tc.mb * BM + q * 32;
+        const bool slice_full = r0 + 32 <= m_g;
+        uint8_t* s_out = smem + L::OUTB + (warp - 2) * L::OUT_WARP;
 #pragma unroll 1
-        for (int c = 0; c < OUT_COLS; c += 32) {
-          uint32_t gv[32], uv[32];
-          ptx::tmem_ld_32x32b_x32(tacc + c, gv);
-          ptx::tmem_ld_32x32b_x32(tacc + OUT_COLS + c, uv);
-          ptx::tmem_ld_wait();
-          if (valid) {
-            uint32_t packed[16];
+        for (int b = 0; b < OUT_COLS / 64; ++b) {
+          uint32_t pk[32];
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const float g0 = __uint_as_float(gv[2 * i]), g1 = __uint_as_float(gv[2 * i + 1]);
-              const float h0 = silu(g0) * __uint_as_float(uv[2 * i]);
-              const float h1 = silu(g1) * __uint_as_float(uv[2 * i + 1]);
-              const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
-              packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
+          for (int h2 = 0; h2 < 2; ++h2) {
+            const int c = 64 * b + 32 * h2;
+            if constexpr (EPI == 1) {
+              uint32_t gv[32], uv[32];
+              ptx::tmem_ld_32x32b_x32(tacc + c, gv);
+              ptx::tmem_ld_32x32b_x32(tacc + OUT_COLS + c, uv);
+              ptx::tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const float h0 = silu(__uint_as_float(gv[2 * i])) * __uint_as_float(uv[2 * i]);
+                const float h1 = silu(__uint_as_float(gv[2 * i + 1])) * __uint_as_float(uv[2 * i + 1]);
+                const __nv_bfloat162 hb = __floats2bfloat162_rn(h0, h1);
+                pk[16 * h2 + i] = *reinterpret_cast<const uint32_t*>(&hb);
+              }
+            } else {
+              uint32_t v[32];
+              ptx::tmem_ld_32x32b_x32(tacc + c, v);
+              ptx::tmem_ld_wait();
+#pragma unroll
+              for (int i = 0; i < 16; ++i) {
+                const __nv_bfloat162 hb =
+                    __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
+                pk[16 * h2 + i] = *reinterpret_cast<const uint32_t*>(&hb);
+              }
             }
-            uint4* dst = reinterpret_cast<uint4*>(C + c);
+          }
+          if (slice_full) {
+            uint8_t* buf = s_out + (b & 1) * 4096;
+            if (lane == 0) ptx::bulk_wait_read_allow1();  // the store that used this buffer has read it
+            __syncwarp();
 #pragma unroll
-            for (int v = 0; v < 4; ++v)
-              dst[v] = make_uint4(packed[4 * v], packed[4 * v + 1], packed[4 * v + 2], packed[4 * v + 3]);
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(buf + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+            ptx::fence_proxy_async_smem();
+            __syncwarp();
+            if (lane == 0) {
+              ptx::tma_store_2d(&tmC, buf, nb * OUT_COLS + 64 * b, s_off[g] + r0);
+              ptx::bulk_commit_group();
+            }
+          } else if (valid) {
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS +
+                                                  64 * b);
+#pragma unroll
+            for (int c = 0; c < 8; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
           }
         }
       } else {
+        // fp32 output (router logits, split-K partial products): direct stores
 #pragma unroll 1
         for (int c = 0; c < OUT_COLS; c += 32) {
           uint32_t v[32];
           ptx::tmem_ld_32x32b_x32(tacc + c, v);
           ptx::tmem_ld_wait();
           if (valid) {
-            if constexpr (OUT == 1) {
-              float* C = static_cast<float*>(p.C) + tc.ks * p.split_stride + grow * p.N + nb * OUT_COLS + c;
-              uint4* dst = reinterpret_cast<uint4*>(C);
+            float* C = static_cast<float*>(p.C) + tc.ks * p.split_stride + grow * p.N + nb * OUT_COLS + c;
+            uint4* dst = reinterpret_cast<uint4*>(C);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
-            } else {
-              __nv_bfloat16* C = static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * OUT_COLS + c;
-              uint32_t packed[16];
-#pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const __nv_bfloat162 hb =
-                    __floats2bfloat162_rn(__uint_as_float(v[2 * i]), __uint_as_float(v[2 * i + 1]));
-                packed[i] = *reinterpret_cast<const uint32_t*>(&hb);
-              }
-              uint4* dst = reinterpret_cast<uint4*>(C);
-#pragma unroll
-              for (int i = 0; i < 4; ++i)
-                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
-            }
+            for (int i = 0; i < 8; ++i) dst[i] = make_uint4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
           }
         }
       }
       ptx::tc_fence_before();
       ptx::mbar_arrive(&tempty[acc]);
     }
+    if (OUT == 0 && lane == 0) ptx::bulk_wait_all();  // this warp's stores are complete before the CTA exits
   }
 
   ptx::tc_fence_before();
@@ -1524,18 +1551,28 @@ __global__ void __launch_bounds__(kThreadsF8, 1)
 constexpr int kThreadsMX = 352;  // TMA producer, MMA issuer, 8 epilogue warps, scale-factor warp
 constexpr int kMXSfWarp = 10;
 
-template <int EPI>
+template <int EPI, int OUT>
 struct MXSmem {
   static constexpr int A_BYTES = BM * 128;
   static constexpr int B_BYTES = 256 * 128;
   static constexpr int SF_BYTES = 3 * 512;  // A atom, two B atoms
-  static constexpr int STAGES = 4;
+  static constexpr int STAGE_ALL = A_BYTES + B_BYTES + SF_BYTES;
+  // output staging per epilogue warp (32 rows of its column half) for the
+  // bulk tensor stores: bf16 128 columns (two 128-byte boxes), bf16 64
+  // columns (one box) or E4M3 64 columns (64-byte rows)
+  static constexpr int OUT_WARP = EPI == 0 ? 8192 : (OUT == 2 ? 2048 : 4096);
+  static constexpr int FIXED = 512 + 2 * (kMaxGroups + 2) * 4 + 2 * 2 * 128 * 4 + 2048;  // + both alignments
+  static constexpr int STAGES_FIT = (227 * 1024 - FIXED - 8 * OUT_WARP) / STAGE_ALL;
+  static constexpr int STAGES = STAGES_FIT > 4 ? 4 : STAGES_FIT;
   static constexpr int SB = STAGES * A_BYTES;                   // B ring
   static constexpr int SFR = SB + STAGES * B_BYTES;             // scale-factor ring
-  static constexpr int BARS = SFR + STAGES * SF_BYTES;          // barriers and flags
+  static constexpr int OUTB = (SFR + STAGES * SF_BYTES + 1023) / 1024 * 1024;  // output staging
+  static constexpr int BARS = OUTB + 8 * OUT_WARP;              // barriers and flags
   static constexpr int TABLES = BARS + 512;                     // group offsets and tile prefix
   static constexpr int AMAX = TABLES + 2 * (kMaxGroups + 2) * 4;  // [2 parity][2 halves][128 rows]
   static constexpr int SMEM = AMAX + 2 * 2 * 128 * 4 + 1024;    // + alignment slack
+  static_assert(STAGES >= 3, "pipeline depth");
+  static_assert(OUTB % 1024 == 0, "128-byte swizzled staging needs 1024-byte alignment");
   static_assert(SMEM <= 227 * 1024, "shared memory budget");
 };
 
@@ -1548,10 +1585,10 @@ __device__ __forceinline__ uint32_t ue8m0_word(float s) {
 template <int EPI, int OUT>  // EPI 1: SiLU gate (OUT 0 bf16 / 2 MX e4m3); EPI 0: OUT 0 bf16
 __global__ void __launch_bounds__(kThreadsMX, 1)
     gg_mx_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                 const __grid_constant__ CUtensorMap tmBx, const Params p) {
+                 const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC, const Params p) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
-  using L = MXSmem<EPI>;
+  using L = MXSmem<EPI, OUT>;
   constexpr int MMA_N = 256;
   constexpr int OUT_COLS = EPI ? 128 : 256;
   constexpr uint32_t IDESC = ptx::make_idesc_mx(BM, MMA_N);
@@ -1868,6 +1905,15 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(tempty);  // the values are in registers: release the accumulator
+        // A warp whose 32 rows all belong to the group stages them in shared
+        // memory and writes them with a bulk tensor store; a slice crossing
+        // the group's end stores its valid rows one by one.
+        const bool slice_full = tc.mb * BM + q * 32 + 32 <= tc.m_g;
+        uint8_t* s_out = smem + L::OUTB + (warp - 2) * L::OUT_WARP;
+        if (slice_full) {
+          if (lane == 0) ptx::bulk_wait_read_all();  // the previous tile's store has read the buffer
+          __syncwarp();
+        }
         if constexpr (OUT == 2) {
           // E4M3 with one power-of-two scale per row per 128 columns: the two halves exchange amax
           float amax = 0.f;
@@ -1891,25 +1937,38 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
             const uint16_t hi = f32x2_to_e4m3x2(__fdiv_rn(h[4 * i + 2], sc), __fdiv_rn(h[4 * i + 3], sc));
             qw[i] = static_cast<uint32_t>(lo) | (static_cast<uint32_t>(hi) << 16);
           }
-          if (valid) {
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.C) + grow * p.N + nb * 128 + hf * 64);
+          if (valid && hf == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
+          uint4* dst = slice_full ? reinterpret_cast<uint4*>(s_out + lane * 64)  // 32 rows x 64 B
+                                  : reinterpret_cast<uint4*>(static_cast<uint8_t*>(p.C) + grow * p.N + nb * 128 +
+                                                             hf * 64);
+          if (slice_full || valid) {
 #pragma unroll
             for (int v = 0; v < 4; ++v) dst[v] = make_uint4(qw[4 * v], qw[4 * v + 1], qw[4 * v + 2], qw[4 * v + 3]);
-            if (hf == 0) p.C_scales[static_cast<size_t>(nb) * p.rows + grow] = sc;
           }
         } else {
-          if (valid) {
+          uint32_t pk[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            const __nv_bfloat162 hb = __floats2bfloat162_rn(h[2 * i], h[2 * i + 1]);
+            pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
+          }
+          if (slice_full) {  // 32 rows x 128 B, 16-byte chunk c of row r at chunk c ^ (r % 8)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(s_out + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          } else if (valid) {
             uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 128 + hf * 64);
 #pragma unroll
-            for (int v = 0; v < 8; ++v) {
-              uint32_t pk[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                const __nv_bfloat162 hb = __floats2bfloat162_rn(h[8 * v + 2 * i], h[8 * v + 2 * i + 1]);
-                pk[i] = *reinterpret_cast<const uint32_t*>(&hb);
-              }
-              dst[v] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            }
+            for (int c = 0; c < 8; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+          }
+        }
+        if (slice_full) {
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            ptx::tma_store_2d(&tmC, s_out, nb * 128 + hf * 64, s_off[g] + tc.mb * BM + q * 32);
+            ptx::bulk_commit_group();
           }
         }
       } else {
@@ -1929,13 +1988,35 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
         ptx::tc_fence_before();
         __syncwarp();
         if (lane == 0) ptx::mbar_arrive(tempty);
-        if (valid) {
+        const bool slice_full = tc.mb * BM + q * 32 + 32 <= tc.m_g;
+        uint8_t* s_out = smem + L::OUTB + (warp - 2) * L::OUT_WARP;
+        if (slice_full) {
+          if (lane == 0) ptx::bulk_wait_read_all();  // the previous tile's stores have read the buffer
+          __syncwarp();
+          // two boxes of 32 rows x 64 columns (128 B), 128-byte swizzled
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              *reinterpret_cast<uint4*>(s_out + b * 4096 + lane * 128 + ((c ^ (lane & 7)) << 4)) =
+                  make_uint4(pk[32 * b + 4 * c], pk[32 * b + 4 * c + 1], pk[32 * b + 4 * c + 2],
+                             pk[32 * b + 4 * c + 3]);
+          ptx::fence_proxy_async_smem();
+          __syncwarp();
+          if (lane == 0) {
+            const int y = s_off[g] + tc.mb * BM + q * 32;
+            ptx::tma_store_2d(&tmC, s_out, nb * 256 + hf * 128, y);
+            ptx::tma_store_2d(&tmC, s_out + 4096, nb * 256 + hf * 128 + 64, y);
+            ptx::bulk_commit_group();
+          }
+        } else if (valid) {
           uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.C) + grow * p.N + nb * 256 + hf * 128);
 #pragma unroll
           for (int v = 0; v < 16; ++v) dst[v] = make_uint4(pk[4 * v], pk[4 * v + 1], pk[4 * v + 2], pk[4 * v + 3]);
         }
       }
     }
+    if (lane == 0) ptx::bulk_wait_all();  // this warp's stores are complete before the CTA exits
   }
 
   ptx::tc_fence_before();
@@ -2046,7 +2127,7 @@ bool a_map(CUtensorMap* m, const GemmArgs& a, int ebytes) {
 
 template <int MMA_N, int EPI, int OUT>
 int run_bf16(const GemmArgs& a, cudaStream_t s) {
-  using L = Tile<MMA_N>;
+  using L = Tile<MMA_N, OUT == 0>;
   static_assert(L::SMEM <= 227 * 1024, "shared memory budget");
   const int nb_rows = EPI ? 2 * a.N : a.N;
   const uint32_t box_b = EPI ? MMA_N / 2 : MMA_N;
@@ -2056,6 +2137,10 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
                                        : static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows;
   if (!make_map(&mB, a.B, 2, b_rows, a.K, box_b)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  // bf16 output: boxes of 32 rows x 64 columns for the epilogue's bulk tensor stores
+  CUtensorMap mC = mA;
+  if (OUT == 0 && !make_store_map(&mC, a.C, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.N, 64, 32, true))
+    return MOE_ERR_CUDA;
   static bool attr_set[64] = {};
   int dev = 0;
   MOE_CUDA_CHECK(cudaGetDevice(&dev));
@@ -2081,7 +2166,7 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   p.a_rows = a.a_rows;
   p.a_src_rows = a.a_src_rows;
   return launch_pdl(__func__, gg_bf16_kernel<MMA_N, EPI, OUT>, dim3(a.grid > 0 ? a.grid : num_sms()), dim3(kThreads),
-                    L::SMEM, s, mA, mB, mBx, p);
+                    L::SMEM, s, mA, mB, mBx, mC, p);
 }
 
 template <int EPI>
@@ -2220,13 +2305,17 @@ int run_fp8(const GemmArgs& a, cudaStream_t s) {
 
 template <int EPI, int OUT>
 int run_mx(const GemmArgs& a, cudaStream_t s) {
-  constexpr int kSmem = MXSmem<EPI>::SMEM;
+  constexpr int kSmem = MXSmem<EPI, OUT>::SMEM;
   const int nb_rows = EPI ? 2 * a.N : a.N;
   const uint32_t box_b = EPI ? 128 : 256;
   CUtensorMap mA, mB, mBx;
   if (!a_map(&mA, a, 1)) return MOE_ERR_CUDA;
   if (!make_map(&mB, a.B, 1, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 1, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
+  // output boxes of one epilogue warp: 32 rows x 64 columns (bf16 128-byte swizzled, or E4M3 64-byte rows)
+  CUtensorMap mC;
+  const uint64_t c_rows = static_cast<uint64_t>(a.rows > 0 ? a.rows : 1);
+  if (!make_store_map(&mC, a.C, OUT == 2 ? 1 : 2, c_rows, a.N, 64, 32, OUT != 2)) return MOE_ERR_CUDA;
   static bool attr_set[64] = {};
   int dev = 0;
   MOE_CUDA_CHECK(cudaGetDevice(&dev));
@@ -2251,7 +2340,8 @@ int run_mx(const GemmArgs& a, cudaStream_t s) {
   p.C_scales = a.C_scales;
   p.a_rows = a.a_rows;
   p.a_src_rows = a.a_src_rows;
-  return launch_pdl(__func__, gg_mx_kernel<EPI, OUT>, dim3(num_sms()), dim3(kThreadsMX), kSmem, s, mA, mB, mBx, p);
+  return launch_pdl(__func__, gg_mx_kernel<EPI, OUT>, dim3(num_sms()), dim3(kThreadsMX), kSmem, s, mA, mB, mBx, mC,
+                    p);
 }
 
 }  // namespace

@@ -93,6 +93,7 @@ int check_config(const moe_config* c) {
   if (c->d % 128 != 0 || c->inter % 128 != 0) return MOE_ERR_UNSUPPORTED;
   if (is_e4m3(c->expert_dtype) && c->d % 256 != 0) return MOE_ERR_UNSUPPORTED;
   if (c->capacity < 0) return MOE_ERR_INVALID;
+  if (c->flags & ~MOE_FLAG_GATHER_A) return MOE_ERR_INVALID;
   const long long rows = static_cast<long long>(c->T) * (c->k + 1);
   if (rows * c->d > (1ll << 40) || rows > kMaxPermuteRows) return MOE_ERR_UNSUPPORTED;
   return MOE_OK;
@@ -458,10 +459,11 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   if (st != MOE_OK) return st;
   if ((st = mark(1)) != MOE_OK) return st;
 
-  // "Permute in the load": when the up GEMM runs on a single-CTA kernel it
-  // gathers its A rows through row_to_token (tile::gather4), so the permute
-  // writes only the plan (plus, for E4M3 experts or fp32 x, each token's row
-  // once, quantised or cast) and the expert-ordered copy of x is never made.
+  // "Permute in the load" (MOE_FLAG_GATHER_A): when the up GEMM runs on a
+  // single-CTA kernel it gathers its A rows through row_to_token
+  // (tile::gather4), so the permute writes only the plan (plus, for E4M3
+  // experts or fp32 x, each token's row once, quantised or cast) and the
+  // expert-ordered copy of x is never made.
   GemmArgs up{};
   up.B = W1;
   up.B_extra = W1_shared;
@@ -476,7 +478,7 @@ int forward_impl(const moe_config* cfg, const void* x, const void* W_r, const fl
   up.c_dtype = fp8 ? qdt : MOE_BF16;
   up.C = base + L.h;
   up.status = status;
-  const bool gather = plan_takes_gathered_a(plan_grouped_gemm(up, num_sms()));
+  const bool gather = (c.flags & MOE_FLAG_GATHER_A) && plan_takes_gathered_a(plan_grouped_gemm(up, num_sms()));
   const bool x_as_is = gather && !fp8 && c.x_dtype == MOE_BF16;  // the GEMM reads x itself
 
   PermuteArgs pa;

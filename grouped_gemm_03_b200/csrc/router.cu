@@ -2,9 +2,8 @@
 //
 // "MegaMoE math model -> DeepGEMM source walk-through" §2.1 (p = Softmax(W_r x_t),
 // keep the k best) and "Dense GEMM -> GroupedGEMM -> TP MoE" §4.2 (route_tokens).
-// Up to 64 experts with a modest T*d*E: one launch, router_fused_kernel
-// (below), which streams x once and keeps every logit on chip.  Otherwise
-// two launches:
+// Up to 16 experts: one launch, router_fused_kernel (below), which streams
+// x once and keeps every logit on chip.  Otherwise two launches:
 //   logits  either the grouped-GEMM kernel on the tensor cores (bf16, large
 //           E and d: the logits GEMM is then near the compute ridge), split
 //           along K into fp32 partial products, or a SIMT kernel that keeps
@@ -365,21 +364,21 @@ int finish_dispatch(const void* parts, int nsplit, size_t stride, int pstride, c
   return MOE_ERR_UNSUPPORTED;
 }
 
-// ------------------------------------------------------------------ fused router (E <= 64)
+// ------------------------------------------------------------------ fused router (E <= 16)
 // One launch: logits, softmax and top-k ("MegaMoE ..." §2.1; the fused
 // logits + softmax kernel of "DeepSeek-R1 deployment on A100" §3.2 and the
 // warp-level top-k of "DeepSeek MoE architecture overview" §2.2).  The
 // logits of a few experts are a short dot product per token, bound by
-// reading x once: a warp takes TPW = 32 / EP tokens at a time (EP = E
-// rounded up to a power of two, at least 8; one token when EP = 64) and its
-// lanes split d into 16-byte chunks, lane l owning chunks l, l + 32, ...;
-// every lane accumulates TPW x EP partial logits in fp32 (packed FMAs), the
-// W_r chunk it needs coming through L1 and reused by the warp's TPW tokens,
-// and the next two chunks of x in flight.  A butterfly reduce-scatter over
-// the lanes leaves lane l with the full logit of (token l / EP, expert
-// l % EP) (EP = 64: experts 2l and 2l + 1 of the warp's one token), and the
-// EP lanes of a token run the softmax and k rounds of an arg-max on packed
-// (logit, ~index) keys, so ties go to the lower expert index.
+// reading x once: a warp takes TPW = 16 / EP tokens at a time (EP = E
+// rounded up to 8 or 16) and its lanes split d into 16-byte chunks, lane l
+// owning chunks l, l + 32, ...; every lane accumulates the 16 (token,
+// expert) partial logits in fp32 (packed FMAs on even / odd columns), the
+// W_r chunk it needs coming through L1 and reused by the warp's tokens,
+// with the next two chunks of x in flight.  A butterfly reduce-scatter over
+// lane bits 16..2 and a final exchange with the neighbouring lane leave
+// lanes 2i and 2i + 1 with the full logit of (token i / EP, expert i % EP);
+// the 2 EP lanes of a token run the softmax and k rounds of an arg-max on
+// packed (logit, ~index) keys, so ties go to the lower expert index.
 constexpr int kFusedWarps = 8;
 
 template <typename T>
@@ -412,7 +411,7 @@ struct Chunk8<float> {
 // lower half of v[0, S), the others the upper half, each adding the
 // partner's copy of the half it keeps; the kept half moves to v[0, S/2).
 template <int S>
-__device__ __forceinline__ void rs_level(float (&v)[64], int lane, int bit) {
+__device__ __forceinline__ void rs_level(float (&v)[16], int lane, int bit) {
   const bool up = lane & bit;
 #pragma unroll
   for (int i = 0; i < S / 2; ++i) {
@@ -423,33 +422,26 @@ __device__ __forceinline__ void rs_level(float (&v)[64], int lane, int bit) {
 }
 
 template <typename XT, typename WT, int EP>
-__global__ void __launch_bounds__(kFusedWarps * 32) router_fused_kernel(const XT* __restrict__ x,
-                                                                      const WT* __restrict__ Wr,
-                                                                      const float* __restrict__ bias, int T, int d,
-                                                                      int E, int k, int renorm,
-                                                                      float* __restrict__ logits_out,
-                                                                      int32_t* __restrict__ idx_out,
-                                                                      float* __restrict__ w_out) {
+__global__ void __launch_bounds__(kFusedWarps * 32, 2) router_fused_kernel(const XT* __restrict__ x,
+                                                                         const WT* __restrict__ Wr,
+                                                                         const float* __restrict__ bias, int T, int d,
+                                                                         int E, int k, int renorm,
+                                                                         float* __restrict__ logits_out,
+                                                                         int32_t* __restrict__ idx_out,
+                                                                         float* __restrict__ w_out) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
-  constexpr int TPW = EP >= 32 ? 1 : 32 / EP;
-  constexpr int NV = TPW * EP;          // partial logits per lane: 32, or 64 when EP = 64
-  constexpr int PER = NV / 32;          // logits per lane after the reduce-scatter
+  static_assert(EP == 8 || EP == 16, "8 or 16 (padded) experts");
+  constexpr int TPW = 16 / EP;  // tokens per warp
+  constexpr int G = 2 * EP;     // lanes of one token after the reduction
   constexpr float kLog2e = 1.4426950408889634f;
   const int lane = threadIdx.x & 31;
   const int nwarps = gridDim.x * kFusedWarps;
-  const int nchunk = d / 8;             // 8-element chunks per row
+  const int nchunk = d / 8;  // 8-element chunks per row
   for (int t0 = (blockIdx.x * kFusedWarps + (threadIdx.x >> 5)) * TPW; t0 < T; t0 += nwarps * TPW) {
-    // fp32 sums per (token, expert); with EP <= 32 two running sums (even and
-    // odd columns, packed FMAs) added at the end
-    constexpr bool kPair = NV == 32;
-    float2 acc2[kPair ? NV : 1];
-    float acc[64];
+    float2 acc2[16];  // (token j, expert e) at j * EP + e: running sums of even and odd columns
 #pragma unroll
-    for (int i = 0; i < NV; ++i) {
-      if constexpr (kPair) acc2[i] = make_float2(0.f, 0.f);
-      acc[i] = 0.f;
-    }
+    for (int i = 0; i < 16; ++i) acc2[i] = make_float2(0.f, 0.f);
     auto fetch = [&](Chunk8<XT>(&dst)[TPW], int c) {
 #pragma unroll
       for (int j = 0; j < TPW; ++j) {
@@ -475,17 +467,9 @@ __global__ void __launch_bounds__(kFusedWarps * 32) router_fused_kernel(const XT
         else
           w.zero();
 #pragma unroll
-        for (int j = 0; j < TPW; ++j) {
-          if constexpr (kPair) {
+        for (int j = 0; j < TPW; ++j)
 #pragma unroll
-            for (int i = 0; i < 4; ++i) acc2[j * EP + e] = __ffma2_rn(cur[j].pair(i), w.pair(i), acc2[j * EP + e]);
-          } else {
-            float2 a2 = make_float2(0.f, 0.f);
-#pragma unroll
-            for (int i = 0; i < 4; ++i) a2 = __ffma2_rn(cur[j].pair(i), w.pair(i), a2);
-            acc[j * EP + e] += a2.x + a2.y;
-          }
-        }
+          for (int i = 0; i < 4; ++i) acc2[j * EP + e] = __ffma2_rn(cur[j].pair(i), w.pair(i), acc2[j * EP + e]);
       }
 #pragma unroll
       for (int j = 0; j < TPW; ++j) {
@@ -493,61 +477,38 @@ __global__ void __launch_bounds__(kFusedWarps * 32) router_fused_kernel(const XT
         nxt[j] = after[j];
       }
     }
-    if constexpr (kPair) {
+    float acc[16];
 #pragma unroll
-      for (int i = 0; i < NV; ++i) acc[i] = acc2[i].x + acc2[i].y;
-    }
-    // reduce-scatter: afterwards acc[0, PER) of lane l are the logits of
-    // partial index [PER l, PER l + PER) (token (PER l) / EP, experts (PER l) % EP ...)
-    if constexpr (NV == 64) rs_level<64>(acc, lane, 16);
-    rs_level<32>(acc, lane, NV == 64 ? 8 : 16);
-    if constexpr (NV == 64) {
-      rs_level<16>(acc, lane, 4);
-      rs_level<8>(acc, lane, 2);
-      rs_level<4>(acc, lane, 1);
-    } else {
-      rs_level<16>(acc, lane, 8);
-      rs_level<8>(acc, lane, 4);
-      rs_level<4>(acc, lane, 2);
-      rs_level<2>(acc, lane, 1);
-    }
-    // the EP / PER lanes of a token: consecutive lanes, group size G
-    constexpr int G = EP / PER;
-    const int t = t0 + (lane * PER) / EP;
-    const int e_base = (lane * PER) % EP;
+    for (int i = 0; i < 16; ++i) acc[i] = acc2[i].x + acc2[i].y;
+    // reduce-scatter over lane bits 16, 8, 4, 2; then lanes 2i and 2i + 1 add
+    // their halves: both hold partial index i = lane / 2
+    rs_level<16>(acc, lane, 16);
+    rs_level<8>(acc, lane, 8);
+    rs_level<4>(acc, lane, 4);
+    rs_level<2>(acc, lane, 2);
+    const float logit = acc[0] + __shfl_xor_sync(0xffffffffu, acc[0], 1);
+    const int t = t0 + (lane >> 1) / EP;
+    const int e = (lane >> 1) % EP;
     const bool tok = t < T;
-    float v[PER];
-    uint64_t key[PER];
-    float m = -INFINITY;
-#pragma unroll
-    for (int i = 0; i < PER; ++i) {
-      const int e = e_base + i;
-      v[i] = acc[i];
-      if (!tok || e >= E) {
-        v[i] = -INFINITY;
-        key[i] = 0ull;
-      } else {
-        if (bias) v[i] += bias[e];
-        if (logits_out) logits_out[static_cast<size_t>(t) * E + e] = v[i];
-        key[i] = sel_key(v[i], e);
-      }
-      m = fmaxf(m, v[i]);
+    const bool real = tok && e < E;
+    float v = -INFINITY;
+    uint64_t key = 0ull;
+    if (real) {
+      v = logit + (bias ? bias[e] : 0.f);
+      if (logits_out && (lane & 1) == 0) logits_out[static_cast<size_t>(t) * E + e] = v;
+      key = sel_key(v, e);
     }
+    float m = v;
 #pragma unroll
     for (int o = G / 2; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-    float sum = 0.f;
-#pragma unroll
-    for (int i = 0; i < PER; ++i)
-      if (e_base + i < E) sum += exp2f((v[i] - m) * kLog2e);
+    float sum = (real && (lane & 1) == 0) ? exp2f((v - m) * kLog2e) : 0.f;  // each expert counted once
 #pragma unroll
     for (int o = G / 2; o; o >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, o);
     const float inv_sum = 1.0f / sum;
     const bool leader = (lane % G) == 0;
     float psum = 0.f;
     for (int r = 0; r < k; ++r) {
-      uint64_t best = 0;
-#pragma unroll
-      for (int i = 0; i < PER; ++i) best = key[i] > best ? key[i] : best;
+      uint64_t best = key;
 #pragma unroll
       for (int o = G / 2; o; o >>= 1) {
         const uint64_t other = __shfl_xor_sync(0xffffffffu, best, o);
@@ -559,8 +520,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32) router_fused_kernel(const XT
         idx_out[static_cast<size_t>(t) * k + r] = key_index(best);
         w_out[static_cast<size_t>(t) * k + r] = pr;
       }
-#pragma unroll
-      for (int i = 0; i < PER; ++i) key[i] = key[i] == best ? 0ull : key[i];
+      key = key == best ? 0ull : key;
     }
     if (renorm && tok && leader)
       for (int r = 0; r < k; ++r) w_out[static_cast<size_t>(t) * k + r] /= psum;
@@ -570,7 +530,7 @@ __global__ void __launch_bounds__(kFusedWarps * 32) router_fused_kernel(const XT
 template <typename XT, typename WT, int EP>
 int fused_launch(const void* x, const void* Wr, const float* bias, int T, int d, int E, int k, int renorm,
                  float* logits_out, int32_t* idx, float* w, cudaStream_t s) {
-  constexpr int TPW = EP >= 32 ? 1 : 32 / EP;
+  constexpr int TPW = 16 / EP;
   const int warps_needed = (T + TPW - 1) / TPW;
   const int blocks = max(1, min((warps_needed + kFusedWarps - 1) / kFusedWarps, num_sms() * 8));
   return launch_pdl("router_fused_kernel", router_fused_kernel<XT, WT, EP>, dim3(blocks), dim3(kFusedWarps * 32), 0,
@@ -582,9 +542,7 @@ template <typename XT, typename WT>
 int fused_dispatch(const void* x, const void* Wr, const float* bias, int T, int d, int E, int k, int renorm,
                    float* lo, int32_t* idx, float* w, cudaStream_t s) {
   if (E <= 8) return fused_launch<XT, WT, 8>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
-  if (E <= 16) return fused_launch<XT, WT, 16>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
-  if (E <= 32) return fused_launch<XT, WT, 32>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
-  return fused_launch<XT, WT, 64>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
+  return fused_launch<XT, WT, 16>(x, Wr, bias, T, d, E, k, renorm, lo, idx, w, s);
 }
 
 template <typename XT, typename WT>
@@ -607,7 +565,9 @@ bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E) {
 int router_padded_experts(int E) { return (E + 63) / 64 * 64; }
 
 bool router_is_fused(int T, int d, int E) {
-  return E <= 64 && (E <= 16 || static_cast<double>(T) * d * E <= static_cast<double>(1ll << 30));
+  (void)T;
+  (void)d;
+  return E <= 16;
 }
 
 int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d, int E,

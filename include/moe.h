@@ -80,12 +80,20 @@ typedef enum moe_epilogue {
  * factor of Dense GEMM -> GroupedGEMM -> TP MoE §5.1 (tokens over an
  * expert's capacity take a fallback path) and DeepSeek MoE architecture
  * overview §3.2 (a bound on one expert's share of a forward's tokens);
- * capacity = ceil(factor * T * k / E) for a capacity factor `factor`. */
+ * capacity = ceil(factor * T * k / E) for a capacity factor `factor`.
+ * flags: MOE_FLAG_GATHER_A makes the up GEMM gather its A rows through
+ * row_to_token in the load (moe_grouped_gemm_gather) whenever it runs on a
+ * single-CTA kernel, so the expert-ordered copy of x is not written; the
+ * result is identical.  It is off by default: on the fine-grained layer the
+ * gathered load (32 tile::gather4 per 128-row tile and k-step) measured
+ * slower than writing and re-reading the copy. */
+#define MOE_FLAG_GATHER_A 1
 typedef struct moe_config {
   int T, d, E, k, inter, shared_inter;
   int x_dtype, router_dtype, expert_dtype, out_dtype;
   int renormalize;
   int capacity;
+  int flags;
 } moe_config;
 
 /* Human-readable name of a status code (static string). */

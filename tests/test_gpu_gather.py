@@ -98,3 +98,34 @@ def test_gathered_gemm_with_overflowed_rows_and_fp32_out_rules():
     assert torch.equal(got[:used], want[:used])
     with pytest.raises(gg.MoEError):  # fp32 C runs on no gathering kernel
         gg.grouped_gemm_gather(x, r2t, B, plan["offsets"], N, c_dtype=torch.float32)
+
+
+@pytest.mark.parametrize("name,over", [
+    ("tiny", dict()),                                                        # fp32 x: cast once per token
+    ("tiny", dict(T=700, E=16, k=4, x_dtype="bf16", router_dtype="bf16")),   # bf16 x read as stored
+    ("tiny", dict(T=300, E=8, k=2, inter=256, fp8=True)),                    # E4M3 quantised once per token
+    ("tiny", dict(T=300, E=8, k=2, inter=256, fp8=True, mx=True, x_dtype="bf16", router_dtype="bf16")),
+])
+def test_forward_with_gathered_up_gemm_equals_the_default(name, over):
+    from workload import make_inputs, shape_of
+    s = shape_of(name, **over)
+    inp = make_inputs(s, seed=5, device=DEV)
+    xdt = gg.MOE_F32 if s.x_dtype == "f32" else gg.MOE_BF16
+    rdt = gg.MOE_F32 if s.router_dtype == "f32" else gg.MOE_BF16
+    edt = (gg.MOE_MXE4M3 if s.mx else gg.MOE_E4M3) if s.fp8 else gg.MOE_BF16
+    if s.fp8:
+        q = gg.quantize_weights_mx if s.mx else gg.quantize_weights_fp8
+        W1q, W1s = q(inp["W1"])
+        W2q, W2s = q(inp["W2"])
+        w = gg.ExpertWeights(W1=W1q, W2=W2q, W1_scales=W1s, W2_scales=W2s)
+        w.W1s, w.W1s_scales = q(inp["W1s"])
+        w.W2s, w.W2s_scales = q(inp["W2s"])
+    else:
+        w = gg.ExpertWeights(W1=inp["W1"], W2=inp["W2"], W1s=inp["W1s"], W2s=inp["W2s"])
+    outs = []
+    for flags in (0, gg.MOE_FLAG_GATHER_A):
+        cfg = gg.make_config(s.T, s.d, s.E, s.k, s.inter, s.shared_inter, xdt, rdt, edt, xdt, flags=flags)
+        ws = torch.empty(gg.workspace_size(cfg), dtype=torch.uint8, device=DEV)
+        outs.append(gg.moe_forward(cfg, inp["x"], inp["W_r"], inp["bias"], w, ws=ws).clone())
+        assert gg.read_device_status(ws) == 0
+    assert torch.equal(outs[0], outs[1])

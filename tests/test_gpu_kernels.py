@@ -100,8 +100,8 @@ def test_router_topk(name, T, renorm):
                                            (129, 512, 64, 8, torch.float32, torch.bfloat16),
                                            (513, 256, 8, 2, torch.bfloat16, torch.float32),
                                            (1, 8, 7, 7, torch.float32, torch.float32)])
-def test_fused_router_shapes(T, d, E, k, xdt, wdt):
-    # the one-launch router (E <= 64): ragged d, E not a power of two, mixed operand types
+def test_router_ragged_shapes(T, d, E, k, xdt, wdt):
+    # ragged d, E not a power of two, mixed operand types (E <= 16 runs the one-launch router)
     g = torch.Generator(device=DEV).manual_seed(T + d + E)
     x = torch.randn((T, d), device=DEV, generator=g).to(xdt)
     W = (torch.randn((E, d), device=DEV, generator=g) * 0.05).to(wdt)
@@ -117,7 +117,7 @@ def test_fused_router_shapes(T, d, E, k, xdt, wdt):
 
 
 @pytest.mark.parametrize("E,k", [(8, 2), (32, 5), (64, 8)])
-def test_fused_router_ties_go_to_the_lower_index(E, k):
+def test_router_ties_go_to_the_lower_index(E, k):
     # every expert row equal: all logits tie, so the selection is experts 0..k-1 in order
     x = torch.randn((300, 512), device=DEV).to(torch.bfloat16)
     W = (torch.randn((1, 512), device=DEV) * 0.05).to(torch.bfloat16).repeat(E, 1).contiguous()

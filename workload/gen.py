@@ -47,6 +47,7 @@ class MoEShape:
     router_dtype: str = "bf16"
     fp8: bool = False       # expert GEMMs in E4M3 with 1x128 / 128x128 scales
     mx: bool = False        # with fp8: power-of-two (MX) scales the tensor core applies
+    gather: bool = False    # the up GEMM gathers its A rows in the load (no expert-ordered copy of x)
     zipf_s: float = 0.0     # 0 = balanced router
     renormalize: bool = False
 
@@ -82,6 +83,9 @@ CONFIGS: dict[str, MoEShape] = {
                         fp8=True, mx=True),
     "fine_mx_skew": MoEShape("fine_mx_skew", T=4096, d=7168, E=256, k=8, inter=2048,
                              shared_inter=2048, fp8=True, mx=True, zipf_s=1.2),
+    # the fine-grained layer with the up GEMM gathering its rows in the load
+    "fine_gather": MoEShape("fine_gather", T=4096, d=7168, E=256, k=8, inter=2048, shared_inter=2048,
+                            gather=True),
     "decode": MoEShape("decode", T=128, d=2048, E=64, k=2, inter=1408, zipf_s=1.5),
 }
 
