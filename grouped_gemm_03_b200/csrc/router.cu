@@ -338,6 +338,100 @@ int finish_launch(const void* parts, int nsplit, size_t stride, int pstride, con
                     pstride, bias, N, E, k, renorm, lo, idx, w);
 }
 
+// ------------------------------------------------------------------ top-k of stored 16-bit logits
+// Thread per token ("DeepSeek MoE architecture overview" §2.2 gives each
+// token its own top-k selection): the thread keeps the token's E logits in
+// registers (16-byte loads), takes the max, the sum of exponentials and an
+// insertion into a list of the 8 largest, kept in (logit descending, expert
+// ascending) order: an entry moves down only for a strictly larger logit, so
+// of equal logits the lower expert index stays first.  E <= 256, E % 8 == 0,
+// k <= 8.
+constexpr int kTopkList = 8;
+
+// Element e of a row held as 16-byte words (e a compile-time constant after unrolling).
+template <typename LT, int NW>
+__device__ __forceinline__ float row_elem(const uint4 (&raw)[NW], int e) {
+  const uint4 q = raw[e >> 3];
+  const int c = (e >> 1) & 3;
+  const uint32_t u = c == 0 ? q.x : c == 1 ? q.y : c == 2 ? q.z : q.w;
+  const uint16_t b = static_cast<uint16_t>((e & 1) ? (u >> 16) : (u & 0xffffu));
+  return to_f32(*reinterpret_cast<const LT*>(&b));
+}
+
+template <typename LT, int EV>  // EV: experts rounded up to a multiple of 8 (registers)
+__global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ logits, int N, int E, int k, int renorm,
+                                                        int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+  pdl_wait();  // the preceding kernel on the stream is complete and visible
+  pdl_launch_dependents();
+  constexpr float kLog2e = 1.4426950408889634f;
+  const int t = blockIdx.x * blockDim.x + threadIdx.x;
+  if (t >= N) return;
+  const LT* row = logits + static_cast<size_t>(t) * E;
+  uint4 raw[EV / 8];
+#pragma unroll
+  for (int i = 0; i < EV / 8; ++i)
+    raw[i] = 8 * i < E ? __ldg(reinterpret_cast<const uint4*>(row) + i) : make_uint4(0, 0, 0, 0);
+  float m = -INFINITY;
+#pragma unroll
+  for (int e = 0; e < EV; ++e)
+    if (e < E) m = fmaxf(m, row_elem<LT>(raw, e));
+  float sum = 0.f;
+  float kv[kTopkList];
+  int ki[kTopkList];
+#pragma unroll
+  for (int j = 0; j < kTopkList; ++j) {
+    kv[j] = -INFINITY;
+    ki[j] = -1;
+  }
+#pragma unroll
+  for (int e = 0; e < EV; ++e) {
+    if (e < E) {
+      float v = row_elem<LT>(raw, e);
+      sum += exp2f((v - m) * kLog2e);
+      if (v > kv[kTopkList - 1] || ki[kTopkList - 1] < 0) {  // enters the list: sift it into place
+        int ie = e;
+#pragma unroll
+        for (int j = 0; j < kTopkList; ++j) {
+          if (ie >= 0 && (v > kv[j] || ki[j] < 0)) {
+            const float tv = kv[j];
+            const int ti = ki[j];
+            kv[j] = v;
+            ki[j] = ie;
+            v = tv;
+            ie = ti;
+          }
+        }
+      }
+    }
+  }
+  const float inv_sum = 1.0f / sum;
+  float psum = 0.f;
+#pragma unroll
+  for (int j = 0; j < kTopkList; ++j) {
+    if (j < k) {
+      const float pr = exp2f((kv[j] - m) * kLog2e) * inv_sum;
+      psum += pr;
+      idx_out[static_cast<size_t>(t) * k + j] = ki[j];
+      w_out[static_cast<size_t>(t) * k + j] = pr;
+    }
+  }
+  if (renorm)
+    for (int j = 0; j < k; ++j) w_out[static_cast<size_t>(t) * k + j] /= psum;
+}
+
+template <typename LT>
+int topk_rows_dispatch(const void* logits, int N, int E, int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
+  const dim3 grid((N + 255) / 256);
+  const LT* l = static_cast<const LT*>(logits);
+#define MOE_TOPK_ROWS(EVV) \
+  launch_pdl("topk_rows_kernel", topk_rows_kernel<LT, EVV>, grid, dim3(256), 0, s, l, N, E, k, renorm, idx, w)
+  if (E <= 32) return MOE_TOPK_ROWS(32);
+  if (E <= 64) return MOE_TOPK_ROWS(64);
+  if (E <= 128) return MOE_TOPK_ROWS(128);
+  return MOE_TOPK_ROWS(256);
+#undef MOE_TOPK_ROWS
+}
+
 template <typename LT>
 int finish_dispatch(const void* parts, int nsplit, size_t stride, int pstride, const float* bias, int N, int E, int k,
                     int renorm, float* lo, int32_t* idx, float* w, cudaStream_t s) {
@@ -632,6 +726,9 @@ int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, cons
 int launch_topk_logits(const void* logits, int dtype, int N, int E, int k, int renorm, int32_t* idx, float* w,
                        cudaStream_t s) {
   if (N == 0) return MOE_OK;
+  if ((dtype == MOE_F16 || dtype == MOE_BF16) && E % 8 == 0 && E <= 256 && k <= kTopkList)
+    return dtype == MOE_F16 ? topk_rows_dispatch<__half>(logits, N, E, k, renorm, idx, w, s)
+                            : topk_rows_dispatch<__nv_bfloat16>(logits, N, E, k, renorm, idx, w, s);
   if (dtype == MOE_F16) return finish_dispatch<__half>(logits, 1, 0, E, nullptr, N, E, k, renorm, nullptr, idx, w, s);
   if (dtype == MOE_F32) return finish_dispatch<float>(logits, 1, 0, E, nullptr, N, E, k, renorm, nullptr, idx, w, s);
   if (dtype == MOE_BF16)

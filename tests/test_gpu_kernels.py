@@ -56,6 +56,23 @@ def test_topk_logits(N, E, k, dtype, renorm):
     np.testing.assert_allclose(w.cpu().numpy(), want_w, rtol=2e-6, atol=1e-7)
 
 
+@pytest.mark.parametrize("E,k,dtype", [(8, 1, torch.float16), (24, 3, torch.bfloat16), (56, 8, torch.float16),
+                                       (128, 4, torch.float16), (200, 5, torch.bfloat16), (256, 8, torch.float16)])
+def test_topk_rows_with_many_ties(E, k, dtype):
+    # 16-bit logits, E % 8 == 0, E <= 256, k <= 8 run one thread per token; integer-valued logits tie
+    # often, so the order (logit descending, expert ascending) is exercised on every token
+    g = torch.Generator(device=DEV).manual_seed(E + k)
+    l = torch.randint(-3, 4, (5000, E), device=DEV, generator=g).to(dtype)
+    for renorm in (False, True):
+        idx, w = gg.topk_logits(l, k, renormalize=renorm)
+        torch.cuda.synchronize()
+        lf = f64(l)
+        want = oracle.topk_select(lf, k)
+        assert np.array_equal(idx.cpu().numpy(), want)
+        np.testing.assert_allclose(w.cpu().numpy(), oracle.gate_weights(oracle.softmax(lf), want, renorm),
+                                   rtol=2e-6, atol=1e-7)
+
+
 def test_topk_logits_ties_take_lower_index():
     l = torch.zeros((64, 32), dtype=torch.float16, device=DEV)
     l[:, 5] = 1.0
