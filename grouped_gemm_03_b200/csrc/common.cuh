@@ -108,7 +108,12 @@ struct PermuteArgs {
   // [T, d] with each token's row once (cast / quantised as xp_dtype says,
   // scales [d/128][T]); with bf16 x and a bf16 xp nothing is copied at all
   int gather = 0;
+  int fuse_scan = 0;  // set by launch_permute (permute_fuses_scan)
 };
+// The scatter computes the expert offsets and its block's bases itself from
+// the histogram (no separate scan launch) when the count matrix is this small.
+constexpr int kFusedScanCounts = 8192;
+bool permute_fuses_scan(int T, int E);
 int permute_blocks(int T);  // number of token blocks the permute kernels use
 int launch_permute(const PermuteArgs& a, cudaStream_t s);
 

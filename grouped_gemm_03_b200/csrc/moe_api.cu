@@ -577,7 +577,8 @@ int moe_forward_launches(const moe_config* cfg) {
   if (check_config(cfg) != MOE_OK) return -1;
   if (cfg->T == 0) return 0;
   const int router = router_is_fused(cfg->T, cfg->d, cfg->E) ? 1 : 2;  // fused, or logits + selection
-  return router + 3 /* histogram, scan, scatter */ + 2 /* grouped GEMMs */ + 1 /* combine */;
+  const int permute = permute_fuses_scan(cfg->T, cfg->E) ? 2 : 3;      // histogram, (scan,) scatter
+  return router + permute + 2 /* grouped GEMMs */ + 1 /* combine */;
 }
 
 size_t moe_host_staging_size(const moe_config* cfg) {

@@ -172,8 +172,66 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   const int xp_rows = a.gather ? a.T : rows_total;  // leading dimension of xp_scales
   const bool writer = blockIdx.y == 0;   // one column block writes the index maps
   __shared__ int s_used;  // rows the experts keep: the shared rows start there
+  // small count matrices: this block reduces the histogram itself (no scan launch)
+  __shared__ int s_tot[kMaxExperts];      // rows each expert keeps
+  __shared__ int s_pre[kMaxExperts];      // pairs of each expert in the blocks before this one
+  __shared__ int s_offx[kMaxExperts + 1];  // exclusive scan of s_tot
+  __shared__ int s_wsum[kPermThreads / 32];
+  const bool fused = a.fuse_scan;
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) s_idx[p] = a.idx[static_cast<size_t>(t0) * k + p];
-  if (threadIdx.x == 0) s_used = a.offsets[E];
+  if (fused) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_pre[e] = 0;
+    __syncthreads();
+    const int nblk = gridDim.x;
+    for (int i = threadIdx.x; i < nblk * E; i += blockDim.x) {
+      const int c = a.block_base[i];  // the histogram: cnt[b'][e] at b' * E + e
+      atomicAdd(&s_tot[i % E], c);
+      if (i / E < b) atomicAdd(&s_pre[i % E], c);
+    }
+    __syncthreads();
+    // kept rows per expert, then their exclusive scan (each thread 4 consecutive experts)
+    int v[4], loc = 0;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = 4 * threadIdx.x + u;
+      v[u] = e < E ? (a.capacity > 0 ? min(s_tot[e], a.capacity) : s_tot[e]) : 0;
+      loc += v[u];
+    }
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    int incl = loc;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += y;
+    }
+    if (lane == 31) s_wsum[warp] = incl;
+    __syncthreads();
+    int wpre = 0;
+    for (int w = 0; w < warp; ++w) wpre += s_wsum[w];
+    int run = wpre + incl - loc;
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int e = 4 * threadIdx.x + u;
+      if (e < E) {
+        s_offx[e] = run;
+        if (b == 0 && writer) {
+          a.counts[e] = v[u];
+          a.offsets[e] = run;
+        }
+      }
+      run += v[u];
+    }
+    if (threadIdx.x == blockDim.x - 1) {
+      s_offx[E] = run;  // the last thread's running sum is the total
+      s_used = run;
+      if (b == 0 && writer) {
+        a.offsets[E] = run;
+        if (a.shared) a.offsets[E + 1] = run + a.T;
+      }
+    }
+  } else if (threadIdx.x == 0) {
+    s_used = a.offsets[E];
+  }
   __syncthreads();
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
     const int tl = p / k, j = p % k;
@@ -182,9 +240,10 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
     if (e >= 0 && e < E) {
       int rank = 0;
       for (int q = 0; q < tl * k; ++q) rank += (s_idx[q] == e);
-      row = a.block_base[static_cast<size_t>(b) * E + e] + rank;
+      const int off_e = fused ? s_offx[e] : a.offsets[e];
+      row = (fused ? off_e + s_pre[e] : a.block_base[static_cast<size_t>(b) * E + e]) + rank;
       // past the expert's capacity: the pair overflows and gets no row
-      if (a.capacity > 0 && row - a.offsets[e] >= a.capacity) row = -1;
+      if (a.capacity > 0 && row - off_e >= a.capacity) row = -1;
       if (row >= R) row = 0;  // only reachable with invalid ids (status already set)
     }
     if (!a.gather) s_row[tl * nd + j] = row;
@@ -310,6 +369,10 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
 
 int permute_blocks(int T) { return (T + kTokPerBlock - 1) / kTokPerBlock; }
 
+bool permute_fuses_scan(int T, int E) {
+  return static_cast<long long>(permute_blocks(T)) * E <= kFusedScanCounts;
+}
+
 int launch_permute(const PermuteArgs& a, cudaStream_t s) {
   const int nblk = permute_blocks(a.T);
   if (a.T == 0) {
@@ -321,22 +384,26 @@ int launch_permute(const PermuteArgs& a, cudaStream_t s) {
   int st = launch_pdl("hist_kernel", hist_kernel, dim3(nblk), dim3(kPermThreads), sizeof(int) * a.E, s, a.idx, a.T,
                       a.E, a.k, a.block_base, a.status);
   if (st != MOE_OK) return st;
-  st = launch_pdl("scan_kernel", scan_kernel, dim3(1), dim3(1024), 0, s, a.block_base, nblk, a.E, a.T, a.shared,
-                  a.capacity, a.counts, a.offsets);
-  if (st != MOE_OK) return st;
+  PermuteArgs b = a;
+  b.fuse_scan = permute_fuses_scan(a.T, a.E) ? 1 : 0;
+  if (!b.fuse_scan) {
+    st = launch_pdl("scan_kernel", scan_kernel, dim3(1), dim3(1024), 0, s, a.block_base, nblk, a.E, a.T, a.shared,
+                    a.capacity, a.counts, a.offsets);
+    if (st != MOE_OK) return st;
+  }
   const bool fp8 = is_e4m3(a.xp_dtype);
   const bool mx = a.xp_dtype == MOE_MXE4M3;
   const bool copies = !(a.gather && !fp8 && a.x_dtype == MOE_BF16);
   const dim3 grid(nblk, copies ? (a.d + kScatterCols - 1) / kScatterCols : 1);
   const dim3 block(kPermThreads);
   if (a.x_dtype == MOE_BF16) {
-    if (!fp8) return launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, false>, grid, block, 0, s, a);
-    return mx ? launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true, true>, grid, block, 0, s, a)
-              : launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true>, grid, block, 0, s, a);
+    if (!fp8) return launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, false>, grid, block, 0, s, b);
+    return mx ? launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true, true>, grid, block, 0, s, b)
+              : launch_pdl("scatter_kernel", scatter_kernel<__nv_bfloat16, true>, grid, block, 0, s, b);
   }
-  if (!fp8) return launch_pdl("scatter_kernel", scatter_kernel<float, false>, grid, block, 0, s, a);
-  return mx ? launch_pdl("scatter_kernel", scatter_kernel<float, true, true>, grid, block, 0, s, a)
-            : launch_pdl("scatter_kernel", scatter_kernel<float, true>, grid, block, 0, s, a);
+  if (!fp8) return launch_pdl("scatter_kernel", scatter_kernel<float, false>, grid, block, 0, s, b);
+  return mx ? launch_pdl("scatter_kernel", scatter_kernel<float, true, true>, grid, block, 0, s, b)
+            : launch_pdl("scatter_kernel", scatter_kernel<float, true>, grid, block, 0, s, b);
 }
 
 }  // namespace moe
