@@ -1799,11 +1799,29 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
       int rowc[4];
 #pragma unroll
       for (int c = 0; c < 4; ++c) rowc[c] = a_source_row(p, min(a_row + lane + 32 * c, p.rows - 1));  // past A: any
+      // the scales of the next two k-steps are in flight while this one is written
+      float qa[2][4] = {}, qb[2][2] = {};
+      auto fetch = [&](float (&fa)[4], float (&fb)[2], int kb) {
+        if (kb < nk) {
+#pragma unroll
+          for (int c = 0; c < 4; ++c) fa[c] = __ldg(p.A_scales + kb * rstride + rowc[c]);
+          fb[0] = __ldg(sb0 + kb);
+          fb[1] = __ldg(sb1 + kb);
+        }
+      };
+      fetch(qa[0], qb[0], 0);
+      fetch(qa[1], qb[1], 1);
       for (int kb = 0; kb < nk; ++kb) {
         float sa[4];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) sa[c] = __ldg(p.A_scales + kb * rstride + rowc[c]);
-        const float b0 = __ldg(sb0 + kb), b1 = __ldg(sb1 + kb);
+        for (int c = 0; c < 4; ++c) {
+          sa[c] = qa[0][c];
+          qa[0][c] = qa[1][c];
+        }
+        const float b0 = qb[0][0], b1 = qb[0][1];
+        qb[0][0] = qb[1][0];
+        qb[0][1] = qb[1][1];
+        fetch(qa[1], qb[1], kb + 2);
         if (!ptx::mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag, kWaitLimitNs)) {
           ok = false;
           break;

@@ -103,8 +103,9 @@ def test_gathered_gemm_with_overflowed_rows_and_fp32_out_rules():
 @pytest.mark.parametrize("name,over", [
     ("tiny", dict()),                                                        # fp32 x: cast once per token
     ("tiny", dict(T=700, E=16, k=4, x_dtype="bf16", router_dtype="bf16")),   # bf16 x read as stored
-    ("tiny", dict(T=300, E=8, k=2, inter=256, fp8=True)),                    # E4M3 quantised once per token
-    ("tiny", dict(T=300, E=8, k=2, inter=256, fp8=True, mx=True, x_dtype="bf16", router_dtype="bf16")),
+    ("tiny", dict(T=300, E=8, k=2, inter=256, shared_inter=256, fp8=True)),  # E4M3 quantised once per token
+    ("tiny", dict(T=300, E=8, k=2, inter=256, shared_inter=256, fp8=True, mx=True, x_dtype="bf16",
+                  router_dtype="bf16")),
 ])
 def test_forward_with_gathered_up_gemm_equals_the_default(name, over):
     from workload import make_inputs, shape_of
