@@ -53,9 +53,11 @@ constexpr int BM = 128;
 constexpr int kThreads = 192;
 constexpr int kSmemBudget = 220 * 1024;
 
-// Shared memory of the single-CTA bf16 kernel.  With bf16 output each of the
-// four epilogue warps stages its 32 rows in two 4 KB boxes (32 rows x 64
-// columns, 128-byte swizzled) for bulk tensor stores, at OUTB.
+// Shared memory of the single-CTA bf16 kernel.  With bf16 output and no
+// gate, each of the four epilogue warps stages its 32 rows in two 4 KB boxes
+// (32 rows x 64 columns, 128-byte swizzled) for bulk tensor stores, at OUTB;
+// that takes one operand stage, which the gated kernel (half the output
+// columns) measured better kept.
 template <int MMA_N, bool kStageOut>
 struct Tile {
   static constexpr int A_BYTES = BM * 128;
@@ -147,9 +149,12 @@ __global__ void __launch_bounds__(kThreads, 1)
                    const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmC, const Params p) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
-  using L = Tile<MMA_N, OUT == 0>;
+  using L = Tile<MMA_N, OUT == 0 && EPI == 0>;
   constexpr int OUT_COLS = EPI ? MMA_N / 2 : MMA_N;
   constexpr uint32_t IDESC = ptx::make_idesc(BM, MMA_N, 1);
+  // 64-row MMA of a group's short last tile: its rows 16j + i (i < 16) land in
+  // TMEM lane 32j + i, the first half of each 32-lane quarter
+  constexpr uint32_t IDESC64 = ptx::make_idesc(64, MMA_N, 1);
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -361,7 +366,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         ptx::tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * MMA_N;
-        const int ks = decode_tile(s_tile, s_off, G, nt, tile).ks;
+        const TileCoord tcm = decode_tile(s_tile, s_off, G, nt, tile);
+        const int ks = tcm.ks;
+        // a group's last tile of at most 64 rows: a 64-row MMA (half the work)
+        const uint32_t idesc = tcm.m_g - tcm.mb * BM <= 64 ? IDESC64 : IDESC;
         const int kb0 = ks * nk / p.ksplit, kb1 = (ks + 1) * nk / p.ksplit;
         for (int kb = kb0; kb < kb1; ++kb) {
           if (!ptx::mbar_wait(&full[stage], phase, abort_flag, p.wait_ns)) {
@@ -373,7 +381,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = ptx::sw128_kmajor_desc(ptx::smem_u32(sB + stage * L::B_BYTES));
 #pragma unroll
           for (int kk = 0; kk < 4; ++kk)
-            ptx::umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, IDESC, (kb > kb0) || (kk > 0));
+            ptx::umma_f16(d_tmem, adesc + 2 * kk, bdesc + 2 * kk, idesc, (kb > kb0) || (kk > 0));
           ptx::umma_commit(&empty[stage]);
           if (++stage == L::STAGES) {
             stage = 0;
@@ -394,7 +402,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   } else {
     // -------------------------------------------------------------- epilogue
     const int q = warp & 3;  // TMEM lane quarter this warp may access
-    const int row_t = q * 32 + lane;
     const uint32_t lane_base = tmem_base + (static_cast<uint32_t>(q * 32) << 16);
     int it = 0;
     for (int tile = blockIdx.x; tile < total; tile += gridDim.x, ++it) {
@@ -402,6 +409,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t use = static_cast<uint32_t>(it >> 1);
       const TileCoord tc = decode_tile(s_tile, s_off, G, nt, tile);
       const int g = tc.g, nb = tc.nb, m_g = tc.m_g;
+      // the lane's row: q * 32 + lane, or after a 64-row MMA q * 16 + lane for lanes 0..15
+      const bool half = m_g - tc.mb * BM <= 64;
+      const int row_t = half ? (lane < 16 ? q * 16 + lane : BM) : q * 32 + lane;
       const int r_in = tc.mb * BM + row_t;
       const bool valid = r_in < m_g;
       const size_t grow = static_cast<size_t>(s_off[g] + r_in);
@@ -423,7 +433,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         // and writes it with a bulk tensor store; a slice crossing the
         // group's end stores its valid rows directly.
         const int r0 = tc.mb * BM + q * 32;
-        const bool slice_full = r0 + 32 <= m_g;
+        // (the gated output, half as wide, keeps the operand stage instead: direct stores)
+        const bool slice_full = L::OUT_WARP > 0 && !half && r0 + 32 <= m_g;
         uint8_t* s_out = smem + L::OUTB + (warp - 2) * L::OUT_WARP;
 #pragma unroll 1
         for (int b = 0; b < OUT_COLS / 64; ++b) {
@@ -494,7 +505,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ptx::tc_fence_before();
       ptx::mbar_arrive(&tempty[acc]);
     }
-    if (OUT == 0 && lane == 0) ptx::bulk_wait_all();  // this warp's stores are complete before the CTA exits
+    if (L::OUT_WARP > 0 && lane == 0) ptx::bulk_wait_all();  // this warp's stores are complete before the CTA exits
   }
 
   ptx::tc_fence_before();
@@ -2145,7 +2156,7 @@ bool a_map(CUtensorMap* m, const GemmArgs& a, int ebytes) {
 
 template <int MMA_N, int EPI, int OUT>
 int run_bf16(const GemmArgs& a, cudaStream_t s) {
-  using L = Tile<MMA_N, OUT == 0>;
+  using L = Tile<MMA_N, OUT == 0 && EPI == 0>;
   static_assert(L::SMEM <= 227 * 1024, "shared memory budget");
   const int nb_rows = EPI ? 2 * a.N : a.N;
   const uint32_t box_b = EPI ? MMA_N / 2 : MMA_N;
@@ -2157,7 +2168,8 @@ int run_bf16(const GemmArgs& a, cudaStream_t s) {
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, box_b)) return MOE_ERR_CUDA;
   // bf16 output: boxes of 32 rows x 64 columns for the epilogue's bulk tensor stores
   CUtensorMap mC = mA;
-  if (OUT == 0 && !make_store_map(&mC, a.C, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.N, 64, 32, true))
+  if (L::OUT_WARP > 0 &&
+      !make_store_map(&mC, a.C, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.N, 64, 32, true))
     return MOE_ERR_CUDA;
   static bool attr_set[64] = {};
   int dev = 0;

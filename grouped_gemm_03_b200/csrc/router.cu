@@ -364,13 +364,25 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ l
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
   constexpr float kLog2e = 1.4426950408889634f;
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= N) return;
-  const LT* row = logits + static_cast<size_t>(t) * E;
+  constexpr int RB = EV * 2 + 16;  // bytes per staged row: padded so 32 rows spread over the banks
+  extern __shared__ __align__(16) uint8_t s_rows[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t0 = (blockIdx.x * 8 + warp) * 32;  // the warp's 32 tokens
+  const int t = t0 + lane;
+  // the warp's rows are contiguous: copy them with coalesced 16-byte loads
+  uint8_t* rows = s_rows + warp * 32 * RB;
+  const int cpr = E / 8;  // 16-byte chunks per row
+  const int nrow = min(32, N - t0);
+  if (nrow <= 0) return;
+  const uint4* src = reinterpret_cast<const uint4*>(logits + static_cast<size_t>(t0) * E);
+  for (int q = lane; q < nrow * cpr; q += 32)
+    *reinterpret_cast<uint4*>(rows + (q / cpr) * RB + (q % cpr) * 16) = __ldg(src + q);
+  __syncwarp();
+  if (lane >= nrow) return;
   uint4 raw[EV / 8];
 #pragma unroll
   for (int i = 0; i < EV / 8; ++i)
-    raw[i] = 8 * i < E ? __ldg(reinterpret_cast<const uint4*>(row) + i) : make_uint4(0, 0, 0, 0);
+    raw[i] = 8 * i < E ? *reinterpret_cast<const uint4*>(rows + lane * RB + i * 16) : make_uint4(0, 0, 0, 0);
   float m = -INFINITY;
 #pragma unroll
   for (int e = 0; e < EV; ++e)
@@ -388,17 +400,21 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ l
     if (e < E) {
       float v = row_elem<LT>(raw, e);
       sum += exp2f((v - m) * kLog2e);
-      if (v > kv[kTopkList - 1] || ki[kTopkList - 1] < 0) {  // enters the list: sift it into place
+      if (v > kv[kTopkList - 1] || ki[kTopkList - 1] < 0) {  // enters the list
+        // it goes before the first entry it strictly exceeds (or the first
+        // empty slot); every entry from there on moves down one place
         int ie = e;
+        bool moving = false;
 #pragma unroll
         for (int j = 0; j < kTopkList; ++j) {
-          if (ie >= 0 && (v > kv[j] || ki[j] < 0)) {
+          if (ie >= 0 && (moving || v > kv[j] || ki[j] < 0)) {
             const float tv = kv[j];
             const int ti = ki[j];
             kv[j] = v;
             ki[j] = ie;
             v = tv;
             ie = ti;
+            moving = true;
           }
         }
       }
@@ -421,15 +437,19 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ l
 
 template <typename LT>
 int topk_rows_dispatch(const void* logits, int N, int E, int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
-  const dim3 grid((N + 255) / 256);
+  const dim3 grid((N + 255) / 256);  // 8 warps of 32 tokens per block
   const LT* l = static_cast<const LT*>(logits);
-#define MOE_TOPK_ROWS(EVV) \
-  launch_pdl("topk_rows_kernel", topk_rows_kernel<LT, EVV>, grid, dim3(256), 0, s, l, N, E, k, renorm, idx, w)
-  if (E <= 32) return MOE_TOPK_ROWS(32);
-  if (E <= 64) return MOE_TOPK_ROWS(64);
-  if (E <= 128) return MOE_TOPK_ROWS(128);
-  return MOE_TOPK_ROWS(256);
-#undef MOE_TOPK_ROWS
+  auto go = [&](auto kernel, int ev) {
+    const size_t smem = static_cast<size_t>(8) * 32 * (ev * 2 + 16);
+    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                               static_cast<int>(smem));
+    if (e != cudaSuccess) return record_cuda_error(e, "topk_rows_kernel smem");
+    return launch_pdl("topk_rows_kernel", kernel, grid, dim3(256), smem, s, l, N, E, k, renorm, idx, w);
+  };
+  if (E <= 32) return go(topk_rows_kernel<LT, 32>, 32);
+  if (E <= 64) return go(topk_rows_kernel<LT, 64>, 64);
+  if (E <= 128) return go(topk_rows_kernel<LT, 128>, 128);
+  return go(topk_rows_kernel<LT, 256>, 256);
 }
 
 template <typename LT>
