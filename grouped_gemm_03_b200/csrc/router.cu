@@ -439,17 +439,25 @@ template <typename LT>
 int topk_rows_dispatch(const void* logits, int N, int E, int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
   const dim3 grid((N + 255) / 256);  // 8 warps of 32 tokens per block
   const LT* l = static_cast<const LT*>(logits);
-  auto go = [&](auto kernel, int ev) {
+  // the shared-memory limit is raised once per device and variant (a host call, kept out of every launch)
+  static bool attr_set[4][64] = {};
+  int dev = 0;
+  MOE_CUDA_CHECK(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
+  auto go = [&](auto kernel, int ev, int slot) {
     const size_t smem = static_cast<size_t>(8) * 32 * (ev * 2 + 16);
-    const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                               static_cast<int>(smem));
-    if (e != cudaSuccess) return record_cuda_error(e, "topk_rows_kernel smem");
+    if (!attr_set[slot][dev]) {
+      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 static_cast<int>(smem));
+      if (e != cudaSuccess) return record_cuda_error(e, "topk_rows_kernel smem");
+      attr_set[slot][dev] = true;
+    }
     return launch_pdl("topk_rows_kernel", kernel, grid, dim3(256), smem, s, l, N, E, k, renorm, idx, w);
   };
-  if (E <= 32) return go(topk_rows_kernel<LT, 32>, 32);
-  if (E <= 64) return go(topk_rows_kernel<LT, 64>, 64);
-  if (E <= 128) return go(topk_rows_kernel<LT, 128>, 128);
-  return go(topk_rows_kernel<LT, 256>, 256);
+  if (E <= 32) return go(topk_rows_kernel<LT, 32>, 32, 0);
+  if (E <= 64) return go(topk_rows_kernel<LT, 64>, 64, 1);
+  if (E <= 128) return go(topk_rows_kernel<LT, 128>, 128, 2);
+  return go(topk_rows_kernel<LT, 256>, 256, 3);
 }
 
 template <typename LT>
