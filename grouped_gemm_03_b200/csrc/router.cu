@@ -348,23 +348,21 @@ int finish_launch(const void* parts, int nsplit, size_t stride, int pstride, con
 // k <= 8.
 constexpr int kTopkList = 8;
 
-// Element e of a row held as 16-byte words (e a compile-time constant after unrolling).
-template <typename LT, int NW>
-__device__ __forceinline__ float row_elem(const uint4 (&raw)[NW], int e) {
-  const uint4 q = raw[e >> 3];
-  const int c = (e >> 1) & 3;
-  const uint32_t u = c == 0 ? q.x : c == 1 ? q.y : c == 2 ? q.z : q.w;
-  const uint16_t b = static_cast<uint16_t>((e & 1) ? (u >> 16) : (u & 0xffffu));
+// Element i (0..7) of a 16-byte word of 16-bit logits.
+template <typename LT>
+__device__ __forceinline__ float chunk_elem(const uint4& q, int i) {
+  const uint32_t u = (i >> 1) == 0 ? q.x : (i >> 1) == 1 ? q.y : (i >> 1) == 2 ? q.z : q.w;
+  const uint16_t b = static_cast<uint16_t>((i & 1) ? (u >> 16) : (u & 0xffffu));
   return to_f32(*reinterpret_cast<const LT*>(&b));
 }
 
-template <typename LT, int EV>  // EV: experts rounded up to a multiple of 8 (registers)
+template <typename LT>
 __global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ logits, int N, int E, int k, int renorm,
                                                         int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
   constexpr float kLog2e = 1.4426950408889634f;
-  constexpr int RB = EV * 2 + 16;  // bytes per staged row: padded so 32 rows spread over the banks
+  const int RB = E * 2 + 16;  // bytes per staged row: padded so 32 rows spread over the banks
   extern __shared__ __align__(16) uint8_t s_rows[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t0 = (blockIdx.x * 8 + warp) * 32;  // the warp's 32 tokens
@@ -379,14 +377,14 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ l
     *reinterpret_cast<uint4*>(rows + (q / cpr) * RB + (q % cpr) * 16) = __ldg(src + q);
   __syncwarp();
   if (lane >= nrow) return;
-  uint4 raw[EV / 8];
-#pragma unroll
-  for (int i = 0; i < EV / 8; ++i)
-    raw[i] = 8 * i < E ? *reinterpret_cast<const uint4*>(rows + lane * RB + i * 16) : make_uint4(0, 0, 0, 0);
+  const uint8_t* mine = rows + lane * RB;
   float m = -INFINITY;
+#pragma unroll 1
+  for (int c = 0; c < cpr; ++c) {
+    const uint4 q = *reinterpret_cast<const uint4*>(mine + c * 16);
 #pragma unroll
-  for (int e = 0; e < EV; ++e)
-    if (e < E) m = fmaxf(m, row_elem<LT>(raw, e));
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, chunk_elem<LT>(q, i));
+  }
   float sum = 0.f;
   float kv[kTopkList];
   int ki[kTopkList];
@@ -395,15 +393,17 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ l
     kv[j] = -INFINITY;
     ki[j] = -1;
   }
+#pragma unroll 1
+  for (int c = 0; c < cpr; ++c) {
+    const uint4 q = *reinterpret_cast<const uint4*>(mine + c * 16);
 #pragma unroll
-  for (int e = 0; e < EV; ++e) {
-    if (e < E) {
-      float v = row_elem<LT>(raw, e);
+    for (int i = 0; i < 8; ++i) {
+      float v = chunk_elem<LT>(q, i);
       sum += exp2f((v - m) * kLog2e);
       if (v > kv[kTopkList - 1] || ki[kTopkList - 1] < 0) {  // enters the list
         // it goes before the first entry it strictly exceeds (or the first
         // empty slot); every entry from there on moves down one place
-        int ie = e;
+        int ie = 8 * c + i;
         bool moving = false;
 #pragma unroll
         for (int j = 0; j < kTopkList; ++j) {
@@ -438,26 +438,19 @@ __global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ l
 template <typename LT>
 int topk_rows_dispatch(const void* logits, int N, int E, int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
   const dim3 grid((N + 255) / 256);  // 8 warps of 32 tokens per block
-  const LT* l = static_cast<const LT*>(logits);
-  // the shared-memory limit is raised once per device and variant (a host call, kept out of every launch)
-  static bool attr_set[4][64] = {};
+  const size_t smem = static_cast<size_t>(8) * 32 * (E * 2 + 16);
+  // the shared-memory limit is raised once per device (a host call, kept out of every launch)
+  static bool attr_set[64] = {};
   int dev = 0;
   MOE_CUDA_CHECK(cudaGetDevice(&dev));
   if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
-  auto go = [&](auto kernel, int ev, int slot) {
-    const size_t smem = static_cast<size_t>(8) * 32 * (ev * 2 + 16);
-    if (!attr_set[slot][dev]) {
-      const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 static_cast<int>(smem));
-      if (e != cudaSuccess) return record_cuda_error(e, "topk_rows_kernel smem");
-      attr_set[slot][dev] = true;
-    }
-    return launch_pdl("topk_rows_kernel", kernel, grid, dim3(256), smem, s, l, N, E, k, renorm, idx, w);
-  };
-  if (E <= 32) return go(topk_rows_kernel<LT, 32>, 32, 0);
-  if (E <= 64) return go(topk_rows_kernel<LT, 64>, 64, 1);
-  if (E <= 128) return go(topk_rows_kernel<LT, 128>, 128, 2);
-  return go(topk_rows_kernel<LT, 256>, 256, 3);
+  if (!attr_set[dev]) {
+    MOE_CUDA_CHECK(cudaFuncSetAttribute(topk_rows_kernel<LT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                        8 * 32 * (256 * 2 + 16)));
+    attr_set[dev] = true;
+  }
+  return launch_pdl("topk_rows_kernel", topk_rows_kernel<LT>, grid, dim3(256), smem, s, static_cast<const LT*>(logits),
+                    N, E, k, renorm, idx, w);
 }
 
 template <typename LT>
