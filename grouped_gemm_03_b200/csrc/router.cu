@@ -16,8 +16,10 @@
 // sum of the selected ones when renormalising).
 #include <cfloat>
 #include <climits>
+#include <type_traits>
 
 #include "common.cuh"
+#include "ptx.cuh"
 
 namespace moe {
 namespace {
@@ -170,7 +172,8 @@ __global__ void __launch_bounds__(kRWarps * 32) logits_simt_kernel(const XT* __r
 // then lower expert index": the float's bits mapped to an order-preserving
 // unsigned integer in the high word, the complemented index in the low word.
 __device__ __forceinline__ uint64_t sel_key(float v, int e) {
-  const uint32_t u = __float_as_uint(v);
+  uint32_t u = __float_as_uint(v);
+  if ((u << 1) == 0u) u = 0u;  // -0 and +0 are the same logit: the lower index must win
   const uint32_t o = (u & 0x80000000u) ? ~u : (u | 0x80000000u);
   return (static_cast<uint64_t>(o) << 32) | static_cast<uint32_t>(~static_cast<uint32_t>(e));
 }
@@ -186,7 +189,8 @@ __device__ __forceinline__ int key_index(uint64_t key) {
 // one 32-bit key, 16-bit order-preserving value over the complemented index.
 template <typename LT>
 __device__ __forceinline__ uint32_t sel_key16(LT v, int e) {
-  const uint16_t u = *reinterpret_cast<const uint16_t*>(&v);
+  uint16_t u = *reinterpret_cast<const uint16_t*>(&v);
+  if ((u & 0x7fffu) == 0u) u = 0u;  // -0 and +0 are the same logit: the lower index must win
   const uint16_t o = (u & 0x8000u) ? static_cast<uint16_t>(~u) : static_cast<uint16_t>(u | 0x8000u);
   return (static_cast<uint32_t>(o) << 16) | static_cast<uint32_t>(0xffffu - e);
 }
@@ -339,118 +343,175 @@ int finish_launch(const void* parts, int nsplit, size_t stride, int pstride, con
 }
 
 // ------------------------------------------------------------------ top-k of stored 16-bit logits
-// Thread per token ("DeepSeek MoE architecture overview" §2.2 gives each
-// token its own top-k selection): the thread keeps the token's E logits in
-// registers (16-byte loads), takes the max, the sum of exponentials and an
-// insertion into a list of the 8 largest, kept in (logit descending, expert
-// ascending) order: an entry moves down only for a strictly larger logit, so
-// of equal logits the lower expert index stays first.  E <= 256, E % 8 == 0,
-// k <= 8.
+// "DeepSeek MoE architecture overview" §2.2 gives each token its own top-k
+// selection.  Two threads share a token, each over alternate 16-byte chunks of
+// its E logits, staged in shared memory.  A logit and its expert form one
+// 32-bit key: the logit's 16-bit order-preserving image over the complemented
+// index, so a larger key means "larger logit, then lower expert", and keys are
+// distinct.  Each thread keeps its K largest keys sorted with a branch-free
+// max/min insertion network (the lanes never diverge) along with the running
+// max logit and the sum of exponentials, rescaled whenever the max grows; the
+// two threads then merge their lists.  E <= 256 (the index fits 16 bits),
+// E % 8 == 0, k <= K <= 8.
 constexpr int kTopkList = 8;
+constexpr int kTopkWarps = 4;
+constexpr int kTopkRowsPerWarp = 16;
 
-// Element i (0..7) of a 16-byte word of 16-bit logits.
+// Order-preserving images of the two 16-bit floats of a word, two at a time:
+// a positive half h maps to h | 0x8000, a negative one to 0x10000 - h, so -0
+// and +0 share the image 0x8000 (the +1 of the negation never carries out of
+// a negative half, whose complement is at most 0x7fff).  And back, for one.
+__device__ __forceinline__ uint32_t ord16x2(uint32_t w) {
+  const uint32_t neg = (w >> 15) & 0x00010001u;
+  return (w ^ ((neg * 0xffffu) | 0x80008000u)) + neg;
+}
+__device__ __forceinline__ uint32_t unord16(uint32_t o) { return (o & 0x8000u) ? (o & 0x7fffu) : (0x10000u - o); }
 template <typename LT>
-__device__ __forceinline__ float chunk_elem(const uint4& q, int i) {
-  const uint32_t u = (i >> 1) == 0 ? q.x : (i >> 1) == 1 ? q.y : (i >> 1) == 2 ? q.z : q.w;
-  const uint16_t b = static_cast<uint16_t>((i & 1) ? (u >> 16) : (u & 0xffffu));
+__device__ __forceinline__ float bits16_f32(uint32_t u) {
+  const uint16_t b = static_cast<uint16_t>(u);
   return to_f32(*reinterpret_cast<const LT*>(&b));
 }
-
 template <typename LT>
-__global__ void __launch_bounds__(256) topk_rows_kernel(const LT* __restrict__ logits, int N, int E, int k, int renorm,
-                                                        int32_t* __restrict__ idx_out, float* __restrict__ w_out) {
+__device__ __forceinline__ float2 word_f32x2(uint32_t w) {
+  if constexpr (std::is_same<LT, __half>::value) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
+  } else {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
+}
+// 2^x by the SFU's approximation (relative error about 2^-22; results below
+// the normal range flush to zero, far under a softmax term's tolerance)
+__device__ __forceinline__ float sfu_exp2(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// insert a key into a descending list of K distinct keys (the smallest falls off)
+template <int K>
+__device__ __forceinline__ void insert_key(uint32_t (&b)[K], uint32_t x) {
+#pragma unroll
+  for (int j = 0; j < K; ++j) {
+    const uint32_t hi = max(b[j], x);
+    x = min(b[j], x);
+    b[j] = hi;
+  }
+}
+
+template <typename LT, int K>
+__global__ void __launch_bounds__(kTopkWarps * 32) topk_rows_kernel(const LT* __restrict__ logits, int N, int E, int k,
+                                                                    int renorm, int32_t* __restrict__ idx_out,
+                                                                    float* __restrict__ w_out) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
   constexpr float kLog2e = 1.4426950408889634f;
-  const int RB = E * 2 + 16;  // bytes per staged row: padded so 32 rows spread over the banks
+  const int RB = E * 2 + 32;  // bytes per staged row: the pad spreads a warp's rows over the banks
   extern __shared__ __align__(16) uint8_t s_rows[];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int t0 = (blockIdx.x * 8 + warp) * 32;  // the warp's 32 tokens
-  const int t = t0 + lane;
-  // the warp's rows are contiguous: copy them with coalesced 16-byte loads
-  uint8_t* rows = s_rows + warp * 32 * RB;
-  const int cpr = E / 8;  // 16-byte chunks per row
-  const int nrow = min(32, N - t0);
+  const int t0 = (blockIdx.x * kTopkWarps + warp) * kTopkRowsPerWarp;  // the warp's 16 tokens
+  const int nrow = min(kTopkRowsPerWarp, N - t0);
   if (nrow <= 0) return;
-  const uint4* src = reinterpret_cast<const uint4*>(logits + static_cast<size_t>(t0) * E);
-  for (int q = lane; q < nrow * cpr; q += 32)
-    *reinterpret_cast<uint4*>(rows + (q / cpr) * RB + (q % cpr) * 16) = __ldg(src + q);
+  uint8_t* rows = s_rows + warp * kTopkRowsPerWarp * RB;
+  int32_t* s_idx = reinterpret_cast<int32_t*>(s_rows + kTopkWarps * kTopkRowsPerWarp * RB) +
+                   warp * kTopkRowsPerWarp * kTopkList;
+  float* s_w = reinterpret_cast<float*>(s_idx + (kTopkWarps - warp) * kTopkRowsPerWarp * kTopkList) +
+               warp * kTopkRowsPerWarp * kTopkList;
+  // the warp's rows are contiguous: all of them in flight at once, 16 bytes a
+  // copy; q / cpr as (q * ceil(2^16 / cpr)) >> 16, exact for q < 2^16 / cpr
+  // (here q < 16 * cpr <= 512 and cpr <= 32)
+  const int cpr = E / 8;  // 16-byte chunks per row
+  const int inv_cpr = (65536 + cpr - 1) / cpr;
+  const uint8_t* src = reinterpret_cast<const uint8_t*>(logits + static_cast<size_t>(t0) * E);
+  for (int q = lane; q < nrow * cpr; q += 32) {
+    const int r = (q * inv_cpr) >> 16;
+    ptx::cp_async_16(rows + r * RB + (q - r * cpr) * 16, src + q * 16);
+  }
+  ptx::cp_async_wait_all();
   __syncwarp();
-  if (lane >= nrow) return;
-  const uint8_t* mine = rows + lane * RB;
-  float m = -INFINITY;
+  const int j = lane >> 1, h = lane & 1;
+  if (j >= nrow) return;
+  const uint32_t pm = 3u << (2 * j);  // the token's two lanes
+  const uint8_t* mine = rows + j * RB;
+
+  uint32_t b[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) b[i] = 0u;  // below every key (a key's low half is at least 0xff00)
+  float m = -INFINITY, sum = 0.f;
 #pragma unroll 1
-  for (int c = 0; c < cpr; ++c) {
+  for (int c = h; c < cpr; c += 2) {
     const uint4 q = *reinterpret_cast<const uint4*>(mine + c * 16);
+    const uint32_t w[4] = {q.x, q.y, q.z, q.w};
+    const uint32_t base = 0xffffu - 8u * c;  // low 3 bits set: base - i == base ^ i
 #pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, chunk_elem<LT>(q, i));
-  }
-  float sum = 0.f;
-  float kv[kTopkList];
-  int ki[kTopkList];
-#pragma unroll
-  for (int j = 0; j < kTopkList; ++j) {
-    kv[j] = -INFINITY;
-    ki[j] = -1;
-  }
-#pragma unroll 1
-  for (int c = 0; c < cpr; ++c) {
-    const uint4 q = *reinterpret_cast<const uint4*>(mine + c * 16);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float v = chunk_elem<LT>(q, i);
-      sum += exp2f((v - m) * kLog2e);
-      if (v > kv[kTopkList - 1] || ki[kTopkList - 1] < 0) {  // enters the list
-        // it goes before the first entry it strictly exceeds (or the first
-        // empty slot); every entry from there on moves down one place
-        int ie = 8 * c + i;
-        bool moving = false;
-#pragma unroll
-        for (int j = 0; j < kTopkList; ++j) {
-          if (ie >= 0 && (moving || v > kv[j] || ki[j] < 0)) {
-            const float tv = kv[j];
-            const int ti = ki[j];
-            kv[j] = v;
-            ki[j] = ie;
-            v = tv;
-            ie = ti;
-            moving = true;
-          }
-        }
-      }
+    for (int jj = 0; jj < 4; ++jj) {
+      const uint32_t o = ord16x2(w[jj]);
+      insert_key<K>(b, (o << 16) | (base ^ (2 * jj)));
+      insert_key<K>(b, (o & 0xffff0000u) | (base ^ (2 * jj + 1)));
     }
+    // the running max logit is the value of the largest key
+    const float mn = bits16_f32<LT>(unord16(b[0] >> 16));
+    const float mnl = mn * kLog2e;
+    float s = sum * sfu_exp2(m * kLog2e - mnl);
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const float2 f = word_f32x2<LT>(w[jj]);
+      s += sfu_exp2(fmaf(f.x, kLog2e, -mnl));
+      s += sfu_exp2(fmaf(f.y, kLog2e, -mnl));
+    }
+    sum = s;
+    m = mn;
   }
+  // merge the two threads' lists and sums (both lanes end with the same ones)
+  uint32_t other[K];
+#pragma unroll
+  for (int i = 0; i < K; ++i) other[i] = __shfl_xor_sync(pm, b[i], 1);
+#pragma unroll
+  for (int i = 0; i < K; ++i) insert_key<K>(b, other[i]);
+  {
+    const float mo = __shfl_xor_sync(pm, m, 1), so = __shfl_xor_sync(pm, sum, 1);
+    const float mn = fmaxf(m, mo);
+    sum = sum * sfu_exp2((m - mn) * kLog2e) + so * sfu_exp2((mo - mn) * kLog2e);
+    m = mn;
+  }
+  // probabilities of the picks (softmax over all E), optionally renormalised
   const float inv_sum = 1.0f / sum;
+  float pr[K];
   float psum = 0.f;
 #pragma unroll
-  for (int j = 0; j < kTopkList; ++j) {
-    if (j < k) {
-      const float pr = exp2f((kv[j] - m) * kLog2e) * inv_sum;
-      psum += pr;
-      idx_out[static_cast<size_t>(t) * k + j] = ki[j];
-      w_out[static_cast<size_t>(t) * k + j] = pr;
+  for (int r = 0; r < K; ++r) {
+    if (r < k) {
+      pr[r] = exp2f((bits16_f32<LT>(unord16(b[r] >> 16)) - m) * kLog2e) * inv_sum;
+      psum += pr[r];
     }
   }
-  if (renorm)
-    for (int j = 0; j < k; ++j) w_out[static_cast<size_t>(t) * k + j] /= psum;
+#pragma unroll
+  for (int r = 0; r < K; ++r) {
+    if (r < k && (r & 1) == h) {
+      s_idx[j * k + r] = 0xffff - static_cast<int>(b[r] & 0xffffu);
+      s_w[j * k + r] = renorm ? pr[r] / psum : pr[r];
+    }
+  }
+  // the warp's k*nrow outputs are contiguous: store them coalesced
+  const int live = 2 * nrow;
+  __syncwarp(live == 32 ? 0xffffffffu : (1u << live) - 1u);
+  for (int q = lane; q < nrow * k; q += live) {
+    idx_out[static_cast<size_t>(t0) * k + q] = s_idx[q];
+    w_out[static_cast<size_t>(t0) * k + q] = s_w[q];
+  }
 }
 
 template <typename LT>
 int topk_rows_dispatch(const void* logits, int N, int E, int k, int renorm, int32_t* idx, float* w, cudaStream_t s) {
-  const dim3 grid((N + 255) / 256);  // 8 warps of 32 tokens per block
-  const size_t smem = static_cast<size_t>(8) * 32 * (E * 2 + 16);
-  // the shared-memory limit is raised once per device (a host call, kept out of every launch)
-  static bool attr_set[64] = {};
-  int dev = 0;
-  MOE_CUDA_CHECK(cudaGetDevice(&dev));
-  if (dev < 0 || dev >= 64) return MOE_ERR_UNSUPPORTED;
-  if (!attr_set[dev]) {
-    MOE_CUDA_CHECK(cudaFuncSetAttribute(topk_rows_kernel<LT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                        8 * 32 * (256 * 2 + 16)));
-    attr_set[dev] = true;
-  }
-  return launch_pdl("topk_rows_kernel", topk_rows_kernel<LT>, grid, dim3(256), smem, s, static_cast<const LT*>(logits),
-                    N, E, k, renorm, idx, w);
+  constexpr int kTokensPerBlock = kTopkWarps * kTopkRowsPerWarp;
+  const dim3 grid((N + kTokensPerBlock - 1) / kTokensPerBlock);
+  // staged rows plus the outputs: 38,912 bytes at E = 256, under the default limit
+  const size_t smem = static_cast<size_t>(kTokensPerBlock) * (E * 2 + 32) +
+                      static_cast<size_t>(kTokensPerBlock) * kTopkList * 8;
+  const LT* l = static_cast<const LT*>(logits);
+  const dim3 block(kTopkWarps * 32);
+  if (k == 1) return launch_pdl("topk_rows_kernel", topk_rows_kernel<LT, 1>, grid, block, smem, s, l, N, E, k, renorm, idx, w);
+  if (k == 2) return launch_pdl("topk_rows_kernel", topk_rows_kernel<LT, 2>, grid, block, smem, s, l, N, E, k, renorm, idx, w);
+  if (k <= 4) return launch_pdl("topk_rows_kernel", topk_rows_kernel<LT, 4>, grid, block, smem, s, l, N, E, k, renorm, idx, w);
+  return launch_pdl("topk_rows_kernel", topk_rows_kernel<LT, 8>, grid, block, smem, s, l, N, E, k, renorm, idx, w);
 }
 
 template <typename LT>
