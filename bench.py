@@ -282,13 +282,13 @@ def traffic_from_profile(workload, stage, kernel_src_hash):
     return d.get("bytes_per_launch")
 
 
-STAGE_SOURCES = {"router": "router.cu", "permute": "permute.cu", "up_gemm": "grouped_gemm.cu",
-                 "down_gemm": "grouped_gemm.cu", "combine": "combine.cu"}
+STAGE_SOURCES = {"router": ("router.cu", "router_tc.cu"), "permute": ("permute.cu",),
+                 "up_gemm": ("grouped_gemm.cu",), "down_gemm": ("grouped_gemm.cu",), "combine": ("combine.cu",)}
 
 
 def kernel_source_hash(stage):
     h = hashlib.sha256()
-    for f in (STAGE_SOURCES[stage], "ptx.cuh", "common.cuh"):
+    for f in STAGE_SOURCES[stage] + ("ptx.cuh", "common.cuh"):
         h.update(open(os.path.join(ROOT, "grouped_gemm_03_b200", "csrc", f), "rb").read())
     return h.hexdigest()
 

@@ -85,7 +85,12 @@ int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, cons
                   int k, int renorm, float* logits_out, int32_t* idx, float* w, float* parts, int* status,
                   cudaStream_t s);
 bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E);
-bool router_is_fused(int T, int d, int E);  // one launch (logits + softmax + top-k on chip)
+// one launch (logits + softmax + top-k on chip)
+bool router_is_fused(int x_dtype, int w_dtype, int T, int d, int E, int k);
+// the tensor-core router (router_tc.cu): bf16 x and W_r, E <= 256, k <= 8
+bool router_tc_applies(int x_dtype, int w_dtype, int d, int E, int k);
+int launch_router_tc(const void* x, const void* W_r, const float* bias, int T, int d, int E, int k, int renorm,
+                     float* logits_out, int32_t* idx, float* w, int* status, cudaStream_t s);
 int router_padded_experts(int E);  // logits columns the tensor-core router computes
 int launch_topk_logits(const void* logits, int dtype, int N, int E, int k, int renorm, int32_t* idx,
                        float* w, cudaStream_t s);

@@ -2057,6 +2057,8 @@ __global__ void __launch_bounds__(kThreadsMX, 1)
 }
 
 // ------------------------------------------------------------------ host side
+}  // namespace
+
 using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
                                    const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
@@ -2095,6 +2097,8 @@ bool make_map(CUtensorMap* m, const void* base, int ebytes, uint64_t rows, uint6
   }
   return true;
 }
+
+namespace {
 
 // 2-D map over a row-major [rows, cols] output for tiled bulk stores of
 // {box_cols, box_rows} boxes (box_cols * ebytes = 128 with 128-byte swizzle).

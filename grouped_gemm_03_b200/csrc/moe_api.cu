@@ -576,7 +576,8 @@ int moe_forward_marked(const moe_config* cfg, const void* x, const void* W_r, co
 int moe_forward_launches(const moe_config* cfg) {
   if (check_config(cfg) != MOE_OK) return -1;
   if (cfg->T == 0) return 0;
-  const int router = router_is_fused(cfg->T, cfg->d, cfg->E) ? 1 : 2;  // fused, or logits + selection
+  const int router =
+      router_is_fused(cfg->x_dtype, cfg->router_dtype, cfg->T, cfg->d, cfg->E, cfg->k) ? 1 : 2;  // or logits + selection
   const int permute = permute_fuses_scan(cfg->T, cfg->E) ? 2 : 3;      // histogram, (scan,) scatter
   return router + permute + 2 /* grouped GEMMs */ + 1 /* combine */;
 }

@@ -740,17 +740,18 @@ bool router_uses_tensor_cores(int x_dtype, int w_dtype, int T, int d, int E) {
 
 int router_padded_experts(int E) { return (E + 63) / 64 * 64; }
 
-bool router_is_fused(int T, int d, int E) {
+bool router_is_fused(int x_dtype, int w_dtype, int T, int d, int E, int k) {
   (void)T;
-  (void)d;
-  return E <= 16;
+  return router_tc_applies(x_dtype, w_dtype, d, E, k) || E <= 16;
 }
 
 int launch_router(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T, int d, int E,
                   int k, int renorm, float* logits_out, int32_t* idx, float* w, float* parts, int* status,
                   cudaStream_t s) {
   if (T == 0) return MOE_OK;
-  if (router_is_fused(T, d, E)) {
+  if (router_tc_applies(x_dtype, w_dtype, d, E, k))
+    return launch_router_tc(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, status, s);
+  if (E <= 16) {
     if (x_dtype == MOE_BF16 && w_dtype == MOE_BF16)
       return fused_dispatch<__nv_bfloat16, __nv_bfloat16>(x, W_r, bias, T, d, E, k, renorm, logits_out, idx, w, s);
     if (x_dtype == MOE_F32 && w_dtype == MOE_F32)

@@ -171,9 +171,13 @@ def test_forward_launch_count():
     mixtral = gg.make_config(T=4096, d=4096, E=8, k=2, inter=14336)
     fine = gg.make_config(T=4096, d=7168, E=256, k=8, inter=2048, shared_inter=2048)
     decode = gg.make_config(T=128, d=2048, E=64, k=2, inter=1408)
-    # fused router (E <= 16) and the scan folded into the scatter (ceil(T/32) * E <= 8192)
+    # one-launch router (bf16, E <= 256, k <= 8) and the scan folded into the
+    # scatter (ceil(T/32) * E <= 8192)
     assert L.moe_forward_launches(ctypes.byref(mixtral)) == 6
-    assert L.moe_forward_launches(ctypes.byref(decode)) == 7    # 64 experts: logits + selection
-    assert L.moe_forward_launches(ctypes.byref(fine)) == 8      # logits + selection, histogram + scan + scatter
+    assert L.moe_forward_launches(ctypes.byref(decode)) == 6
+    assert L.moe_forward_launches(ctypes.byref(fine)) == 7      # histogram + scan + scatter
+    # fp32 x with 64 experts: logits + selection
+    decode32 = gg.make_config(T=128, d=2048, E=64, k=2, inter=1408, x_dtype=gg.MOE_F32)
+    assert L.moe_forward_launches(ctypes.byref(decode32)) == 7
     assert L.moe_forward_launches(ctypes.byref(gg.make_config(T=0, d=256, E=8, k=2, inter=512))) == 0
     assert L.moe_forward_launches(ctypes.byref(gg.make_config(T=4, d=100, E=8, k=2, inter=512))) == -1

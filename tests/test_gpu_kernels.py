@@ -116,9 +116,15 @@ def test_router_topk(name, T, renorm):
                                            (70, 1024, 33, 3, torch.bfloat16, torch.bfloat16),
                                            (129, 512, 64, 8, torch.float32, torch.bfloat16),
                                            (513, 256, 8, 2, torch.bfloat16, torch.float32),
-                                           (1, 8, 7, 7, torch.float32, torch.float32)])
+                                           (1, 8, 7, 7, torch.float32, torch.float32),
+                                           (3, 8, 4, 2, torch.bfloat16, torch.bfloat16),
+                                           (200, 2048, 100, 6, torch.bfloat16, torch.bfloat16),
+                                           (20000, 512, 256, 8, torch.bfloat16, torch.bfloat16),
+                                           (20000, 256, 8, 2, torch.bfloat16, torch.bfloat16)])
 def test_router_ragged_shapes(T, d, E, k, xdt, wdt):
-    # ragged d, E not a power of two, mixed operand types (E <= 16 runs the one-launch router)
+    # ragged d, E not a power of two, mixed operand types; bf16 operands with
+    # E <= 256 and k <= 8 run the tensor-core router (one cluster of up to 8
+    # CTAs per 128 tokens; a single CTA per tile once 128-token tiles fill the SMs)
     g = torch.Generator(device=DEV).manual_seed(T + d + E)
     x = torch.randn((T, d), device=DEV, generator=g).to(xdt)
     W = (torch.randn((E, d), device=DEV, generator=g) * 0.05).to(wdt)
