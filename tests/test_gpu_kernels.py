@@ -252,6 +252,13 @@ GEMM_CASES = [
     ([640, 641, 384, 0, 1000, 1153, 257], 384, 256, gg.EPI_SILU_GATE, torch.bfloat16),
     # fp32 output on CTA pairs, last tiles of 76 and 30 rows (128-row pair MMAs)
     ([1100, 30], 256, 128, gg.EPI_NONE, torch.float32),
+    # 320..512 rows per group on average: the single-CTA 128x256 kernel (64-row MMA for short tails)
+    ([400, 350, 0, 700, 333], 256, 512, gg.EPI_NONE, torch.bfloat16),
+    ([340, 512, 330], 256, 384, gg.EPI_SILU_GATE, torch.bfloat16),
+    # fine-grained groups: 128-row tiles and 64-row MMAs for short last tiles (1..64 rows)
+    ([144, 150, 139, 0, 256, 257, 511, 300], 256, 256, gg.EPI_SILU_GATE, torch.bfloat16),
+    ([1, 2, 300, 40], 128, 128, gg.EPI_NONE, torch.bfloat16),
+    ([17, 33, 49, 65, 81, 97, 113, 129, 145], 128, 1024, gg.EPI_NONE, torch.bfloat16),
     # a few tokens per group (fewer than 32 rows per group on average): the weights take the
     # MMA's 128-row side (swap-AB), tokens the 32-wide side
     ([1, 0, 3, 2, 5, 33, 0, 1, 0, 7, 64, 1], 256, 128, gg.EPI_NONE, torch.bfloat16),
