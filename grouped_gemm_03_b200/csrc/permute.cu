@@ -74,8 +74,17 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, 
   const int e = threadIdx.x / tpe, c = threadIdx.x % tpe;
   const bool active = e < E;
   const int b0 = c * chunk, b1 = min(nblk, b0 + chunk);
+  // up to 32 blocks per thread (E >= 32 with up to 1024 token blocks, or fewer
+  // experts): the counts stay in registers, one round trip to read them all
+  const bool held = chunk <= 32;
+  int held_v[32];
   int local = 0;
-  if (active) {
+  if (active && held) {
+#pragma unroll
+    for (int u = 0; u < 32; ++u) held_v[u] = b0 + u < b1 ? base[static_cast<size_t>(b0 + u) * E + e] : 0;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) local += held_v[u];
+  } else if (active) {
     for (int b = b0; b < b1; b += kScanBatch) {
       int v[kScanBatch];
 #pragma unroll
@@ -129,7 +138,14 @@ __global__ void __launch_bounds__(1024) scan_kernel(int32_t* __restrict__ base, 
     if (shared) offsets[E + 1] = used + T;
   }
   __syncthreads();
-  if (active) {
+  if (active && held) {
+    int run = s_off[e] + chunk_pre;
+#pragma unroll
+    for (int u = 0; u < 32; ++u) {
+      if (b0 + u < b1) base[static_cast<size_t>(b0 + u) * E + e] = run;
+      run += held_v[u];
+    }
+  } else if (active) {
     int run = s_off[e] + chunk_pre;
     for (int b = b0; b < b1; b += kScanBatch) {
       int v[kScanBatch];
@@ -177,8 +193,11 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   __shared__ int s_pre[kMaxExperts];      // pairs of each expert in the blocks before this one
   __shared__ int s_offx[kMaxExperts + 1];  // exclusive scan of s_tot
   __shared__ int s_wsum[kPermThreads / 32];
+  __shared__ int s_rank[kTokPerBlock * kMaxTopK];  // pair p's rank among the block's earlier pairs of its expert
+  __shared__ int s_cnt[kMaxExperts];               // pairs per expert ranked so far
   const bool fused = a.fuse_scan;
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) s_idx[p] = a.idx[static_cast<size_t>(t0) * k + p];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
   if (fused) {
     for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_pre[e] = 0;
     __syncthreads();
@@ -233,13 +252,31 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
     s_used = a.offsets[E];
   }
   __syncthreads();
+  if (threadIdx.x < 32) {
+    // ranks in pair order (token order: a token's experts are distinct), 32
+    // pairs at a time: lanes holding the same expert find each other with a
+    // match; the highest of them advances the expert's count
+    const int lane = threadIdx.x;
+    for (int p0 = 0; p0 < nt * k; p0 += 32) {
+      const int p = p0 + lane;
+      const bool in = p < nt * k;
+      const int e = in ? s_idx[p] : -1;
+      const bool valid = in && e >= 0 && e < E;
+      const unsigned m = __match_any_sync(0xffffffffu, valid ? e : -2 - lane);
+      const int prior = valid ? s_cnt[e] : 0;
+      __syncwarp();
+      if (valid && (m >> lane) == 1u) s_cnt[e] = prior + __popc(m);
+      __syncwarp();
+      if (in) s_rank[p] = prior + __popc(m & ((1u << lane) - 1u));
+    }
+  }
+  __syncthreads();
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) {
     const int tl = p / k, j = p % k;
     const int e = s_idx[p];
     int row = 0;
     if (e >= 0 && e < E) {
-      int rank = 0;
-      for (int q = 0; q < tl * k; ++q) rank += (s_idx[q] == e);
+      const int rank = s_rank[p];
       const int off_e = fused ? s_offx[e] : a.offsets[e];
       row = (fused ? off_e + s_pre[e] : a.block_base[static_cast<size_t>(b) * E + e]) + rank;
       // past the expert's capacity: the pair overflows and gets no row
