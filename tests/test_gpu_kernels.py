@@ -120,7 +120,13 @@ def test_router_topk(name, T, renorm):
                                            (3, 8, 4, 2, torch.bfloat16, torch.bfloat16),
                                            (200, 2048, 100, 6, torch.bfloat16, torch.bfloat16),
                                            (20000, 512, 256, 8, torch.bfloat16, torch.bfloat16),
-                                           (20000, 256, 8, 2, torch.bfloat16, torch.bfloat16)])
+                                           (20000, 256, 8, 2, torch.bfloat16, torch.bfloat16),
+                                           # bf16 outside the tensor-core router's range: E > 256 (split-K
+                                           # logits + selection kernel), k > 8 with E > 16 (SIMT logits +
+                                           # selection), k > 8 with E <= 16 (the SIMT one-launch router)
+                                           (600, 1024, 300, 6, torch.bfloat16, torch.bfloat16),
+                                           (200, 512, 64, 12, torch.bfloat16, torch.bfloat16),
+                                           (300, 512, 16, 10, torch.bfloat16, torch.bfloat16)])
 def test_router_ragged_shapes(T, d, E, k, xdt, wdt):
     # ragged d, E not a power of two, mixed operand types; bf16 operands with
     # E <= 256 and k <= 8 run the tensor-core router (one cluster of up to 8
