@@ -98,7 +98,9 @@ L2_NOTE = "flushed between timed steps (2x L2 buffer rewritten then read back, o
 
 def config_block(s):
     return {"workload": workload_desc(s), "tokens_per_step": s.T, "seed": 1234, "l2": L2_NOTE,
-            "parallelism": "replicas (one independent layer per GPU)"}
+            "parallelism": "replicas (one independent layer per GPU)",
+            "kernels_note": "kernels.<stage>.us: inside whole forwards, an event before each kernel; "
+                            "kernels.<stage>.isolated: " + ISOLATED_NOTE}
 
 
 def host_cpu():
@@ -267,6 +269,78 @@ def time_marked(gg, cfg, inp, weights, out, counts, ws, steps, flush, stream):
         for i, n in enumerate(STAGES):
             per[n].append(evs[i].elapsed_time(evs[i + 1]))
     return {n: float(np.mean(v)) for n, v in per.items()}
+
+
+ISOLATED_HOLD_CYCLES = 8_000_000  # ~4 ms spin: every launch of the run is enqueued before it ends
+ISOLATED_NOTE = ("the stage's own launches back to back through the library's entry point (moe_router_topk, "
+                 "moe_permute, moe_combine), queued behind a spin kernel, each on its own copy of the "
+                 "stage's input (copies totalling >= 2x L2, so every launch reads HBM); one event pair "
+                 "over all launches")
+
+
+def rotating_copies(t, dev, at_least=2):
+    """Copies of `t` whose total size is at least twice the L2 cache (at most 16)."""
+    l2 = torch.cuda.get_device_properties(dev).L2_cache_size
+    nbytes = t.numel() * t.element_size()
+    n = int(min(16, max(at_least, -(-2 * l2 // max(nbytes, 1)))))
+    return [t.clone() for _ in range(n)]
+
+
+def time_back_to_back(fn, reps, flush, stream):
+    """Device time per call of fn(i), i = 0..reps-1, launched back to back."""
+    for i in range(2):
+        fn(i)
+    torch.cuda.synchronize()
+    flush()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda._sleep(ISOLATED_HOLD_CYCLES)
+    a.record(stream)
+    for i in range(reps):
+        fn(i)
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b) / reps
+
+
+def time_isolated(gg, s, inp, alg, dev, flush, stream, reps=16):
+    """Per-launch device time of the router, permute and combine stages on their own
+    (the in-forward breakdown puts an event between kernels, which also times each
+    launch's latency; here consecutive launches overlap as they do in the forward)."""
+    shared = bool(s.shared_inter)
+    xs = rotating_copies(inp["x"], dev)
+    rws = torch.empty(gg.lib().moe_router_workspace_size(s.T, s.E), dtype=torch.uint8, device=dev)
+    pws = torch.empty(gg.lib().moe_permute_workspace_size(s.T, s.E), dtype=torch.uint8, device=dev)
+    out = {}
+
+    def router(i):
+        return gg.router_topk(xs[i % len(xs)], inp["W_r"], s.k, bias=inp["bias"], renormalize=s.renormalize,
+                              ws=rws)
+
+    out["router"] = time_back_to_back(router, reps, flush, stream)
+    idx, w = router(0)
+
+    def permute(i):
+        return gg.permute(xs[i % len(xs)], idx, s.E, append_shared=shared, fp8=s.fp8, mx=s.mx, ws=pws)
+
+    if not s.gather:  # (with the gather flag the forward's permute writes only the plan)
+        out["permute"] = time_back_to_back(permute, reps, flush, stream)
+    plan = permute(0)
+    rows = plan["row_to_token"].numel()
+    Y = torch.randn((rows, s.d), device=dev).to(torch.bfloat16)
+    Ys = rotating_copies(Y, dev)
+    del Y, xs
+    o = torch.empty((s.T, s.d), dtype=torch.bfloat16 if s.x_dtype != "f32" else torch.float32, device=dev)
+
+    def combine(i):
+        gg.combine(Ys[i % len(Ys)], plan["token_to_row"], w, shared, out_dtype=o.dtype, out=o)
+
+    out["combine"] = time_back_to_back(combine, reps, flush, stream)
+    del Ys
+    torch.cuda.empty_cache()
+    res = {}
+    for name, t_ms in out.items():
+        res[name] = {"us": round(t_ms * 1e3, 2), "gbs": round(alg[name]["bytes"] / (t_ms * 1e-3) / 1e9, 1)}
+    return res
 
 
 def traffic_from_profile(workload, stage, kernel_src_hash):
@@ -510,6 +584,9 @@ def measure_layer(gg, s, steps, warmup, world, dev, flush, seed, graph=True, e2e
             e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
         e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
         kern[name] = e
+    iso = time_isolated(gg, s, inp, alg, dev, flush, stream)
+    for name, e in iso.items():
+        kern[name]["isolated"] = e
     r.update(kernels=kern, counts=c, alg=alg, inp=inp)
     return r
 
@@ -522,6 +599,10 @@ def layer_report(s, r, peaks, peak_kind, world):
     gemm_tf = s.gemm_flops() / (gemm_us * 1e-6) / 1e12
     tensor_peak = float(peaks["bf16_tflops"]) * (2.0 if s.fp8 else 1.0)
     c = r["counts"]
+    hbm = float(peaks["hbm_gbs"])
+    for e in r["kernels"].values():
+        if "isolated" in e:
+            e["isolated"]["frac_of_hbm"] = round(e["isolated"]["gbs"] / hbm, 4)
     rep = {"workload": workload_desc(s), "tokens_per_step": T,
            "dtype": ("mx-e4m3" if s.mx else "e4m3") if s.fp8 else "bf16",
            "ms_per_step": round(r["ms"], 4), "value": round(job_tokens_per_s(T, world, r["ms"]), 1),
@@ -635,9 +716,13 @@ def router_micro_shape(overrides):
     return tuple(overrides.get(key, ROUTER_MICRO[key]) for key in ("N", "E", "k"))
 
 
+ROUTER_MICRO_L2 = ("inputs larger than L2: each step reads its own copy of the logits, the copies together "
+                   ">= 2x L2; the steps run back to back between one pair of events")
+
+
 def router_micro_desc(N, E, k):
     return {"workload": f"router_micro: N={N} tokens, E={E} experts, top-{k}, fp16 logits ~ N(0,1)",
-            "tokens_per_step": N, "seed": 1234, "l2": L2_NOTE}
+            "tokens_per_step": N, "seed": 1234, "l2": ROUTER_MICRO_L2}
 
 
 def measure_router_micro(gg, steps, warmup, world, rank, dev, flush, overrides):
@@ -648,14 +733,25 @@ def measure_router_micro(gg, steps, warmup, world, rank, dev, flush, overrides):
     idx = torch.empty((N, k), dtype=torch.int32, device=dev)
     w = torch.empty((N, k), dtype=torch.float32, device=dev)
 
+    copies = rotating_copies(logits, dev)  # the steps' inputs together exceed twice the L2 size
+
+    def step_i(i):
+        gg.topk_logits(copies[i % len(copies)], k, out_idx=idx, out_w=w)
+
+    for i in range(warmup):
+        step_i(i)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(dev) as clk:
+        # each bracket times exactly `steps` steps, one launch each on the next copy
+        times = [time_back_to_back(step_i, steps, flush, stream) for _ in range(8)]
+    ms = max_over_ranks(float(np.mean(times)), world, dev)
+    del copies
+
     def step():
         gg.topk_logits(logits, k, out_idx=idx, out_w=w)
 
-    if world > 1:
-        torch.distributed.barrier()
-    with ClockSampler(dev) as clk:
-        times = time_steps(step, steps, warmup, flush, stream)
-    ms = max_over_ranks(float(np.mean(times)), world, dev)
     lh = logits.cpu().pin_memory()
     ih = torch.empty((N, k), dtype=torch.int32).pin_memory()
     wh = torch.empty((N, k), dtype=torch.float32).pin_memory()

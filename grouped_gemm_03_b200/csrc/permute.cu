@@ -199,13 +199,46 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
   for (int p = threadIdx.x; p < nt * k; p += blockDim.x) s_idx[p] = a.idx[static_cast<size_t>(t0) * k + p];
   for (int e = threadIdx.x; e < E; e += blockDim.x) s_cnt[e] = 0;
   if (fused) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x) s_tot[e] = s_pre[e] = 0;
-    __syncthreads();
+    // the histogram is cnt[b'][e] at b' * E + e.  P parts per expert each sum
+    // every P-th block (no atomics, a fixed order); P = 1 when E >= threads
     const int nblk = gridDim.x;
-    for (int i = threadIdx.x; i < nblk * E; i += blockDim.x) {
-      const int c = a.block_base[i];  // the histogram: cnt[b'][e] at b' * E + e
-      atomicAdd(&s_tot[i % E], c);
-      if (i / E < b) atomicAdd(&s_pre[i % E], c);
+    const int P = E < static_cast<int>(blockDim.x) ? static_cast<int>(blockDim.x) / E : 1;
+    if (P > 1) {
+      int* s_part_tot = s_rank;  // [P][E] <= threads entries (free until the ranks are taken)
+      int* s_part_pre = s_rank + blockDim.x;
+      const int e = threadIdx.x % E, part = threadIdx.x / E;
+      if (part < P) {
+        int tot = 0, pre = 0;
+        for (int b2 = part; b2 < nblk; b2 += P) {
+          const int c = a.block_base[static_cast<size_t>(b2) * E + e];
+          tot += c;
+          pre += b2 < b ? c : 0;
+        }
+        s_part_tot[part * E + e] = tot;
+        s_part_pre[part * E + e] = pre;
+      }
+      __syncthreads();
+      for (int e2 = threadIdx.x; e2 < E; e2 += blockDim.x) {
+        int tot = 0, pre = 0;
+        for (int q = 0; q < P; ++q) {
+          tot += s_part_tot[q * E + e2];
+          pre += s_part_pre[q * E + e2];
+        }
+        s_tot[e2] = tot;
+        s_pre[e2] = pre;
+      }
+    } else {
+      for (int e2 = threadIdx.x; e2 < E; e2 += blockDim.x) {
+        int tot = 0, pre = 0;
+#pragma unroll 4
+        for (int b2 = 0; b2 < nblk; ++b2) {
+          const int c = a.block_base[static_cast<size_t>(b2) * E + e2];
+          tot += c;
+          pre += b2 < b ? c : 0;
+        }
+        s_tot[e2] = tot;
+        s_pre[e2] = pre;
+      }
     }
     __syncthreads();
     // kept rows per expert, then their exclusive scan (each thread 4 consecutive experts)
