@@ -347,14 +347,20 @@ __global__ void __launch_bounds__(kPermThreads) scatter_kernel(PermuteArgs a) {
     __nv_bfloat16* xp = static_cast<__nv_bfloat16*>(a.xp);
     const int nvec = cw / 8;
     const int items = nt * nvec;
+    // a full column block has 64 vectors per token: shift and mask instead of dividing
+    const bool pow2 = nvec == kScatterCols / 8;
+    constexpr int kVecShift = 6;
+    static_assert(kScatterCols / 8 == 1 << kVecShift, "vectors per full column block");
     for (int base = threadIdx.x; base < items; base += U * blockDim.x) {
       uint4 v[U];
       int tl[U], c[U];
 #pragma unroll
       for (int u = 0; u < U; ++u) {
         const int it = base + u * blockDim.x;
-        tl[u] = it < items ? it / nvec : -1;
-        c[u] = it < items ? cbeg + (it % nvec) * 8 : 0;
+        const int q = pow2 ? it >> kVecShift : it / nvec;
+        const int rmd = pow2 ? it & ((1 << kVecShift) - 1) : it - q * nvec;
+        tl[u] = it < items ? q : -1;
+        c[u] = it < items ? cbeg + rmd * 8 : 0;
         if (tl[u] < 0) continue;
         const XT* src = x + static_cast<size_t>(t0 + tl[u]) * d + c[u];
         if constexpr (sizeof(XT) == 2) {
