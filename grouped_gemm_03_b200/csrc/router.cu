@@ -2,8 +2,10 @@
 //
 // "MegaMoE math model -> DeepGEMM source walk-through" §2.1 (p = Softmax(W_r x_t),
 // keep the k best) and "Dense GEMM -> GroupedGEMM -> TP MoE" §4.2 (route_tokens).
-// Up to 16 experts: one launch, router_fused_kernel (below), which streams
-// x once and keeps every logit on chip.  Otherwise two launches:
+// bf16 x and W_r with E <= 256 and k <= 8 take the one-launch tensor-core
+// router (router_tc.cu).  This file holds the other paths.  Up to 16
+// experts: one launch, router_fused_kernel (below), which streams x once and
+// keeps every logit on chip.  Otherwise two launches:
 //   logits  either the grouped-GEMM kernel on the tensor cores (bf16, large
 //           E and d: the logits GEMM is then near the compute ridge), split
 //           along K into fp32 partial products, or a SIMT kernel that keeps

@@ -84,6 +84,25 @@ def test_topk_logits_ties_take_lower_index():
     assert (idx1.cpu() == torch.tensor([0, 1], dtype=torch.int32)).all()
 
 
+@pytest.mark.parametrize("dtype,E", [(torch.float16, 64), (torch.bfloat16, 128), (torch.float32, 40)])
+def test_topk_signed_zeros_tie(dtype, E):
+    # -0 and +0 compare equal, so they tie and the lower expert comes first,
+    # whichever sign it carries (rows of -1, -0, +0 and -2: the top picks are zeros)
+    g = np.random.default_rng(E)
+    vals = np.array([-1.0, -0.0, 0.0, -2.0])
+    l = vals[g.integers(0, 4, size=(700, E))]
+    l[:, 0] = -0.0  # every row has zeros of both signs
+    l[:, 1] = 0.0
+    lt = torch.tensor(l, dtype=dtype, device=DEV)
+    for k in (1, 3, 6):
+        idx, w = gg.topk_logits(lt, k)
+        torch.cuda.synchronize()
+        want = oracle.topk_select(l, k)
+        assert np.array_equal(idx.cpu().numpy(), want)
+        np.testing.assert_allclose(w.cpu().numpy(), oracle.gate_weights(oracle.softmax(l), want), rtol=2e-6,
+                                   atol=1e-7)
+
+
 def test_topk_k1_renormalised_is_one():
     l = make_router_logits(1000, 16, seed=2, device=DEV, dtype=torch.float32)
     _, w = gg.topk_logits(l, 1, renormalize=True)
@@ -120,6 +139,7 @@ def test_router_topk(name, T, renorm):
                                            (3, 8, 4, 2, torch.bfloat16, torch.bfloat16),
                                            (200, 2048, 100, 6, torch.bfloat16, torch.bfloat16),
                                            (20000, 512, 256, 8, torch.bfloat16, torch.bfloat16),
+                                           (6000, 512, 32, 4, torch.bfloat16, torch.bfloat16),  # 2-CTA clusters
                                            (20000, 256, 8, 2, torch.bfloat16, torch.bfloat16),
                                            # bf16 outside the tensor-core router's range: E > 256 (split-K
                                            # logits + selection kernel), k > 8 with E > 16 (SIMT logits +
