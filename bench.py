@@ -554,6 +554,25 @@ def measure_layer(gg, s, steps, warmup, world, dev, flush, seed, graph=True, e2e
         raise RuntimeError(f"{s.name}: device status {status}")
     r = dict(ms=max_over_ranks(float(np.mean(times)), world, dev), clocks=clk.summary())
 
+    # the per-kernel breakdown right after the headline steps (same clock and
+    # thermal state; the two-stream e2e phase below loads the GPU harder)
+    with ClockSampler(dev) as kclk:
+        kt = time_marked(gg, cfg, inp, weights, out, counts, ws, max(3, steps // 2), flush, stream)
+    c = counts.cpu().numpy()
+    alg = algorithmic(s, c)
+    kern = {}
+    for name, t_ms in kt.items():
+        a = alg[name]
+        e = {"us": round(t_ms * 1e3, 2)}
+        if "flops" in a:
+            e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
+        e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
+        kern[name] = e
+    iso = time_isolated(gg, s, inp, alg, dev, flush, stream)
+    for name, e in iso.items():
+        kern[name]["isolated"] = e
+    r["kernels_clocks"] = kclk.summary()
+
     if graph:  # the same forward replayed from a CUDA graph (one launch of the whole layer)
         gstream = torch.cuda.Stream()
         gstream.wait_stream(stream)
@@ -608,20 +627,6 @@ def measure_layer(gg, s, steps, warmup, world, dev, flush, seed, graph=True, e2e
         r["h2d"] = xh[0].numel() * xh[0].element_size()
         r["d2h"] = oh[0].numel() * oh[0].element_size()
 
-    kt = time_marked(gg, cfg, inp, weights, out, counts, ws, max(3, steps // 2), flush, stream)
-    c = counts.cpu().numpy()
-    alg = algorithmic(s, c)
-    kern = {}
-    for name, t_ms in kt.items():
-        a = alg[name]
-        e = {"us": round(t_ms * 1e3, 2)}
-        if "flops" in a:
-            e["tflops"] = round(a["flops"] / (t_ms * 1e-3) / 1e12, 1)
-        e["gbs"] = round(a["bytes"] / (t_ms * 1e-3) / 1e9, 1)
-        kern[name] = e
-    iso = time_isolated(gg, s, inp, alg, dev, flush, stream)
-    for name, e in iso.items():
-        kern[name]["isolated"] = e
     r.update(kernels=kern, counts=c, alg=alg, inp=inp)
     return r
 
@@ -644,7 +649,7 @@ def layer_report(s, r, peaks, peak_kind, world):
            "unit": "tokens/s",
            # grouped-GEMM FLOP over the two GEMM kernels' own time, against the dense tensor peak
            "gemm_tflops": round(gemm_tf, 1), "gemm_frac_of_peak": round(gemm_tf / tensor_peak, 4),
-           "roofline": roof, "kernels": r["kernels"], "clocks": r["clocks"],
+           "roofline": roof, "kernels": r["kernels"], "clocks": r["clocks"], "kernels_clocks": r["kernels_clocks"],
            "expert_counts": {"min": int(c.min()), "max": int(c.max()), "mean": float(c.mean()),
                              "zeros": int((c == 0).sum())}}
     if "graph_ms" in r:
@@ -716,7 +721,8 @@ def main():
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": rep["dtype"],
             "data": "synthetic (seeded N(0,1) activations, N(0,0.02) weights)", "config": config_block(s),
             "gemm_tflops": rep["gemm_tflops"], "gemm_frac_of_peak": rep["gemm_frac_of_peak"],
-            "roofline": rep["roofline"], "kernels": rep["kernels"], "e2e": rep["e2e"], "graph": rep["graph"],
+            "roofline": rep["roofline"], "kernels": rep["kernels"], "kernels_clocks": rep["kernels_clocks"],
+            "e2e": rep["e2e"], "graph": rep["graph"],
             "gpu_launches": gg.forward_launches(make_cfg(gg, s)) * args.steps, "clocks": rep["clocks"],
             "expert_counts": rep["expert_counts"]}
         if rank == 0 and world == 1 and not args.no_cpu_baseline:
