@@ -64,7 +64,9 @@ struct Tile {
   static constexpr int B_BYTES = MMA_N * 128;
   static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
   static constexpr int TABLE_BYTES = 2 * (kMaxGroups + 2) * 4;
-  static constexpr int OUT_WARP = kStageOut ? 8192 : 0;
+  // one 4 KiB box buffer per epilogue warp: with it, four operand stages of
+  // 48 KiB still fit (two buffers would leave three)
+  static constexpr int OUT_WARP = kStageOut ? 4096 : 0;
   static constexpr int STAGES_RAW = (kSmemBudget - 2048 - TABLE_BYTES - 512 - 4 * OUT_WARP) / STAGE_BYTES;
   static constexpr int STAGES = STAGES_RAW > 8 ? 8 : STAGES_RAW;
   static constexpr int TMEM_COLS = 2 * MMA_N;
@@ -429,9 +431,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       const uint32_t tacc = lane_base + acc * MMA_N;
       if constexpr (OUT == 0) {
         // bf16 output in 64-column boxes.  A warp whose 32 rows all belong to
-        // the group stages each box (128-byte swizzled, two buffers in turn)
-        // and writes it with a bulk tensor store; a slice crossing the
-        // group's end stores its valid rows directly.
+        // the group stages each box (128-byte swizzled) in its buffer and
+        // writes it with a bulk tensor store; a slice crossing the group's
+        // end stores its valid rows directly.
         const int r0 = tc.mb * BM + q * 32;
         // (the gated output, half as wide, keeps the operand stage instead: direct stores)
         const bool slice_full = L::OUT_WARP > 0 && !half && r0 + 32 <= m_g;
@@ -467,8 +469,14 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
           }
           if (slice_full) {
-            uint8_t* buf = s_out + (b & 1) * 4096;
-            if (lane == 0) ptx::bulk_wait_read_allow1();  // the store that used this buffer has read it
+            constexpr int kBufs = L::OUT_WARP / 4096 > 0 ? L::OUT_WARP / 4096 : 1;
+            uint8_t* buf = s_out + (b % kBufs) * 4096;
+            if (lane == 0) {  // the store that used this buffer has read it
+              if constexpr (kBufs > 1)
+                ptx::bulk_wait_read_allow1();
+              else
+                ptx::bulk_wait_read_all();
+            }
             __syncwarp();
 #pragma unroll
             for (int c = 0; c < 8; ++c)
