@@ -116,13 +116,18 @@ int moe_read_device_status(const void* ws, void* stream, int* status);
  * p_i = Softmax(W_r x_t)_i; "Dense GEMM -> GroupedGEMM -> TP MoE" §4.2
  * route_tokens: F.linear -> softmax -> topk).
  *   x        [T, d]  x_dtype (MOE_F32 | MOE_BF16)
- *   W_r      [E, d]  w_dtype (MOE_F32 | MOE_BF16); fp32 W_r requires fp32 x
+ *   W_r      [E, d]  w_dtype (MOE_F32 | MOE_BF16)
  *   bias     [E] fp32 added to the logits before the softmax, or NULL
  *   logits_out [T, E] fp32, or NULL (the logits every later step depends on)
  *   topk_idx [T, k] int32: selected experts, descending logit, ties -> lower index
+ *            (-0 and +0 are equal logits)
  *   topk_w   [T, k] fp32: p of the selected experts (renormalised if asked)
  *   ws       scratch of moe_router_workspace_size(T, E) bytes (status word + logits)
- * 1 <= k <= min(E, 32), E <= 1024, d % 8 == 0. */
+ * 1 <= k <= min(E, 32), E <= 1024, d % 8 == 0; x and W_r 16-byte aligned.
+ * bf16 x and W_r with E <= 256 and k <= 8 run as one launch (tensor-core
+ * logits, K split over a thread-block cluster, softmax and top-k on chip);
+ * the logits are then summed over the K slices in a fixed order, so they do
+ * not vary from run to run. */
 size_t moe_router_workspace_size(int T, int E);
 int moe_router_topk(const void* x, int x_dtype, const void* W_r, int w_dtype, const float* bias, int T,
                     int d, int E, int k, int renormalize, float* logits_out, int32_t* topk_idx,
