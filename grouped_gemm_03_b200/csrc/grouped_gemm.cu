@@ -801,7 +801,8 @@ template <int EPI, int OUT>
 __global__ void __launch_bounds__(kThreads, 1)
     gg_bf16_pair_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                         const __grid_constant__ CUtensorMap tmBx, const __grid_constant__ CUtensorMap tmB64,
-                        const __grid_constant__ CUtensorMap tmBx64, const Params p) {
+                        const __grid_constant__ CUtensorMap tmBx64, const __grid_constant__ CUtensorMap tmA64,
+                        const Params p) {
   pdl_wait();  // the preceding kernel on the stream is complete and visible
   pdl_launch_dependents();
   constexpr int MMA_N = 256;
@@ -926,8 +927,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           const uint32_t fb = ptx::map_to_rank(ptx::smem_u32(&full[stage]), 0);
-          if (leader) ptx::mbar_arrive_expect_tx(&full[stage], 2 * STAGE_BYTES);
-          ptx::tma_load_2d_pair(sA + stage * A_BYTES, &tmA, fb, kb * 64, a_row);
+          // a half tile's MMA reads 64 A rows per CTA: load just those (64-row box)
+          if (leader) ptx::mbar_arrive_expect_tx(&full[stage], half ? 2 * (A_BYTES / 2 + B_BYTES) : 2 * STAGE_BYTES);
+          ptx::tma_load_2d_pair(sA + stage * A_BYTES, half ? &tmA64 : &tmA, fb, kb * 64, a_row);
           if (EPI && half) {
             ptx::tma_load_2d_pair(sB + stage * B_BYTES, mB64, fb, kb * 64, hrow);
             ptx::tma_load_2d_pair(sB + stage * B_BYTES + 64 * 128, mB64, fb, kb * 64, hrow + p.N);
@@ -2256,9 +2258,11 @@ int run_bf16_pair(const GemmArgs& a, cudaStream_t s) {
   if (!make_map(&mB, a.B, 2, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, 128)) return MOE_ERR_CUDA;
   if (!make_map(&mBx, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, 128)) return MOE_ERR_CUDA;
   // 64-row boxes for the gated half tiles (64 gate rows, then the 64 matching up rows)
-  CUtensorMap mB64, mBx64;
+  CUtensorMap mB64, mBx64, mA64;
   if (!make_map(&mB64, a.B, 2, static_cast<uint64_t>(a.G > 0 ? a.G : 1) * nb_rows, a.K, 64)) return MOE_ERR_CUDA;
   if (!make_map(&mBx64, a.has_extra ? a.B_extra : a.B, 2, nb_rows, a.K, 64)) return MOE_ERR_CUDA;
+  // 64-row A boxes for the half tiles (64 rows per CTA)
+  if (!make_map(&mA64, a.A, 2, static_cast<uint64_t>(a.rows > 0 ? a.rows : 1), a.K, 64)) return MOE_ERR_CUDA;
   static int clusters[64] = {};
   int dev = 0;
   MOE_CUDA_CHECK(cudaGetDevice(&dev));
@@ -2299,7 +2303,7 @@ int run_bf16_pair(const GemmArgs& a, cudaStream_t s) {
   p.ksplit = 1;
   p.C = a.C;
   p.status = a.status;
-  MOE_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gg_bf16_pair_kernel<EPI, OUT>, mA, mB, mBx, mB64, mBx64, p));
+  MOE_CUDA_CHECK(cudaLaunchKernelEx(&cfg, gg_bf16_pair_kernel<EPI, OUT>, mA, mB, mBx, mB64, mBx64, mA64, p));
   return MOE_OK;
 }
 
